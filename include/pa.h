@@ -1,0 +1,216 @@
+/*
+ * pa.h -- paged KV-cache attention for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The hot path of a paged-KV serving engine's attention layer:
+ *
+ *   1. pa_reshape_and_cache  -- scatter this step's new K/V rows into 16-token
+ *      physical blocks through a per-token slot mapping
+ *      ("vLLM 架构源码解析 | 第 1 篇" §3.3.3: reshape_and_cache(k, v, kv_cache,
+ *      slot_mapping) runs before paged_attention in every attention layer).
+ *   2. pa_decode             -- one query row per request attends to its
+ *      cached context through its block-table row
+ *      ("vLLM 深度拆解：当 KV Cache 学会「分页」" §3.3 and §6.2;
+ *      "vLLM 架构源码解析" §3.3.3 paged_attention(q, kv_cache, block_tables,
+ *      context_lens)).
+ *   3. pa_varlen             -- the scheduler's mixed batch: decode rows next
+ *      to causal chunked-prefill chunks whose earlier context is cached
+ *      ("vLLM 深度拆解" §4.3 chunked prefill; "vLLM 架构源码解析" §3.2 unified
+ *      token budget and §3.3.2 query_start_loc / positions / seq_lens).
+ *
+ * Attention is softmax(q . K^T * scale) . V ("vLLM 深度拆解" §2.2).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer argument except the returned strings is a DEVICE pointer on
+ *   the current CUDA device, owned by the caller.  The library keeps no
+ *   pointer after the call returns and allocates no device memory: scratch
+ *   space is the caller's `workspace`, sized by the *_workspace_size query.
+ * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *   NULL = the legacy default stream).  No call synchronises, except
+ *   pa_get_device_error.  Order pa_reshape_and_cache before the attention call
+ *   that must see its rows on the same stream.
+ * - All tensors are dense and row-major with the shapes given below; base
+ *   pointers must be 16-byte aligned.
+ * - KV cache layout: k_cache and v_cache are each
+ *   [num_blocks, num_kv_heads, block_size, head_dim].  Each (block, head)
+ *   holds block_size consecutive tokens of one request as a contiguous
+ *   block_size x head_dim row-major tile.  (The pages print two layouts,
+ *   [blocks, heads, head_size, block_size] in "vLLM 深度拆解" §6.2 and
+ *   [blocks, block_size, d_k] in "vLLM 架构源码解析" §4.2; this one keeps a
+ *   token's head_dim values contiguous so that one 16-byte load carries eight
+ *   16-bit values of one token.)
+ * - block_size must be 16 ("vLLM 架构源码解析" §1.1 and §5.1, the default).
+ * - block_tables is int32 [num_seqs, block_table_stride]: entry [r][j] is the
+ *   physical block holding tokens j*16 .. j*16+15 of request r
+ *   ("vLLM 深度拆解" §3.3: block_tables[seq_id * stride + block_idx]).
+ *   Entries past ceil(len/16) are never read.
+ * - Grouped-query attention: query head h reads KV head
+ *   h / (num_q_heads / num_kv_heads).  num_q_heads % num_kv_heads == 0.
+ * - head_dim is 64 or 128.  dtype: PA_F32, PA_BF16 or PA_F16; q, k, v, the
+ *   caches and out all have that dtype.  Arithmetic is fp32 with one
+ *   round-to-nearest-even conversion of the output.
+ * - Errors: a status other than PA_OK returned by a call means nothing was
+ *   launched (argument checks are done on the host before any launch) or a
+ *   launch failed (PA_ERR_CUDA).  Checks that need device data (a block id
+ *   outside [0, num_blocks), a slot outside the pool, a length above the
+ *   host-given maximum, a bounded wait that ran out) are made inside the
+ *   kernels: the offending access is skipped, the first such event is
+ *   recorded in a per-device error word, and pa_get_device_error reports it.
+ *   No kernel faults, traps or waits without bound on bad metadata.
+ * - Thread safety: calls may be made from several host threads; the device
+ *   error word is shared per device.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* a null/misaligned pointer, a negative size, Hq % Hkv != 0, ... */
+  PA_ERR_UNSUPPORTED = 2,   /* a valid but unimplemented shape: head_dim, block_size, dtype */
+  PA_ERR_WORKSPACE = 3,     /* workspace_bytes below the size query's answer */
+  PA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  PA_ERR_DEVICE_BOUNDS = 5, /* (device) bad metadata: block id, slot or length out of range */
+  PA_ERR_TIMEOUT = 6        /* (device) a bounded wait inside a kernel gave up */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
+
+/*
+ * Kernel family selection, for tests and measurements.  PA_PATH_AUTO picks
+ * the fastest family that supports the shape: the TMA + tensor-core kernel for
+ * 16-bit types, the CUDA-core kernel for fp32, and the tcgen05 (TMEM) tile
+ * kernel for the prefill chunks of pa_varlen.  The other values force one
+ * family; forcing a family that does not support the call's shape makes the
+ * call return PA_ERR_UNSUPPORTED.  The setting is process-wide.
+ */
+typedef enum {
+  PA_PATH_AUTO = 0,
+  PA_PATH_SIMT = 1,     /* CUDA-core kernel, plain vector loads (any dtype) */
+  PA_PATH_MMA = 2,      /* TMA bulk-tensor loads + warp-level bf16/f16 tensor-core MMA */
+  PA_PATH_TCGEN05 = 3   /* as PA_PATH_MMA, with prefill chunks on tcgen05/TMEM tiles */
+} pa_path;
+
+/*
+ * pa_reshape_and_cache -- write this step's new K/V rows into the cache.
+ *
+ * "vLLM 架构源码解析" §3.3.3 (LlamaAttention.forward calls
+ * cache_ops.reshape_and_cache(k, v, kv_cache, slot_mapping) before
+ * paged_attention) and §3.3.2 (_prepare_inputs builds the slot mapping).
+ *
+ *   k, v          [num_tokens, num_kv_heads, head_dim]   this step's rows
+ *   k_cache,      [num_blocks, num_kv_heads, block_size, head_dim], updated
+ *   v_cache         in place
+ *   slot_mapping  int32 [num_tokens]: token t goes to physical block
+ *                 slot/block_size, offset slot%block_size.  slot < 0 marks a
+ *                 padding token: it is skipped.  A slot >= num_blocks *
+ *                 block_size is skipped and recorded as PA_ERR_DEVICE_BOUNDS.
+ *
+ * Bytes are copied exactly.  Two tokens naming the same slot in one call
+ * leave an unspecified one of the two rows.  num_tokens == 0 is a no-op.
+ */
+pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                               const int32_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               void* stream);
+
+/*
+ * Workspace (bytes) pa_decode needs for these sizes.  Includes the split-K
+ * partial results (contexts longer than one 512-token partition are split
+ * and reduced by log-sum-exp) and the schedule.  Returns 0 only for empty
+ * batches.
+ */
+size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                int max_context_len);
+
+/*
+ * pa_decode -- decode attention over the paged cache.
+ *
+ * "vLLM 深度拆解" §3.3 (the block-table walk, padding past context_len
+ * skipped) and §6.2 (the kernel's arguments); "vLLM 架构源码解析" §3.3.3.
+ *
+ *   out           [num_seqs, num_q_heads, head_dim], written
+ *   q             [num_seqs, num_q_heads, head_dim]  one query row per request
+ *   block_tables  int32 [num_seqs, block_table_stride]
+ *   context_lens  int32 [num_seqs]: cached tokens of each request, including
+ *                 the one written this step by pa_reshape_and_cache.  The
+ *                 query attends to tokens 0 .. context_lens[r]-1.  A zero
+ *                 length gives a zero output row.  A length above
+ *                 max_context_len or above block_table_stride*block_size is
+ *                 a device-side bounds error (row left unwritten).
+ *   max_context_len  host-side upper bound on context_lens (sizes the grid
+ *                 and workspace without reading device memory).
+ *   scale         multiplies q.k before the softmax (1/sqrt(head_dim) for
+ *                 the pages' formula).
+ *   workspace     device scratch of at least pa_decode_workspace_size(...)
+ *                 bytes, 256-byte aligned, owned by the caller; its contents
+ *                 are not preserved.  Concurrent calls need separate workspaces.
+ */
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int block_table_stride,
+                    const int32_t* context_lens, int num_seqs, int num_q_heads,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                    int max_context_len, float scale, void* workspace, size_t workspace_bytes,
+                    pa_dtype dtype, void* stream);
+
+/* Workspace (bytes) pa_varlen needs for these sizes. */
+size_t pa_varlen_workspace_size(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,
+                                int head_dim, int max_query_len, int max_seq_len);
+
+/*
+ * pa_varlen -- attention for a mixed scheduler batch.
+ *
+ * "vLLM 架构源码解析" §3.2 (one token budget shared by prefill and decode;
+ * num_new_tokens == 1 is a decode row) and §3.3.2 (query_start_loc is
+ * [0, L1, L1+L2, ...]; positions run from num_computed_tokens);
+ * "vLLM 深度拆解" §4.3 (chunked prefill).
+ *
+ *   out              [total_q, num_q_heads, head_dim], written
+ *   q                [total_q, num_q_heads, head_dim]
+ *   query_start_loc  int32 [num_seqs + 1]: request r owns query rows
+ *                    query_start_loc[r] .. query_start_loc[r+1]-1;
+ *                    query_start_loc[num_seqs] == total_q.
+ *   seq_lens         int32 [num_seqs]: cached plus new tokens of request r
+ *                    (the new rows already written by pa_reshape_and_cache).
+ *   Query row i of request r sits at position seq_lens[r] - q_len_r + i and
+ *   attends causally to keys 0 .. that position.
+ *   max_query_len, max_seq_len  host-side upper bounds.
+ *   workspace        as for pa_decode, sized by pa_varlen_workspace_size.
+ */
+pa_status pa_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int block_table_stride,
+                    const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
+                    int total_q, int max_query_len, int max_seq_len, int num_q_heads,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                    void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream);
+
+/*
+ * Synchronise `stream`, then return and clear the current device's error
+ * word: PA_OK, PA_ERR_DEVICE_BOUNDS or PA_ERR_TIMEOUT (PA_ERR_CUDA if the
+ * synchronisation itself failed).  Details go to pa_last_error_message.
+ */
+pa_status pa_get_device_error(void* stream);
+
+/* Select the kernel family (process-wide).  Returns the previous value. */
+pa_path pa_set_path(pa_path path);
+
+/* Static, human-readable name of a status code. */
+const char* pa_status_string(pa_status status);
+
+/* Detail of the last non-OK status produced on the calling host thread. */
+const char* pa_last_error_message(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */
