@@ -1,0 +1,32 @@
+"""Paged KV-cache attention for NVIDIA B200 (sm_100a).
+
+The hot path of a paged-KV serving engine's attention layer as a C-ABI
+library (``libpa.so``, declared in ``include/pa.h``) with hand-written CUDA
+kernels, and this thin Python binding of it:
+
+* :func:`pa_reshape_and_cache` -- scatter new K/V rows into 16-token blocks;
+* :func:`pa_decode` -- block-table-indirected decode attention (GQA, online
+  softmax, split-K with a log-sum-exp reduce);
+* :func:`pa_varlen` -- mixed batches of decode rows and causal prefill chunks.
+
+PyTorch provides device memory and streams only.  The seeded workload
+generator lives in :mod:`.workload`; byte/flop accounting in :mod:`.accounting`.
+"""
+
+from ._binding import (  # noqa: F401
+    LIBRARY_PATH,
+    PaError,
+    Path,
+    Status,
+    alloc_workspace,
+    lib,
+    pa_decode,
+    pa_decode_workspace_size,
+    pa_get_device_error,
+    pa_reshape_and_cache,
+    pa_set_path,
+    pa_status_string,
+    pa_varlen,
+    pa_varlen_workspace_size,
+    pa_version,
+)

@@ -1,0 +1,469 @@
+// Host side of the C ABI declared in include/pa.h: argument checks, workspace
+// carving, TMA tensor-map encoding, kernel choice and launches.  Every entry
+// point validates on the host before touching the device, returns a status
+// and never synchronises (except pa_get_device_error).
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+
+#include "pa_attn_mma.cuh"
+#include "pa_attn_simt.cuh"
+#include "pa_reshape.cuh"
+#include "pa_sched.cuh"
+
+namespace {
+
+thread_local std::string g_msg;
+std::atomic<int> g_path{PA_PATH_AUTO};
+
+pa_status fail(pa_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+pa_status fail(pa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_msg = buf;
+  return st;
+}
+
+pa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int elem_bytes(pa_dtype dt) { return dt == PA_F32 ? 4 : 2; }
+
+bool valid_dtype(int dt) { return dt == PA_F32 || dt == PA_BF16 || dt == PA_F16; }
+
+int sm_count() {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  cache[dev] = n;
+  return n;
+}
+
+// Set the dynamic shared-memory limit of a kernel and return its occupancy,
+// once per (kernel, device).
+template <typename K>
+cudaError_t prepare(K kernel, int threads, int smem, int* occ) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *occ = it->second;
+    return cudaSuccess;
+  }
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, kernel, threads, smem);
+  if (e != cudaSuccess) return e;
+  if (*occ < 1) return cudaErrorInvalidConfiguration;
+  cache[key] = *occ;
+  return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime, so the
+// library does not link libcuda directly).
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D view [rows][inner] of a 16-bit tensor, box {64, box_rows}, 128 B swizzle.
+pa_status make_map_2d(CUtensorMap* map, const void* base, pa_dtype dt, uint64_t inner,
+                      uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (2d) failed: %d", r);
+  return PA_OK;
+}
+
+// 3-D view [d2][d1][inner] of a 16-bit tensor, box {64, b1, b2}, 128 B swizzle.
+pa_status make_map_3d(CUtensorMap* map, const void* base, pa_dtype dt, uint64_t inner,
+                      uint64_t d1, uint64_t d2, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[3] = {inner, d1, d2};
+  const cuuint64_t strides[2] = {inner * 2, inner * d1 * 2};
+  const cuuint32_t box[3] = {64, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (3d) failed: %d", r);
+  return PA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Attention (decode and varlen share everything below)
+// ---------------------------------------------------------------------------
+struct AttnArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  int table_stride;
+  const int32_t* qsl;  // null for decode
+  const int32_t* seq_lens;
+  int num_seqs, total_q, max_query_len, max_seq_len;
+  int num_q_heads, num_kv_heads, head_dim, block_size, num_blocks;
+  float scale;
+  void* workspace;
+  size_t workspace_bytes;
+  pa_dtype dtype;
+  cudaStream_t stream;
+};
+
+constexpr int kNcw = 4;
+constexpr int kStages = 8;
+
+struct Plan {
+  pa::Shape s;
+  size_t off_part_lse, off_part_o, bytes;
+  long long max_units;
+};
+
+Plan make_plan(int num_seqs, int total_q, int hq, int hkv, int d, int max_len, bool varlen) {
+  Plan p{};
+  pa::Shape& s = p.s;
+  s.num_seqs = num_seqs;
+  s.num_q_heads = hq;
+  s.num_kv_heads = hkv;
+  s.group = hkv > 0 ? hq / hkv : 1;
+  s.gs = s.group < pa::kRows ? s.group : pa::kRows;
+  s.ns = (s.group + pa::kRows - 1) / pa::kRows;
+  s.qpt = varlen ? (pa::kRows / s.gs > 0 ? pa::kRows / s.gs : 1) : 1;
+  s.head_dim = d;
+  s.total_q = total_q;
+  s.p_stride = max_len > 0 ? (max_len + pa::kPart - 1) / pa::kPart : 1;
+  size_t off = align256(static_cast<size_t>(num_seqs + 1) * 4);
+  p.off_part_lse = off;
+  if (s.p_stride > 1) {
+    const size_t slots = static_cast<size_t>(total_q) * hq * s.p_stride;
+    off = align256(off + slots * 4);
+    p.off_part_o = off;
+    off = align256(off + slots * d * 4);
+  } else {
+    p.off_part_o = off;
+  }
+  p.bytes = num_seqs > 0 ? off : 0;
+  const long long items =
+      varlen ? (static_cast<long long>(total_q) + static_cast<long long>(num_seqs) * (s.qpt - 1)) /
+                   s.qpt
+             : num_seqs;
+  p.max_units = items * s.p_stride * hkv * s.ns;
+  return p;
+}
+
+pa_status check_common(const AttnArgs& a) {
+  if (!valid_dtype(a.dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", a.dtype);
+  if (a.num_seqs < 0 || a.total_q < 0 || a.max_query_len < 0 || a.max_seq_len < 0 ||
+      a.num_blocks < 0 || a.table_stride < 0)
+    return fail(PA_ERR_INVALID_ARG, "negative size");
+  if (a.num_q_heads <= 0 || a.num_kv_heads <= 0 || a.num_q_heads % a.num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                a.num_q_heads, a.num_kv_heads);
+  if (a.head_dim != 64 && a.head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", a.head_dim);
+  if (a.block_size != pa::kBlock)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 16)", a.block_size);
+  if (!(std::isfinite(a.scale))) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+  if (static_cast<long long>(a.num_blocks) * a.num_kv_heads * pa::kBlock > 0x7fffffffLL)
+    return fail(PA_ERR_UNSUPPORTED, "pool of %d blocks x %d heads exceeds 2^31 token rows",
+                a.num_blocks, a.num_kv_heads);
+  if (static_cast<long long>(a.total_q) * a.num_q_heads > 0x7fffffffLL)
+    return fail(PA_ERR_UNSUPPORTED, "too many query rows");
+  if (a.total_q == 0 || a.num_seqs == 0) return PA_OK;
+  const void* ptrs[] = {a.out, a.q, a.k_cache, a.v_cache};
+  for (const void* p : ptrs) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(p, 16)) return fail(PA_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  }
+  if (!a.block_tables || !a.seq_lens) return fail(PA_ERR_INVALID_ARG, "null metadata pointer");
+  if (!aligned(a.block_tables, 4) || !aligned(a.seq_lens, 4))
+    return fail(PA_ERR_INVALID_ARG, "metadata pointer not 4-byte aligned");
+  if (a.num_blocks == 0) return fail(PA_ERR_INVALID_ARG, "empty KV pool");
+  if (a.table_stride == 0) return fail(PA_ERR_INVALID_ARG, "block_table_stride is 0");
+  return PA_OK;
+}
+
+template <typename T, int D>
+pa_status launch_simt(const AttnArgs& a, const Plan& p, int* row_start, float* part_lse,
+                      float* part_o) {
+  auto kern = pa::attn_simt_kernel<T, D>;
+  int occ = 0;
+  cudaError_t e = prepare(kern, 128, 0, &occ);
+  if (e != cudaSuccess) return cuda_fail(e, "simt kernel set-up");
+  long long grid = static_cast<long long>(sm_count()) * occ;
+  if (p.max_units < grid) grid = p.max_units;
+  if (grid < 1) grid = 1;
+  kern<<<static_cast<unsigned>(grid), 128, 0, a.stream>>>(
+      p.s, static_cast<T*>(a.out), static_cast<const T*>(a.q), static_cast<const T*>(a.k_cache),
+      static_cast<const T*>(a.v_cache), a.block_tables, a.qsl, a.seq_lens, row_start,
+      static_cast<float>(a.scale * M_LOG2E), part_o, part_lse);
+  return PA_OK;
+}
+
+template <typename T, int D>
+pa_status launch_mma(const AttnArgs& a, const Plan& p, int* row_start, float* part_lse,
+                     float* part_o) {
+  using L = pa::MmaLayout<D, kNcw, kStages>;
+  auto kern = pa::attn_mma_kernel<T, D, kNcw, kStages>;
+  const int threads = (kNcw + 1) * 32;
+  int occ = 0;
+  cudaError_t e = prepare(kern, threads, L::kSmem, &occ);
+  if (e != cudaSuccess) return cuda_fail(e, "mma kernel set-up");
+  CUtensorMap tk, tv, tq;
+  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * pa::kBlock;
+  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, pa::kBlock);
+  if (st != PA_OK) return st;
+  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, pa::kBlock);
+  if (st != PA_OK) return st;
+  st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.qpt);
+  if (st != PA_OK) return st;
+  long long grid = static_cast<long long>(sm_count()) * occ;
+  if (p.max_units < grid) grid = p.max_units;
+  if (grid < 1) grid = 1;
+  kern<<<static_cast<unsigned>(grid), threads, L::kSmem, a.stream>>>(
+      tk, tv, tq, p.s, static_cast<T*>(a.out), a.block_tables, a.qsl, a.seq_lens, row_start,
+      static_cast<float>(a.scale * M_LOG2E), part_o, part_lse);
+  return PA_OK;
+}
+
+template <typename T>
+pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
+  char* ws = static_cast<char*>(a.workspace);
+  int* row_start = reinterpret_cast<int*>(ws);
+  float* part_lse = reinterpret_cast<float*>(ws + p.off_part_lse);
+  float* part_o = reinterpret_cast<float*>(ws + p.off_part_o);
+  pa::schedule_kernel<T><<<1, 1024, 0, a.stream>>>(p.s, a.qsl, a.seq_lens, row_start,
+                                                   static_cast<T*>(a.out));
+  pa_status st;
+  if constexpr (sizeof(T) == 2) {
+    if (use_mma)
+      st = a.head_dim == 128 ? launch_mma<T, 128>(a, p, row_start, part_lse, part_o)
+                             : launch_mma<T, 64>(a, p, row_start, part_lse, part_o);
+    else
+      st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, row_start, part_lse, part_o)
+                             : launch_simt<T, 64>(a, p, row_start, part_lse, part_o);
+  } else {
+    st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, row_start, part_lse, part_o)
+                           : launch_simt<T, 64>(a, p, row_start, part_lse, part_o);
+  }
+  if (st != PA_OK) return st;
+  if (p.s.p_stride > 1) {
+    const long long warps = static_cast<long long>(a.total_q) * a.num_q_heads;
+    const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+    if (a.head_dim == 128)
+      pa::reduce_kernel<T, 128><<<blocks, 256, 0, a.stream>>>(
+          p.s, a.qsl, a.seq_lens, part_o, part_lse, static_cast<T*>(a.out));
+    else
+      pa::reduce_kernel<T, 64><<<blocks, 256, 0, a.stream>>>(
+          p.s, a.qsl, a.seq_lens, part_o, part_lse, static_cast<T*>(a.out));
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return PA_OK;
+}
+
+pa_status run_attention(const AttnArgs& a, bool varlen) {
+  pa_status st = check_common(a);
+  if (st != PA_OK) return st;
+  if (a.total_q == 0 || a.num_seqs == 0) return PA_OK;
+  const int max_len = a.max_seq_len;
+  Plan p = make_plan(a.num_seqs, a.total_q, a.num_q_heads, a.num_kv_heads, a.head_dim, max_len,
+                     varlen);
+  p.s.table_stride = a.table_stride;
+  p.s.num_blocks = a.num_blocks;
+  p.s.max_seq_len = a.max_seq_len;
+  p.s.max_query_len = varlen ? a.max_query_len : 1;
+  if (!a.workspace) return fail(PA_ERR_WORKSPACE, "null workspace (%zu bytes needed)", p.bytes);
+  if (!aligned(a.workspace, 256)) return fail(PA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (a.workspace_bytes < p.bytes)
+    return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", a.workspace_bytes, p.bytes);
+  if (varlen) {
+    if (!a.qsl || !aligned(a.qsl, 4)) return fail(PA_ERR_INVALID_ARG, "bad query_start_loc");
+  }
+  const int path = g_path.load();
+  const bool sixteen = a.dtype != PA_F32;
+  if (path == PA_PATH_MMA || path == PA_PATH_TCGEN05) {
+    if (!sixteen)
+      return fail(PA_ERR_UNSUPPORTED, "tensor-core path needs bf16 or f16 (got fp32)");
+  }
+  const bool use_mma = sixteen && path != PA_PATH_SIMT;
+  switch (a.dtype) {
+    case PA_BF16: return run_typed<__nv_bfloat16>(a, p, use_mma);
+    case PA_F16: return run_typed<__half>(a, p, use_mma);
+    default: return run_typed<float>(a, p, false);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                               const int32_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               void* stream) {
+  if (!valid_dtype(dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks < 0)
+    return fail(PA_ERR_INVALID_ARG, "bad sizes");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
+  if (block_size != pa::kBlock)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 16)", block_size);
+  if (num_tokens == 0) return PA_OK;
+  const void* ptrs[] = {k, v, k_cache, v_cache};
+  for (const void* p : ptrs) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(p, 16)) return fail(PA_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  }
+  if (!slot_mapping || !aligned(slot_mapping, 4))
+    return fail(PA_ERR_INVALID_ARG, "bad slot_mapping pointer");
+  const int row_vecs = head_dim * elem_bytes(dtype) / 16;
+  const long long warps = static_cast<long long>(num_tokens) * num_kv_heads;
+  const long long blocks = (warps * 32 + 255) / 256;
+  if (blocks > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many tokens");
+  pa::reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                                 static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, row_vecs,
+      static_cast<long long>(num_blocks) * pa::kBlock);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache launch");
+  return PA_OK;
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                int max_context_len) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
+  return make_plan(num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                   false)
+      .bytes;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int block_table_stride,
+                    const int32_t* context_lens, int num_seqs, int num_q_heads,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                    int max_context_len, float scale, void* workspace, size_t workspace_bytes,
+                    pa_dtype dtype, void* stream) {
+  AttnArgs a{out, q, k_cache, v_cache, block_tables, block_table_stride, nullptr, context_lens,
+             num_seqs, num_seqs, 1, max_context_len, num_q_heads, num_kv_heads, head_dim,
+             block_size, num_blocks, scale, workspace, workspace_bytes, dtype,
+             static_cast<cudaStream_t>(stream)};
+  return run_attention(a, false);
+}
+
+size_t pa_varlen_workspace_size(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,
+                                int head_dim, int max_query_len, int max_seq_len) {
+  (void)max_query_len;
+  if (num_seqs <= 0 || total_q <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return 0;
+  return make_plan(num_seqs, total_q, num_q_heads, num_kv_heads, head_dim, max_seq_len, true)
+      .bytes;
+}
+
+pa_status pa_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int block_table_stride,
+                    const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
+                    int total_q, int max_query_len, int max_seq_len, int num_q_heads,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                    void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream) {
+  AttnArgs a{out, q, k_cache, v_cache, block_tables, block_table_stride, query_start_loc,
+             seq_lens, num_seqs, total_q, max_query_len, max_seq_len, num_q_heads,
+             num_kv_heads, head_dim, block_size, num_blocks, scale, workspace, workspace_bytes,
+             dtype, static_cast<cudaStream_t>(stream)};
+  return run_attention(a, true);
+}
+
+pa_status pa_get_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  pa::DeviceError rec{};
+  e = cudaMemcpyFromSymbol(&rec, pa::g_device_error, sizeof(rec));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (rec.code == 0) return PA_OK;
+  const pa::DeviceError zero{};
+  e = cudaMemcpyToSymbol(pa::g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  static const char* where[] = {"?", "reshape_and_cache slot", "block-table entry",
+                                "row metadata", "wait for K/V tile", "wait for free stage",
+                                "wait for query tile", "tensor memory", "wait for MMA/barrier"};
+  const int w = rec.where >= 0 && rec.where <= 8 ? rec.where : 0;
+  return fail(static_cast<pa_status>(rec.code), "device: %s (%s; a=%lld b=%lld)",
+              pa_status_string(static_cast<pa_status>(rec.code)), where[w], rec.a, rec.b);
+}
+
+pa_path pa_set_path(pa_path path) {
+  return static_cast<pa_path>(g_path.exchange(static_cast<int>(path)));
+}
+
+const char* pa_status_string(pa_status status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_DEVICE_BOUNDS: return "PA_ERR_DEVICE_BOUNDS";
+    case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT";
+  }
+  return "PA_ERR_UNKNOWN";
+}
+
+const char* pa_last_error_message(void) { return g_msg.c_str(); }
+
+int pa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,167 @@
+// CUDA-core paged attention: the fp32 path, and a fallback for 16-bit types.
+//
+// Same work units as the tensor-core kernel (pa_sched.cuh), processed by a
+// persistent grid of 4-warp CTAs.  Inside a unit, warp w takes the unit's
+// 16-token blocks w, w+4, ... ; each block is found through the request's
+// block-table row ("vLLM 深度拆解" §3.3) and read with plain vector loads.
+// Each warp keeps an online softmax (running max m, sum l, unnormalised o)
+// per tile row in the log2 domain; the epilogue merges the four warps.
+//
+// Lane layout for one block: for scores, lane = 2 * token + half, each lane
+// dots half of head_dim and a shuffle joins the halves; for P.V, lane owns
+// head dims lane, lane + 32, ...
+#pragma once
+
+#include "pa_sched.cuh"
+
+namespace pa {
+
+template <typename T, int D>
+__device__ __forceinline__ void load_half_row(const T* __restrict__ src, float (&dst)[D / 2]) {
+  constexpr int kBytes = D / 2 * sizeof(T);
+  static_assert(kBytes % 16 == 0, "row half must be 16-byte vectors");
+  const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int c = 0; c < kBytes / 16; ++c) {
+    const uint4 w = __ldg(p + c);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+    if constexpr (sizeof(T) == 4) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dst[c * 4 + e] = __uint_as_float(wv[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack2<T>(wv[e]);
+        dst[c * 8 + 2 * e] = f.x;
+        dst[c * 8 + 2 * e + 1] = f.y;
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128, 1)
+    attn_simt_kernel(Shape s, T* __restrict__ out, const T* __restrict__ q,
+                     const T* __restrict__ k_cache, const T* __restrict__ v_cache,
+                     const int* __restrict__ block_tables, const int* __restrict__ qsl,
+                     const int* __restrict__ seq_lens, const int* __restrict__ row_start,
+                     float scale_log2, float* __restrict__ part_o,
+                     float* __restrict__ part_lse) {
+  constexpr int NW = 4;
+  constexpr int HALF = D / 2;
+  constexpr int PER = D / 32;
+  __shared__ __align__(16) float q_s[kRows][D];
+  __shared__ float cm[NW * kRows];
+  __shared__ float cl[NW * kRows];
+  __shared__ __align__(16) float co[NW][kRows][D + 8];
+  __shared__ Unit u_s;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int total = row_start[s.num_seqs];
+  const int tok = lane >> 1, half = lane & 1;
+
+  for (int unit = blockIdx.x; unit < total; unit += gridDim.x) {
+    if (tid == 0) {
+      const int row = find_row_thread(row_start, s.num_seqs, unit);
+      const RowInfo ri = load_row(s, qsl, seq_lens, row);
+      u_s = decode_unit(s, ri, row, unit - row_start[row]);
+    }
+    __syncthreads();
+    const Unit u = u_s;
+    if (u.kv_begin >= u.kv_end) {  // tile rows see no key of this partition
+      __syncthreads();
+      continue;
+    }
+    const int nrows = u.nq * s.gs;
+    for (int idx = tid; idx < kRows * D; idx += NW * 32) {
+      const int r = idx / D, d = idx % D, i = r / s.gs, g = r % s.gs;
+      float val = 0.f;
+      if (i < u.nq && g < u.rows)
+        val = to_f32<T>(q[(static_cast<size_t>(u.token0 + i) * s.num_q_heads + u.head0 + g) * D + d]);
+      q_s[r][d] = val;
+    }
+    __syncthreads();
+
+    float m[kRows], l[kRows], o[kRows][PER], pr[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      m[r] = -INFINITY;
+      l[r] = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o[r][e] = 0.f;
+    }
+
+    const int nblk = ceil_div(u.kv_end - u.kv_begin, kBlock);
+    const int* table = block_tables + static_cast<size_t>(u.row) * s.table_stride;
+    for (int j = warp; j < nblk; j += NW) {
+      const int blk_start = u.kv_begin + j * kBlock;
+      int pb = __ldg(table + blk_start / kBlock);
+      if (pb < 0 || pb >= s.num_blocks) {
+        if (lane == 0) report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, u.row, pb);
+        pb = 0;
+      }
+      const size_t tile = (static_cast<size_t>(pb) * s.num_kv_heads + u.kvh) * kBlock;
+      float kr[HALF];
+      load_half_row<T, D>(k_cache + (tile + tok) * D + half * HALF, kr);
+      const int kidx = blk_start + tok;
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        if (r < nrows) {
+          float sc = 0.f;
+#pragma unroll
+          for (int e = 0; e < HALF; ++e) sc = fmaf(q_s[r][half * HALF + e], kr[e], sc);
+          sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+          const int lim = u.lim0 + r / s.gs;
+          const float x = kidx < lim ? sc * scale_log2 : -INFINITY;
+          float bm = x;
+#pragma unroll
+          for (int off = 2; off < 32; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+          const float mn = fmaxf(m[r], bm);
+          const float mu = mn == -INFINITY ? 0.f : mn;
+          const float alpha = exp2f(m[r] - mu);
+          const float p = exp2f(x - mu);
+          float ps = half == 0 ? p : 0.f;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+          l[r] = l[r] * alpha + ps;
+          m[r] = mn;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) o[r][e] *= alpha;
+          pr[r] = p;
+        }
+      }
+      const int nvalid = u.kv_end - blk_start;  // V rows at or past this are padding
+      const T* vt = v_cache + tile * D;
+#pragma unroll 4
+      for (int t2 = 0; t2 < kBlock; ++t2) {
+        float vv[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e)
+          vv[e] = t2 < nvalid ? to_f32<T>(vt[t2 * D + lane + 32 * e]) : 0.f;
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          if (r < nrows) {
+            const float pp = __shfl_sync(0xffffffffu, pr[r], 2 * t2);
+#pragma unroll
+            for (int e = 0; e < PER; ++e) o[r][e] = fmaf(pp, vv[e], o[r][e]);
+          }
+        }
+      }
+    }
+
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      if (lane == 0) {
+        cm[warp * kRows + r] = m[r];
+        cl[warp * kRows + r] = l[r];
+      }
+#pragma unroll
+      for (int e = 0; e < PER; ++e) co[warp][r][lane + 32 * e] = o[r][e];
+    }
+    __syncthreads();
+    combine_and_store<T, D, NW>(s, u, cm, cl, co, out, part_o, part_lse, tid);
+    __syncthreads();
+  }
+}
+
+}  // namespace pa
