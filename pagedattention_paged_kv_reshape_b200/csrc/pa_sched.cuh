@@ -56,13 +56,12 @@ __device__ __forceinline__ RowInfo load_row(const Shape& s, const int* __restric
     ri.q_len = qsl[row + 1] - ri.token0;
   } else {
     ri.token0 = row;
-    ri.q_len = 1;
+    ri.q_len = ri.seq_len > 0 ? 1 : 0;  // an empty decode context: a zero output row
   }
   ri.ok = ri.seq_len >= 0 && ri.seq_len <= s.max_seq_len &&
           ri.seq_len <= s.table_stride * kBlock && ri.q_len >= 0 &&
           ri.q_len <= ri.seq_len && ri.token0 >= 0 && ri.token0 + ri.q_len <= s.total_q &&
           (qsl == nullptr || ri.q_len <= s.max_query_len);
-  if (qsl == nullptr && ri.seq_len == 0) ri.q_len = 0;  // empty decode row: zero output
   return ri;
 }
 
