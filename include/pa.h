@@ -24,7 +24,8 @@
  * - Every pointer argument except the returned strings is a DEVICE pointer on
  *   the current CUDA device, owned by the caller.  The library keeps no
  *   pointer after the call returns and allocates no device memory: scratch
- *   space is the caller's `workspace`, sized by the *_workspace_size query.
+ *   space is the caller's `workspace`, sized by the *_workspace_size query
+ *   (pa_decode_static uses a fixed array built into the library instead).
  * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *   NULL = the legacy default stream).  No call synchronises, except
  *   pa_get_device_error.  Order pa_reshape_and_cache before the attention call
@@ -158,6 +159,38 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
                     int max_context_len, float scale, void* workspace, size_t workspace_bytes,
                     pa_dtype dtype, void* stream);
+
+/*
+ * pa_decode_static -- pa_decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart: this is a convenience of this library.
+ * Some callers are handed only their input and output buffers and have no
+ * way to obtain scratch memory -- a plugin inside a host runtime that owns
+ * every device allocation, or a hot loop that must not call cudaMalloc
+ * because cudaMalloc can synchronise the whole device.  This entry point
+ * takes the same arguments as pa_decode minus the workspace, and uses a
+ * fixed scratch array built into the library instead.
+ *
+ * - The scratch is PA_STATIC_WORKSPACE_BYTES (32 MiB) of device memory that
+ *   every GPU which loads the library holds until the process exits.  A call
+ *   whose pa_decode_workspace_size(...) exceeds it is rejected with
+ *   PA_ERR_WORKSPACE and launches nothing.
+ * - The first call on each device looks up the scratch's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ * - All calls on a device share the one array: calls that may overlap on the
+ *   GPU (different streams without ordering) race and corrupt each other's
+ *   results.  Order them on one stream.  The array keeps the last call's
+ *   contents; each call rewrites everything it reads before reading it.
+ * - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *   routine.  Everything else -- arguments, layouts, errors -- is pa_decode's.
+ */
+#define PA_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+pa_status pa_decode_static(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int block_table_stride,
+                           const int32_t* context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_context_len, float scale, pa_dtype dtype, void* stream);
 
 /* Workspace (bytes) pa_varlen needs for these sizes. */
 size_t pa_varlen_workspace_size(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,

@@ -20,7 +20,9 @@ from ._binding import (  # noqa: F401
     Status,
     alloc_workspace,
     lib,
+    STATIC_WORKSPACE_BYTES,
     pa_decode,
+    pa_decode_static,
     pa_decode_workspace_size,
     pa_get_device_error,
     pa_reshape_and_cache,

@@ -48,6 +48,8 @@ _SIGNATURES = {
     "pa_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "pa_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _c_int,
                            _c_int, _c_int, _c_int, _c_float, _vp, _c_size, _c_int, _vp]),
+    "pa_decode_static": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
+                                  _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "pa_varlen_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                            _c_int]),
     "pa_varlen": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int, _c_int, _c_int,
@@ -170,6 +172,27 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
         block_tables.shape[1], _ptr(context_lens), S, hq, k_cache.shape[1], d, k_cache.shape[2],
         k_cache.shape[0], int(max_context_len), float(scale), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream)))
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 32 << 20
+
+
+def pa_decode_static(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                     scale: float, stream=None) -> torch.Tensor:
+    """:func:`pa_decode` for callers that cannot allocate device memory: the
+    split-K scratch is a fixed 32 MiB array built into the library.  Calls on
+    one device share it, so calls that may overlap on the GPU race; the first
+    call on a device should come before any stream capture."""
+    _dense(out, q, k_cache, v_cache, block_tables, context_lens)
+    _require(q.shape == out.shape and q.dim() == 3 and q.dtype == out.dtype, "q/out shape")
+    _require(block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32,
+             "metadata must be int32")
+    S, hq, d = q.shape
+    _check(lib().pa_decode_static(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), S, hq, k_cache.shape[1], d, k_cache.shape[2],
+        k_cache.shape[0], int(max_context_len), float(scale), _dtype_code(q), _stream(stream)))
     return out
 
 

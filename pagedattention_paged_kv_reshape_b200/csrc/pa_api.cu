@@ -347,6 +347,30 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
   }
 }
 
+// Scratch for pa_decode_static: a fixed array in the library's device image,
+// for callers that cannot allocate (see include/pa.h).  Host code may not use
+// the symbol itself as a device address; static_workspace() looks the address
+// up once per device with that device current.
+static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
+
+pa_status static_workspace(void** ptr) {
+  static std::mutex mu;
+  static std::map<int, void*> addr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = addr.find(dev);
+  if (it == addr.end()) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+    it = addr.emplace(dev, p).first;
+  }
+  *ptr = it->second;
+  return PA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -403,6 +427,28 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
              block_size, num_blocks, scale, workspace, workspace_bytes, dtype,
              static_cast<cudaStream_t>(stream)};
   return run_attention(a, false);
+}
+
+pa_status pa_decode_static(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int block_table_stride,
+                           const int32_t* context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_context_len, float scale, pa_dtype dtype, void* stream) {
+  const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                               max_context_len);
+  if (need > PA_STATIC_WORKSPACE_BYTES)
+    return fail(PA_ERR_WORKSPACE,
+                "pa_decode_static: these sizes need %zu bytes of scratch; the built-in array "
+                "holds %zu (use pa_decode with a workspace)",
+                need, static_cast<size_t>(PA_STATIC_WORKSPACE_BYTES));
+  void* ws = nullptr;
+  if (need > 0) {
+    const pa_status st = static_workspace(&ws);
+    if (st != PA_OK) return st;
+  }
+  return pa_decode(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                   num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                   max_context_len, scale, ws, PA_STATIC_WORKSPACE_BYTES, dtype, stream);
 }
 
 size_t pa_varlen_workspace_size(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,
