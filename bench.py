@@ -330,6 +330,24 @@ def time_e2e(torch, pa, b, steps):
     return start.elapsed_time(end) / steps, h2d, d2h
 
 
+def combine_over_ranks(local_ms: float, local_bytes: float, local_tokens: float, device):
+    """Whole-job throughput: the slowest rank's time, every rank's bytes and
+    tokens.  Returns (max_ms, GB/s, tokens/s); works on any process group
+    backend (NCCL on GPUs, gloo in the CPU tests) or with none."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    nb = torch.tensor([float(local_bytes)], dtype=torch.float64, device=device)
+    tok = torch.tensor([float(local_tokens)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(nb, op=dist.ReduceOp.SUM)
+        dist.all_reduce(tok, op=dist.ReduceOp.SUM)
+    max_ms = float(t.item())
+    return max_ms, nb.item() / (max_ms / 1e3) / 1e9, tok.item() / (max_ms / 1e3)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -367,15 +385,8 @@ def run_ours(args):
     total_ms, attn_ms, _ = time_steps(torch, pa, b, args.steps, args.warmup)
     clocks = sampler.stop() if sampler else None
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    nbytes = torch.tensor([float(step_bytes) * args.steps], dtype=torch.float64, device=dev)
-    tok = torch.tensor([float(b.total_q) * args.steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dist.all_reduce(nbytes, op=dist.ReduceOp.SUM)
-        dist.all_reduce(tok, op=dist.ReduceOp.SUM)
-    max_ms = float(t.item())
-    value = nbytes.item() / (max_ms / 1e3) / 1e9
+    max_ms, value, tok_per_s = combine_over_ranks(total_ms, step_bytes * args.steps,
+                                                  b.total_q * args.steps, dev)
 
     e2e_ms, h2d, d2h = time_e2e(torch, pa, b, args.e2e_steps)
     e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
@@ -407,7 +418,7 @@ def run_ours(args):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "seed": args.seed},
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-        "tokens_per_s": round(tok.item() / (max_ms / 1e3), 1),
+        "tokens_per_s": round(tok_per_s, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(args.workload),
