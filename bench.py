@@ -20,7 +20,6 @@ from __future__ import annotations
 
 import argparse
 import datetime
-import glob
 import hashlib
 import json
 import math
@@ -64,11 +63,15 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# Sources the attention kernel is compiled from (its traffic record is keyed to them).
+ATTENTION_SOURCES = ("pa_common.cuh", "pa_sched.cuh", "pa_attn_mma.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "pagedattention_paged_kv_reshape_b200", "csrc",
-                                           "*"))):
-        with open(p, "rb") as f:
+    for name in ATTENTION_SOURCES:
+        with open(os.path.join(ROOT, "pagedattention_paged_kv_reshape_b200", "csrc", name),
+                  "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 

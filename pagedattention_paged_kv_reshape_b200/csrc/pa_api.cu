@@ -15,6 +15,7 @@
 
 #include "pa_attn_mma.cuh"
 #include "pa_attn_simt.cuh"
+#include "pa_reduce.cuh"
 #include "pa_reshape.cuh"
 #include "pa_sched.cuh"
 
@@ -163,15 +164,20 @@ struct AttnArgs {
   cudaStream_t stream;
 };
 
+#ifndef PA_STAGES
+#define PA_STAGES 8  // K/V stages of 8 KB per CTA (two CTAs per SM)
+#endif
 constexpr int kNcw = 4;
-constexpr int kStages = 8;
+constexpr int kStages = PA_STAGES;
 
 struct Plan {
   pa::Shape s;
-  size_t off_part_lse, off_part_o, bytes;
+  size_t off_row_a, off_row_b, off_part_lse, off_part_o, bytes;
   long long max_units;
 };
 
+// Workspace layout: the schedule block (Sched), the two per-row unit prefixes,
+// then the split-K partials (only when some context can exceed one partition).
 Plan make_plan(int num_seqs, int total_q, int hq, int hkv, int d, int max_len, bool varlen) {
   Plan p{};
   pa::Shape& s = p.s;
@@ -185,15 +191,17 @@ Plan make_plan(int num_seqs, int total_q, int hq, int hkv, int d, int max_len, b
   s.head_dim = d;
   s.total_q = total_q;
   s.p_stride = max_len > 0 ? (max_len + pa::kPart - 1) / pa::kPart : 1;
-  size_t off = align256(static_cast<size_t>(num_seqs + 1) * 4);
+  const size_t rows = static_cast<size_t>(num_seqs) + 1;
+  p.off_row_a = sizeof(pa::Sched);
+  p.off_row_b = p.off_row_a + rows * 4;
+  size_t off = align256(p.off_row_b + rows * 4);
   p.off_part_lse = off;
+  p.off_part_o = off;
   if (s.p_stride > 1) {
     const size_t slots = static_cast<size_t>(total_q) * hq * s.p_stride;
     off = align256(off + slots * 4);
     p.off_part_o = off;
     off = align256(off + slots * d * 4);
-  } else {
-    p.off_part_o = off;
   }
   p.bytes = num_seqs > 0 ? off : 0;
   const long long items =
@@ -202,6 +210,36 @@ Plan make_plan(int num_seqs, int total_q, int hq, int hkv, int d, int max_len, b
              : num_seqs;
   p.max_units = items * s.p_stride * hkv * s.ns;
   return p;
+}
+
+pa::Work carve(void* workspace, const Plan& p) {
+  char* ws = static_cast<char*>(workspace);
+  pa::Work w;
+  w.sched = reinterpret_cast<pa::Sched*>(ws);
+  w.row_a = reinterpret_cast<int*>(ws + p.off_row_a);
+  w.row_b = reinterpret_cast<int*>(ws + p.off_row_b);
+  w.part_lse = reinterpret_cast<float*>(ws + p.off_part_lse);
+  w.part_o = reinterpret_cast<float*>(ws + p.off_part_o);
+  return w;
+}
+
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel on the stream (the prep kernel) runs; it calls
+// griddepcontrol.wait before reading that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 pa_status check_common(const AttnArgs& a) {
@@ -237,8 +275,7 @@ pa_status check_common(const AttnArgs& a) {
 }
 
 template <typename T, int D>
-pa_status launch_simt(const AttnArgs& a, const Plan& p, int* row_start, float* part_lse,
-                      float* part_o) {
+pa_status launch_simt(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   auto kern = pa::attn_simt_kernel<T, D>;
   int occ = 0;
   cudaError_t e = prepare(kern, 128, 0, &occ);
@@ -246,21 +283,20 @@ pa_status launch_simt(const AttnArgs& a, const Plan& p, int* row_start, float* p
   long long grid = static_cast<long long>(sm_count()) * occ;
   if (p.max_units < grid) grid = p.max_units;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), 128, 0, a.stream>>>(
-      p.s, static_cast<T*>(a.out), static_cast<const T*>(a.q), static_cast<const T*>(a.k_cache),
-      static_cast<const T*>(a.v_cache), a.block_tables, a.qsl, a.seq_lens, row_start,
-      static_cast<float>(a.scale * M_LOG2E), part_o, part_lse);
+  e = launch_pdl(kern, static_cast<unsigned>(grid), 128, 0, a.stream, p.s,
+                 static_cast<T*>(a.out), static_cast<const T*>(a.q),
+                 static_cast<const T*>(a.k_cache), static_cast<const T*>(a.v_cache),
+                 a.block_tables, a.qsl, a.seq_lens, w, static_cast<float>(a.scale * M_LOG2E));
+  if (e != cudaSuccess) return cuda_fail(e, "simt kernel launch");
   return PA_OK;
 }
 
 template <typename T, int D>
-pa_status launch_mma(const AttnArgs& a, const Plan& p, int* row_start, float* part_lse,
-                     float* part_o) {
+pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   using L = pa::MmaLayout<D, kNcw, kStages>;
   auto kern = pa::attn_mma_kernel<T, D, kNcw, kStages>;
-  const int threads = (kNcw + 1) * 32;
   int occ = 0;
-  cudaError_t e = prepare(kern, threads, L::kSmem, &occ);
+  cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "mma kernel set-up");
   CUtensorMap tk, tv, tq;
   const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * pa::kBlock;
@@ -273,45 +309,38 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, int* row_start, float* pa
   long long grid = static_cast<long long>(sm_count()) * occ;
   if (p.max_units < grid) grid = p.max_units;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), threads, L::kSmem, a.stream>>>(
-      tk, tv, tq, p.s, static_cast<T*>(a.out), a.block_tables, a.qsl, a.seq_lens, row_start,
-      static_cast<float>(a.scale * M_LOG2E), part_o, part_lse);
+  e = launch_pdl(kern, static_cast<unsigned>(grid), L::kThreads, L::kSmem, a.stream, tk, tv, tq,
+                 p.s, static_cast<T*>(a.out), a.block_tables, a.qsl, a.seq_lens, w,
+                 static_cast<float>(a.scale * M_LOG2E));
+  if (e != cudaSuccess) return cuda_fail(e, "mma kernel launch");
   return PA_OK;
 }
 
 template <typename T>
 pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
-  char* ws = static_cast<char*>(a.workspace);
-  int* row_start = reinterpret_cast<int*>(ws);
-  float* part_lse = reinterpret_cast<float*>(ws + p.off_part_lse);
-  float* part_o = reinterpret_cast<float*>(ws + p.off_part_o);
-  pa::schedule_kernel<T><<<1, 1024, 0, a.stream>>>(p.s, a.qsl, a.seq_lens, row_start,
+  const pa::Work w = carve(a.workspace, p);
+  pa::schedule_kernel<T><<<1, 1024, 0, a.stream>>>(p.s, a.qsl, a.seq_lens, w,
                                                    static_cast<T*>(a.out));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
   pa_status st;
   if constexpr (sizeof(T) == 2) {
     if (use_mma)
-      st = a.head_dim == 128 ? launch_mma<T, 128>(a, p, row_start, part_lse, part_o)
-                             : launch_mma<T, 64>(a, p, row_start, part_lse, part_o);
+      st = a.head_dim == 128 ? launch_mma<T, 128>(a, p, w) : launch_mma<T, 64>(a, p, w);
     else
-      st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, row_start, part_lse, part_o)
-                             : launch_simt<T, 64>(a, p, row_start, part_lse, part_o);
+      st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, w) : launch_simt<T, 64>(a, p, w);
   } else {
-    st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, row_start, part_lse, part_o)
-                           : launch_simt<T, 64>(a, p, row_start, part_lse, part_o);
+    st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, w) : launch_simt<T, 64>(a, p, w);
   }
-  if (st != PA_OK) return st;
-  if (p.s.p_stride > 1) {
-    const long long warps = static_cast<long long>(a.total_q) * a.num_q_heads;
-    const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
-    if (a.head_dim == 128)
-      pa::reduce_kernel<T, 128><<<blocks, 256, 0, a.stream>>>(
-          p.s, a.qsl, a.seq_lens, part_o, part_lse, static_cast<T*>(a.out));
-    else
-      pa::reduce_kernel<T, 64><<<blocks, 256, 0, a.stream>>>(
-          p.s, a.qsl, a.seq_lens, part_o, part_lse, static_cast<T*>(a.out));
-  }
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  if (st != PA_OK || p.s.p_stride <= 1) return st;
+  const long long warps = static_cast<long long>(a.total_q) * a.num_q_heads;
+  const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+  e = a.head_dim == 128
+          ? launch_pdl(pa::reduce_kernel<T, 128>, blocks, 256, 0, a.stream, p.s, a.qsl,
+                       a.seq_lens, w, static_cast<T*>(a.out))
+          : launch_pdl(pa::reduce_kernel<T, 64>, blocks, 256, 0, a.stream, p.s, a.qsl,
+                       a.seq_lens, w, static_cast<T*>(a.out));
+  if (e != cudaSuccess) return cuda_fail(e, "reduce kernel launch");
   return PA_OK;
 }
 

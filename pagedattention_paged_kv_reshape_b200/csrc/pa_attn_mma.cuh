@@ -1,30 +1,39 @@
 // Paged attention on sm_100a: TMA-staged K/V tiles + warp-level tensor-core MMA.
 //
-// Persistent, warp-specialised CTA (NCW consumer warps + 1 producer warp):
+// Persistent, warp-specialised CTA: NCW consumer warps, one TMA warp, one
+// scheduler warp.
 //
-// * The producer walks this CTA's work units (pa_sched.cuh), looks each
-//   logical block up in the request's block-table row ("vLLM 深度拆解" §3.3:
-//   physical = block_tables[seq*stride + logical]) and issues
-//   cp.async.bulk.tensor loads of the (block, KV head) K tile and V tile --
-//   16 tokens x head_dim, 4 KB each at bf16 x 128 -- into a STAGES-deep ring
-//   of shared-memory stages, completed on mbarriers.  It also loads the tile's
-//   query rows.  The tensor maps use 128-byte swizzling so the ldmatrix reads
-//   below are free of bank conflicts.  Nothing else sits between HBM and the
-//   MMA, and no load waits for compute: the ring keeps up to STAGES * 8 KB in
-//   flight per CTA.
-// * Consumer warp w takes the unit's blocks w, w+NCW, ...  For each block it
-//   computes S = Q K^T (16 tile rows x 16 tokens, m16n8k16 MMAs, fp32
-//   accumulate), masks keys past each row's limit, updates its online softmax
-//   in the log2 domain (running max m, sum l), rounds P to the input type and
-//   accumulates O += P V with the same MMA.  A whole GQA group (up to 16 query
-//   heads) shares one K/V tile, so each KV block is read once per KV head.
-// * At the end of a unit the consumer warps merge their (m, l, O) states and
-//   write the output row, or the partition's partial for the split-K reduce.
+// * The scheduler warp claims work units (pa_sched.cuh) from a global counter,
+//   decodes them and loads the request's block-table entries for the unit's
+//   partition ("vLLM 深度拆解" §3.3: physical = block_tables[seq*stride +
+//   logical]) into a ring of shared-memory slots, running several units ahead
+//   so that the dependent global loads of that lookup never delay the stream.
+// * The TMA warp takes each slot and issues cp.async.bulk.tensor loads of the
+//   tile's query rows and of every (block, KV head) K tile and V tile --
+//   16 tokens x head_dim, 4 KB each at bf16 x 128 -- into a STAGES-deep ring of
+//   shared-memory stages completed on mbarriers.  The tensor maps use 128-byte
+//   swizzling, so the ldmatrix reads below are free of bank conflicts.
+// * Consumer warp w takes the unit's blocks w, w+NCW, ...: S = Q K^T (16 tile
+//   rows x 16 tokens, m16n8k16 MMAs, fp32 accumulate), masking of keys past
+//   each row's limit, online softmax in the log2 domain (running max m, sum
+//   l), P rounded to the input type, O += P V with the same MMA.  A whole GQA
+//   group (up to 16 query heads) shares one K/V tile, so each KV block is read
+//   once per KV head.
+// * At the end of a unit the consumer warps merge their states and write the
+//   output row, or the partition's partial for the split-K reduce.
 #pragma once
 
 #include "pa_sched.cuh"
 
 namespace pa {
+
+constexpr int kMetaSlots = 4;
+
+// One scheduler-ring slot: a decoded unit and its partition's block ids.
+struct MetaSlot {
+  Unit u;
+  int pb[kPart / kBlock];
+};
 
 template <int D, int NCW, int STAGES>
 struct MmaLayout {
@@ -40,11 +49,14 @@ struct MmaLayout {
   static constexpr int kOffCm = kOffCo + kCoBytes;
   static constexpr int kOffCl = kOffCm + NCW * kRows * 4;
   static constexpr int kOffBar = kOffCl + NCW * kRows * 4;
-  static constexpr int kNumBars = 2 * STAGES + 2 * kQSlots + 1;  // + consumer barrier
+  // full[S], empty[S], qfull[2], qempty[2], meta_full[M], meta_empty[M], consumers
+  static constexpr int kNumBars = 2 * STAGES + 2 * kQSlots + 2 * kMetaSlots + 1;
   static constexpr int kOffDesc = kOffBar + kNumBars * 8;
-  static constexpr int kOffAbort = kOffDesc + kQSlots * static_cast<int>(sizeof(Unit));
-  static constexpr int kBytes = kOffAbort + 16;
+  static constexpr int kOffMeta = kOffDesc + kQSlots * static_cast<int>(sizeof(Unit));
+  static constexpr int kOffFlags = kOffMeta + kMetaSlots * static_cast<int>(sizeof(MetaSlot));
+  static constexpr int kBytes = kOffFlags + 16;
   static constexpr int kSmem = kBytes + 1024;  // slack to align the base to 1024 B
+  static constexpr int kThreads = (NCW + 2) * 32;
   static_assert(kOffQ % 1024 == 0 && kQSlotBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
 };
 
@@ -56,13 +68,12 @@ __device__ __forceinline__ uint32_t swz(int r, int ch) {
 }
 
 template <typename T, int D, int NCW, int STAGES>
-__global__ void __launch_bounds__((NCW + 1) * 32, 2)
+__global__ void __launch_bounds__((NCW + 2) * 32, 2)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, Shape s, T* __restrict__ out,
                     const int* __restrict__ block_tables, const int* __restrict__ qsl,
-                    const int* __restrict__ seq_lens, const int* __restrict__ row_start,
-                    float scale_log2, float* __restrict__ part_o, float* __restrict__ part_lse) {
+                    const int* __restrict__ seq_lens, Work w, float scale_log2) {
   using L = MmaLayout<D, NCW, STAGES>;
   constexpr int KSTEPS = D / 16;  // k-steps of QK^T, also n-tile pairs of PV
   constexpr int NT = D / 8;       // PV n-tiles of 8 dims
@@ -75,9 +86,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 2)
   auto empty_bar = [&](int st) { return bar0 + 8u * (STAGES + st); };
   auto qfull_bar = [&](int qs) { return bar0 + 8u * (2 * STAGES + qs); };
   auto qempty_bar = [&](int qs) { return bar0 + 8u * (2 * STAGES + L::kQSlots + qs); };
-  const uint32_t cons_bar = bar0 + 8u * (2 * STAGES + 2 * L::kQSlots);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
+  auto mfull_bar = [&](int ms) { return bar0 + 8u * (2 * STAGES + 2 * L::kQSlots + ms); };
+  auto mempty_bar = [&](int ms) {
+    return bar0 + 8u * (2 * STAGES + 2 * L::kQSlots + kMetaSlots + ms);
+  };
+  const uint32_t cons_bar = bar0 + 8u * (2 * STAGES + 2 * L::kQSlots + 2 * kMetaSlots);
   Unit* desc = reinterpret_cast<Unit*>(smem + L::kOffDesc);
+  MetaSlot* meta = reinterpret_cast<MetaSlot*>(smem + L::kOffMeta);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffFlags);
   float* cm = reinterpret_cast<float*>(smem + L::kOffCm);
   float* cl = reinterpret_cast<float*>(smem + L::kOffCl);
   auto co = reinterpret_cast<float(*)[kRows][D + 8]>(smem + L::kOffCo);
@@ -92,100 +108,118 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 2)
       mbar_init(qfull_bar(qs), 1);
       mbar_init(qempty_bar(qs), NCW);
     }
+    for (int ms = 0; ms < kMetaSlots; ++ms) {
+      mbar_init(mfull_bar(ms), 1);
+      mbar_init(mempty_bar(ms), 1);
+    }
     mbar_init(cons_bar, NCW);
     *abort_flag = 0;
     fence_barrier_init();
   }
   // unused query rows of a tile must hold finite values
-  for (int i = tid; i < L::kQSlots * L::kQSlotBytes / 16; i += blockDim.x)
+  for (int i = tid; i < L::kQSlots * L::kQSlotBytes / 16; i += L::kThreads)
     reinterpret_cast<uint4*>(smem + L::kOffQ)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   __syncthreads();
+  // Everything above overlapped the prep kernel; its results are read below.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  const int total = row_start[s.num_seqs];
-
-  if (warp == NCW) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      prefetch_tensormap(&tm_q);
-    }
-    const uint32_t q_bytes = static_cast<uint32_t>(L::kHalves * 128 * s.gs * s.qpt);
-    int n = 0, k = 0, cursor = 0, issued = 0;
-    bool ok = true;
-    for (int unit = blockIdx.x; ok; unit += gridDim.x) {
+  if (warp == NCW + 1) {
+    // ----------------------------------------------------------- scheduler
+    const int total_a = __ldcg(&w.sched->total_a);
+    const int total = total_a + __ldcg(&w.sched->total_b);
+    int cur_a = 0, cur_b = 0, j = 0;
+    int next = 0;
+    if (lane == 0) next = atomicAdd(&w.sched->next, 1);
+    next = __shfl_sync(0xffffffffu, next, 0);
+    while (true) {
+      const int unit = next;
       const bool done = unit >= total;
+      if (!done) {  // claim the following unit now; its value is needed next round
+        int nx = 0;
+        if (lane == 0) nx = atomicAdd(&w.sched->next, 1);
+        next = __shfl_sync(0xffffffffu, nx, 0);
+      }
       Unit un;
+      int e = 0;
       if (!done) {
-        int start;
-        const int row = find_row_warp(row_start, s.num_seqs, unit, cursor, start);
-        cursor = row;
+        int local, cls;
+        const int row = locate_unit_warp(s, w, total_a, unit, cur_a, cur_b, local, cls);
         const RowInfo ri = load_row(s, qsl, seq_lens, row);
-        un = decode_unit(s, ri, row, unit - start);
+        un = decode_unit(s, ri, row, local, cls);
         if (un.kv_begin >= un.kv_end) continue;  // no key of this partition is visible
-      } else {
-        un.row = -1;
-      }
-      const int qs = k & 1;
-      const uint32_t qph = (k >> 1) & 1;
-      if (lane == 0) {
-        ok = mbar_wait(qempty_bar(qs), qph ^ 1, kWhereWaitQ, abort_flag);
-        if (ok) {
-          desc[qs] = un;
-          if (done) {
-            mbar_arrive(qfull_bar(qs));
-          } else {
-            mbar_arrive_expect_tx(qfull_bar(qs), q_bytes);
-            const uint32_t qdst = sbase + L::kOffQ + qs * L::kQSlotBytes;
-#pragma unroll
-            for (int h = 0; h < L::kHalves; ++h)
-              tma_load_3d(qdst + h * (kRows * 128), &tm_q, qfull_bar(qs), h * 64, un.head0,
-                          un.token0);
-          }
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++k;
-      if (done || !ok) break;
-      const int nblk = ceil_div(un.kv_end - un.kv_begin, kBlock);
-      const int* table = block_tables + static_cast<size_t>(un.row) * s.table_stride +
-                         un.kv_begin / kBlock;
-      for (int c = 0; c < nblk && ok; c += 32) {
-        int e = 0;
-        if (c + lane < nblk) {
-          e = __ldg(table + c + lane);
+        const int nblk = ceil_div(un.kv_end - un.kv_begin, kBlock);
+        if (lane < nblk) {
+          e = __ldg(block_tables + static_cast<size_t>(row) * s.table_stride +
+                    un.kv_begin / kBlock + lane);
           if (e < 0 || e >= s.num_blocks) {
-            report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, un.row, e);
+            report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, row, e);
             e = 0;
           }
         }
-        const int cnt = min(32, nblk - c);
-        for (int jj = 0; jj < cnt; ++jj) {
-          const int pb = __shfl_sync(0xffffffffu, e, jj);
-          if (lane == 0 && ok) {
-            const int st = n % STAGES;
-            const uint32_t ph = (n / STAGES) & 1;
-            ok = mbar_wait(empty_bar(st), ph ^ 1, kWhereWaitEmpty, abort_flag);
-            if (ok) {
-              ++issued;
-              mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
-              const int y = (pb * s.num_kv_heads + un.kvh) * kBlock;
-              const uint32_t kdst = sbase + st * L::kStageBytes;
-#pragma unroll
-              for (int h = 0; h < L::kHalves; ++h) {
-                tma_load_2d(kdst + h * L::kHalfBytes, &tm_k, full_bar(st), h * 64, y);
-                tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes, &tm_v, full_bar(st), h * 64,
-                            y);
-              }
-            }
-          }
-          ++n;
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+      } else {
+        un.row = -1;
       }
+      const int ms = j % kMetaSlots;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(mempty_bar(ms), ((j / kMetaSlots) & 1) ^ 1, kWhereWaitQ,
+                                    abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      meta[ms].pb[lane] = e;
+      if (lane == 0) meta[ms].u = un;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(mfull_bar(ms));
+      ++j;
+      if (done) break;
     }
-    if (!ok && lane == 0) {
+    return;
+  }
+
+  if (warp == NCW) {
+    // ----------------------------------------------------------------- TMA
+    if (lane != 0) return;
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_q);
+    const uint32_t q_bytes = static_cast<uint32_t>(L::kHalves * 128 * s.gs * s.qpt);
+    int n = 0, issued = 0;
+    bool ok = true;
+    for (int j = 0; ok; ++j) {
+      const int ms = j % kMetaSlots;
+      if (!(ok = mbar_wait(mfull_bar(ms), (j / kMetaSlots) & 1, kWhereWaitQ, abort_flag))) break;
+      const Unit un = meta[ms].u;
+      const int qs = j & 1;
+      if (!(ok = mbar_wait(qempty_bar(qs), ((j >> 1) & 1) ^ 1, kWhereWaitQ, abort_flag))) break;
+      desc[qs] = un;
+      if (un.row < 0) {
+        mbar_arrive(qfull_bar(qs));
+        break;
+      }
+      mbar_arrive_expect_tx(qfull_bar(qs), q_bytes);
+      const uint32_t qdst = sbase + L::kOffQ + qs * L::kQSlotBytes;
+#pragma unroll
+      for (int h = 0; h < L::kHalves; ++h)
+        tma_load_3d(qdst + h * (kRows * 128), &tm_q, qfull_bar(qs), h * 64, un.head0, un.token0);
+      const int nblk = ceil_div(un.kv_end - un.kv_begin, kBlock);
+      for (int jj = 0; jj < nblk; ++jj, ++n) {
+        const int pb = meta[ms].pb[jj];
+        const int st = n % STAGES;
+        if (!(ok = mbar_wait(empty_bar(st), ((n / STAGES) & 1) ^ 1, kWhereWaitEmpty, abort_flag)))
+          break;
+        ++issued;
+        mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
+        const int y = (pb * s.num_kv_heads + un.kvh) * kBlock;
+        const uint32_t kdst = sbase + st * L::kStageBytes;
+#pragma unroll
+        for (int h = 0; h < L::kHalves; ++h) {
+          tma_load_2d(kdst + h * L::kHalfBytes, &tm_k, full_bar(st), h * 64, y);
+          tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes, &tm_v, full_bar(st), h * 64, y);
+        }
+      }
+      mbar_arrive(mempty_bar(ms));
+    }
+    if (!ok) {
       // A wait gave up: let the loads already issued land before leaving
       // (each wait bounded again, independently of the CTA's abort flag).
       volatile int drain_flag = 0;
@@ -214,7 +248,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 2)
     const uint32_t qph = (k >> 1) & 1;
     if (!mbar_wait(qfull_bar(qs), qph, kWhereWaitQ, abort_flag)) return;
     const Unit u = desc[qs];
-    if (u.row < 0) break;
+    if (u.row < 0) {
+      // no more work for this CTA: a dependent reduce kernel may start launching
+      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+      break;
+    }
     uint32_t qa[KSTEPS][4];
     {
       const uint32_t qb = sbase + L::kOffQ + qs * L::kQSlotBytes;
@@ -349,7 +387,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 2)
       *reinterpret_cast<float2*>(&co[warp][r1][t * 8 + 2 * quad]) = make_float2(o[t][2], o[t][3]);
     }
     if (!consumers_sync()) return;
-    combine_and_store<T, D, NCW>(s, u, cm, cl, co, out, part_o, part_lse, tid);
+    epilogue<T, D, NCW>(s, u, cm, cl, co, out, w, tid, NCW * 32);
     if (!consumers_sync()) return;
   }
 }

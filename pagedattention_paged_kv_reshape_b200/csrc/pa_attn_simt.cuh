@@ -44,9 +44,7 @@ __global__ void __launch_bounds__(128, 1)
     attn_simt_kernel(Shape s, T* __restrict__ out, const T* __restrict__ q,
                      const T* __restrict__ k_cache, const T* __restrict__ v_cache,
                      const int* __restrict__ block_tables, const int* __restrict__ qsl,
-                     const int* __restrict__ seq_lens, const int* __restrict__ row_start,
-                     float scale_log2, float* __restrict__ part_o,
-                     float* __restrict__ part_lse) {
+                     const int* __restrict__ seq_lens, Work w, float scale_log2) {
   constexpr int NW = 4;
   constexpr int HALF = D / 2;
   constexpr int PER = D / 32;
@@ -56,18 +54,26 @@ __global__ void __launch_bounds__(128, 1)
   __shared__ __align__(16) float co[NW][kRows][D + 8];
   __shared__ Unit u_s;
 
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the prep kernel's results
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int total = row_start[s.num_seqs];
+  const int total_a = __ldcg(&w.sched->total_a);
+  const int total = total_a + __ldcg(&w.sched->total_b);
   const int tok = lane >> 1, half = lane & 1;
-
-  for (int unit = blockIdx.x; unit < total; unit += gridDim.x) {
+  while (true) {
     if (tid == 0) {
-      const int row = find_row_thread(row_start, s.num_seqs, unit);
-      const RowInfo ri = load_row(s, qsl, seq_lens, row);
-      u_s = decode_unit(s, ri, row, unit - row_start[row]);
+      const int unit = atomicAdd(&w.sched->next, 1);
+      if (unit < total) {
+        int local, cls;
+        const int row = locate_unit_thread(s, w, total_a, unit, local, cls);
+        const RowInfo ri = load_row(s, qsl, seq_lens, row);
+        u_s = decode_unit(s, ri, row, local, cls);
+      } else {
+        u_s.row = -1;
+      }
     }
     __syncthreads();
     const Unit u = u_s;
+    if (u.row < 0) break;
     if (u.kv_begin >= u.kv_end) {  // tile rows see no key of this partition
       __syncthreads();
       continue;
@@ -159,7 +165,7 @@ __global__ void __launch_bounds__(128, 1)
       for (int e = 0; e < PER; ++e) co[warp][r][lane + 32 * e] = o[r][e];
     }
     __syncthreads();
-    combine_and_store<T, D, NW>(s, u, cm, cl, co, out, part_o, part_lse, tid);
+    epilogue<T, D, NW>(s, u, cm, cl, co, out, w, tid, NW * 32);
     __syncthreads();
   }
 }

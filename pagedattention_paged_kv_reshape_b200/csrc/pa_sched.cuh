@@ -1,21 +1,29 @@
-// Work decomposition shared by the attention kernels, the split-K reduce and
-// the epilogue that merges per-warp online-softmax states.
+// Work decomposition shared by the attention kernels, and the epilogue that
+// merges online-softmax states (across warps, then across split-K partitions).
 //
 // A batch is a list of rows (requests).  Row r has q_len query tokens (1 for
 // a decode row) at positions seq_len - q_len + i ("vLLM 架构源码解析" §3.3.2:
-// positions run from num_computed_tokens) and reads keys 0 .. position.
+// positions run from num_computed_tokens); query i reads keys 0 .. position.
 //
 // Work unit = (row, query tile, KV head slice, partition):
-//   * query tile   : up to `qpt` consecutive query tokens of the row;
-//   * head slice   : up to 16 query heads of one KV head (all of a GQA group
-//                    when it has <= 16 heads), so each KV block is streamed
-//                    once per KV head and tile;
-//   * partition    : keys [p*512, (p+1)*512) -- the split-K unit.
+//   * query tile  : up to `qpt` consecutive query tokens of the row;
+//   * head slice  : up to 16 query heads of one KV head (a whole GQA group
+//                   when it has <= 16 heads), so each KV block is streamed
+//                   once per KV head and tile;
+//   * partition   : keys [p*512, (p+1)*512), the split-K unit.
 // Tile rows are (query token, head) pairs, row = i * gs + g, at most 16.
 //
-// A one-CTA prep kernel writes row_start[r] = number of units before row r,
-// so a persistent attention CTA maps a unit index to its row with a short
-// forward scan and decodes the rest by division.
+// Units come in two classes so the longest go first: class A holds every
+// partition but a row's last (always 512 keys), class B the last partitions.
+// A one-CTA prep kernel validates the rows and writes prefix sums of both
+// classes; CTAs of the attention kernel claim unit indices from an atomic
+// counter, so the short tail units are spread over whichever CTAs free up.
+//
+// When a tile's keys span several partitions, each unit writes its rows'
+// partial state (normalised o and log2-sum-exp) to the workspace and
+// reduce_kernel merges them by log-sum-exp.  (Merging inside the attention
+// kernel, by the last unit of each tile, was measured slower: the merge
+// stalls that CTA's consumer warps while the stage ring drains.)
 #pragma once
 
 #include "pa_common.cuh"
@@ -37,6 +45,23 @@ struct Shape {
   int max_query_len;
   int total_q;
   int p_stride;     // partitions per (token, head) in the workspace
+};
+
+// Schedule block at the start of the workspace.
+struct Sched {
+  int next;      // next unit index to claim
+  int total_a;   // class-A units
+  int total_b;   // class-B units
+  int pad;
+};
+
+// Pointers into the workspace.
+struct Work {
+  Sched* sched;
+  int* row_a;       // [num_seqs + 1] prefix of class-A units
+  int* row_b;       // [num_seqs + 1] prefix of class-B units
+  float* part_lse;  // [total_q][Hq][p_stride]
+  float* part_o;    // [total_q][Hq][p_stride][D]
 };
 
 // Per-row metadata.  `qsl` is null for decode batches (row r owns token r).
@@ -65,11 +90,16 @@ __device__ __forceinline__ RowInfo load_row(const Shape& s, const int* __restric
   return ri;
 }
 
-__device__ __forceinline__ int row_units(const Shape& s, const RowInfo& ri) {
-  if (!ri.ok || ri.q_len == 0) return 0;
+__device__ __forceinline__ int head_units(const Shape& s) { return s.num_kv_heads * s.ns; }
+
+// Units of each class in a row.
+__device__ __forceinline__ void row_units(const Shape& s, const RowInfo& ri, int& a, int& b) {
+  a = b = 0;
+  if (!ri.ok || ri.q_len == 0) return;
   const int items = ceil_div(ri.q_len, s.qpt);
   const int parts = ceil_div(ri.seq_len, kPart);
-  return items * parts * s.num_kv_heads * s.ns;
+  b = items * head_units(s);
+  a = b * (parts - 1);
 }
 
 struct Unit {
@@ -85,18 +115,24 @@ struct Unit {
   int lim0;      // keys visible to tile row 0 (its position + 1); row i*gs+g sees lim0 + i
 };
 
-// Decode the unit at offset `local` inside row `row`.  Unit order inside a row:
-// query tile fastest, then partition, then head slice -- consecutive units of
-// a prefill chunk read the same KV blocks, which stay in L2.
+// Decode the unit at offset `local` of class `cls` inside row `row`.  Inside a
+// row the query tile varies fastest, so consecutive units of a prefill chunk
+// read the same KV blocks while they are in L2.
 __device__ __forceinline__ Unit decode_unit(const Shape& s, const RowInfo& ri, int row,
-                                            int local) {
+                                            int local, int cls) {
   Unit u;
   const int items = ceil_div(ri.q_len, s.qpt);
   const int parts = ceil_div(ri.seq_len, kPart);
   const int item = local % items;
   const int rest = local / items;
-  u.p = rest % parts;
-  const int hu = rest / parts;
+  int hu;
+  if (cls == 0) {
+    u.p = rest % (parts - 1);
+    hu = rest / (parts - 1);
+  } else {
+    u.p = parts - 1;
+    hu = rest;
+  }
   u.kvh = hu / s.ns;
   const int slice = hu % s.ns;
   u.head0 = u.kvh * s.group + slice * kRows;
@@ -111,77 +147,19 @@ __device__ __forceinline__ Unit decode_unit(const Shape& s, const RowInfo& ri, i
   return u;
 }
 
-// Number of partitions whose partial state a query at `limit` visible keys
-// has (1 = written directly as output, no reduce).
+// Number of partitions holding keys visible to a query that sees `limit` keys
+// (1 = its output is written directly, without partials).
 __device__ __forceinline__ int parts_for(int limit) { return ceil_div(limit, kPart); }
 
-// ---------------------------------------------------------------------------
-// Prep kernel: validate rows, write row_start (exclusive prefix of units),
-// zero the output rows of empty decode requests.  One CTA of 1024 threads.
-// ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(1024) schedule_kernel(Shape s, const int* __restrict__ qsl,
-                                                        const int* __restrict__ seq_lens,
-                                                        int* __restrict__ row_start,
-                                                        T* __restrict__ out) {
-  __shared__ int warp_tot[32];
-  __shared__ int carry_s;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) {
-    carry_s = 0;
-    if (qsl && (qsl[0] != 0 || qsl[s.num_seqs] != s.total_q))
-      report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, -1, qsl[s.num_seqs]);
-  }
-  __syncthreads();
-  for (int base = 0; base < s.num_seqs; base += 1024) {
-    const int r = base + tid;
-    int v = 0;
-    if (r < s.num_seqs) {
-      const RowInfo ri = load_row(s, qsl, seq_lens, r);
-      if (!ri.ok) report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, r, ri.seq_len);
-      v = row_units(s, ri);
-      if (ri.ok && qsl == nullptr && ri.seq_len == 0) {
-        // attention over an empty context: a zero row
-        T* o = out + static_cast<size_t>(r) * s.num_q_heads * s.head_dim;
-        for (int i = 0; i < s.num_q_heads * s.head_dim; ++i) o[i] = from_f32<T>(0.f);
-      }
-    }
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_tot[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = warp_tot[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      warp_tot[lane] = w;
-    }
-    __syncthreads();
-    const int excl = carry_s + x - v + (warp > 0 ? warp_tot[warp - 1] : 0);
-    if (r < s.num_seqs) row_start[r] = excl;
-    __syncthreads();
-    if (tid == 1023) carry_s = excl + v;
-    __syncthreads();
-  }
-  if (tid == 0) row_start[s.num_seqs] = carry_s;
-}
-
 // Largest r with row_start[r] <= u, scanning forward from `cursor` one warp
-// (32 rows) at a time.  All lanes of the warp call it; returns the row and
-// its row_start in `start`.  Requires u < row_start[num_seqs].
+// (32 rows) at a time.  All lanes of the warp call it; returns the row and its
+// row_start.  Requires row_start non-decreasing and u < row_start[num_seqs].
 __device__ __forceinline__ int find_row_warp(const int* __restrict__ row_start, int num_seqs,
                                              int u, int cursor, int& start) {
   const int lane = threadIdx.x & 31;
   while (true) {
     const int idx = cursor + lane;
-    const int v = idx <= num_seqs ? row_start[idx] : 0x7fffffff;
+    const int v = idx <= num_seqs ? __ldcg(row_start + idx) : 0x7fffffff;
     const unsigned m = __ballot_sync(0xffffffffu, v <= u);
     const int cnt = __popc(m);
     if (cnt < 32) {
@@ -192,13 +170,13 @@ __device__ __forceinline__ int find_row_warp(const int* __restrict__ row_start, 
   }
 }
 
-// Binary search version for a single thread.
+// Same, binary search, one thread.
 __device__ __forceinline__ int find_row_thread(const int* __restrict__ row_start, int num_seqs,
                                                int u) {
   int lo = 0, hi = num_seqs - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (row_start[mid] <= u)
+    if (__ldcg(row_start + mid) <= u)
       lo = mid;
     else
       hi = mid - 1;
@@ -206,40 +184,173 @@ __device__ __forceinline__ int find_row_thread(const int* __restrict__ row_start
   return lo;
 }
 
+// Map a claimed unit index to (row, local offset, class); class-A units come
+// first.  Warp form: forward scans from the caller's cursors.
+__device__ __forceinline__ int locate_unit_warp(const Shape& s, const Work& w, int total_a, int u,
+                                                int& cur_a, int& cur_b, int& local, int& cls) {
+  int start;
+  int row;
+  if (u < total_a) {
+    cls = 0;
+    row = find_row_warp(w.row_a, s.num_seqs, u, cur_a, start);
+    cur_a = row;
+    local = u - start;
+  } else {
+    cls = 1;
+    const int ub = u - total_a;
+    row = find_row_warp(w.row_b, s.num_seqs, ub, cur_b, start);
+    cur_b = row;
+    local = ub - start;
+  }
+  return row;
+}
+
+// Thread form: binary search.
+__device__ __forceinline__ int locate_unit_thread(const Shape& s, const Work& w, int total_a,
+                                                  int u, int& local, int& cls) {
+  int row;
+  if (u < total_a) {
+    cls = 0;
+    row = find_row_thread(w.row_a, s.num_seqs, u);
+    local = u - __ldcg(w.row_a + row);
+  } else {
+    cls = 1;
+    const int ub = u - total_a;
+    row = find_row_thread(w.row_b, s.num_seqs, ub);
+    local = ub - __ldcg(w.row_b + row);
+  }
+  return row;
+}
+
 // ---------------------------------------------------------------------------
-// Epilogue: merge NW warps' online-softmax states for the tile's rows and
-// write either the final output (row's keys all in partition 0) or this
-// partition's partial (normalised o and log2-sum-exp) for the reduce.
-//
-// Shared layout: cm[NW][16], cl[NW][16] (running max in log2 units and sum),
-// co[NW][16][D + 8] (unnormalised accumulators).
+// Prep kernel: validate rows, write the two prefix sums and the totals, zero
+// the claim counter, zero the output rows of empty decode requests.  One CTA of 1024 threads.  It lets the attention kernel
+// launch at once (programmatic dependent launch); that kernel waits for this
+// grid to complete before it reads any of the above.
 // ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(1024) schedule_kernel(Shape s, const int* __restrict__ qsl,
+                                                        const int* __restrict__ seq_lens,
+                                                        Work w, T* __restrict__ out) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ int warp_tot[2][32];
+  __shared__ int carry_s[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    carry_s[0] = carry_s[1] = 0;
+    if (qsl && (qsl[0] != 0 || qsl[s.num_seqs] != s.total_q))
+      report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, -1, qsl[s.num_seqs]);
+  }
+  __syncthreads();
+  for (int base = 0; base < s.num_seqs; base += 1024) {
+    const int r = base + tid;
+    int va = 0, vb = 0;
+    if (r < s.num_seqs) {
+      const RowInfo ri = load_row(s, qsl, seq_lens, r);
+      if (!ri.ok) report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, r, ri.seq_len);
+      row_units(s, ri, va, vb);
+      if (ri.ok && qsl == nullptr && ri.seq_len == 0) {
+        T* o = out + static_cast<size_t>(r) * s.num_q_heads * s.head_dim;
+        for (int i = 0; i < s.num_q_heads * s.head_dim; ++i) o[i] = from_f32<T>(0.f);
+      }
+    }
+    int xa = va, xb = vb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, xa, o);
+      const int yb = __shfl_up_sync(0xffffffffu, xb, o);
+      if (lane >= o) {
+        xa += ya;
+        xb += yb;
+      }
+    }
+    if (lane == 31) {
+      warp_tot[0][warp] = xa;
+      warp_tot[1][warp] = xb;
+    }
+    __syncthreads();
+    if (warp < 2) {
+      int t = warp_tot[warp][lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      warp_tot[warp][lane] = t;
+    }
+    __syncthreads();
+    const int ea = carry_s[0] + xa - va + (warp > 0 ? warp_tot[0][warp - 1] : 0);
+    const int eb = carry_s[1] + xb - vb + (warp > 0 ? warp_tot[1][warp - 1] : 0);
+    if (r < s.num_seqs) {
+      w.row_a[r] = ea;
+      w.row_b[r] = eb;
+    }
+    __syncthreads();
+    if (tid == 1023) {
+      carry_s[0] = ea + va;
+      carry_s[1] = eb + vb;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    w.row_a[s.num_seqs] = carry_s[0];
+    w.row_b[s.num_seqs] = carry_s[1];
+    w.sched->next = 0;
+    w.sched->total_a = carry_s[0];
+    w.sched->total_b = carry_s[1];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue of one unit, run by the `nthreads` consumer threads of a CTA: merge
+// NW warps' states per tile row (cm/cl: running max in log2 units and sum; co:
+// unnormalised accumulators) and write the output row directly if its keys fit
+// one partition, else this partition's partial (normalised o, log2-sum-exp).
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__device__ __forceinline__ void store_row8(const Shape& s, T* __restrict__ out, int token,
+                                           int head, int c, const float (&acc)[8], float inv) {
+  T* o = out + (static_cast<size_t>(token) * s.num_q_heads + head) * D + c * 8;
+  if constexpr (sizeof(T) == 2) {
+    uint4 v;
+    v.x = pack2<T>(acc[0] * inv, acc[1] * inv);
+    v.y = pack2<T>(acc[2] * inv, acc[3] * inv);
+    v.z = pack2<T>(acc[4] * inv, acc[5] * inv);
+    v.w = pack2<T>(acc[6] * inv, acc[7] * inv);
+    *reinterpret_cast<uint4*>(o) = v;
+  } else {
+    *reinterpret_cast<float4*>(o) =
+        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<float4*>(o + 4) =
+        make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  }
+}
+
 template <typename T, int D, int NW>
-__device__ __forceinline__ void combine_and_store(const Shape& s, const Unit& u, float* cm,
-                                                  float* cl, float (*co)[kRows][D + 8],
-                                                  T* __restrict__ out, float* __restrict__ part_o,
-                                                  float* __restrict__ part_lse, int tid) {
+__device__ __forceinline__ void epilogue(const Shape& s, const Unit& u, const float* cm,
+                                         const float* cl, const float (*co)[kRows][D + 8],
+                                         T* __restrict__ out, const Work& w, int tid,
+                                         int nthreads) {
   constexpr int kChunks = D / 8;
-  for (int task = tid; task < kRows * kChunks; task += NW * 32) {
+  for (int task = tid; task < kRows * kChunks; task += nthreads) {
     const int r = task / kChunks, c = task % kChunks;
     const int i = r / s.gs, g = r % s.gs;
     if (i >= u.nq || g >= u.rows) continue;
-    const int limit = u.lim0 + i;
-    const int parts = parts_for(limit);
+    const int parts = parts_for(u.lim0 + i);
     if (u.p >= parts) continue;  // no key of this partition is visible to the row
     float mx = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) mx = fmaxf(mx, cm[w * kRows + r]);
+    for (int q = 0; q < NW; ++q) mx = fmaxf(mx, cm[q * kRows + r]);
     float L = 0.f;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float f = exp2f(cm[w * kRows + r] - mx);
-      L += f * cl[w * kRows + r];
-      const float4 a = *reinterpret_cast<const float4*>(&co[w][r][c * 8]);
-      const float4 b = *reinterpret_cast<const float4*>(&co[w][r][c * 8 + 4]);
+    for (int q = 0; q < NW; ++q) {
+      const float f = exp2f(cm[q * kRows + r] - mx);
+      L += f * cl[q * kRows + r];
+      const float4 a = *reinterpret_cast<const float4*>(&co[q][r][c * 8]);
+      const float4 b = *reinterpret_cast<const float4*>(&co[q][r][c * 8 + 4]);
       acc[0] += f * a.x; acc[1] += f * a.y; acc[2] += f * a.z; acc[3] += f * a.w;
       acc[4] += f * b.x; acc[5] += f * b.y; acc[6] += f * b.z; acc[7] += f * b.w;
     }
@@ -247,97 +358,17 @@ __device__ __forceinline__ void combine_and_store(const Shape& s, const Unit& u,
     const int token = u.token0 + i;
     const int head = u.head0 + g;
     if (parts == 1) {
-      T* o = out + (static_cast<size_t>(token) * s.num_q_heads + head) * D + c * 8;
-      if constexpr (sizeof(T) == 2) {
-        uint4 v;
-        v.x = pack2<T>(acc[0] * inv, acc[1] * inv);
-        v.y = pack2<T>(acc[2] * inv, acc[3] * inv);
-        v.z = pack2<T>(acc[4] * inv, acc[5] * inv);
-        v.w = pack2<T>(acc[6] * inv, acc[7] * inv);
-        *reinterpret_cast<uint4*>(o) = v;
-      } else {
-        *reinterpret_cast<float4*>(o) =
-            make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-        *reinterpret_cast<float4*>(o + 4) =
-            make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-      }
+      store_row8<T, D>(s, out, token, head, c, acc, inv);
     } else {
       const size_t slot = (static_cast<size_t>(token) * s.num_q_heads + head) * s.p_stride + u.p;
-      float* po = part_o + slot * D + c * 8;
+      float* po = w.part_o + slot * D + c * 8;
       *reinterpret_cast<float4*>(po) =
           make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
       *reinterpret_cast<float4*>(po + 4) =
           make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-      if (c == 0) part_lse[slot] = L > 0.f ? mx + log2f(L) : -INFINITY;
+      if (c == 0) w.part_lse[slot] = L > 0.f ? mx + log2f(L) : -INFINITY;
     }
   }
-}
-
-// ---------------------------------------------------------------------------
-// Split-K reduce: for every (query token, head) whose keys span more than one
-// partition, merge the partials by log-sum-exp:
-//   M = max_p lse_p,  w_p = 2^(lse_p - M),  out = sum_p w_p o_p / sum_p w_p.
-// One warp per (token, head).
-// ---------------------------------------------------------------------------
-template <typename T, int D>
-__global__ void __launch_bounds__(256) reduce_kernel(Shape s, const int* __restrict__ qsl,
-                                                     const int* __restrict__ seq_lens,
-                                                     const float* __restrict__ part_o,
-                                                     const float* __restrict__ part_lse,
-                                                     T* __restrict__ out) {
-  const int lane = threadIdx.x & 31;
-  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int token = static_cast<int>(gw / s.num_q_heads);
-  const int head = static_cast<int>(gw % s.num_q_heads);
-  if (token >= s.total_q) return;
-  int row = token;
-  if (qsl) {  // the request owning this token
-    int lo = 0, hi = s.num_seqs - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (qsl[mid] <= token)
-        lo = mid;
-      else
-        hi = mid - 1;
-    }
-    row = lo;
-  }
-  const RowInfo ri = load_row(s, qsl, seq_lens, row);
-  if (!ri.ok || ri.q_len == 0) return;
-  const int limit = ri.seq_len - ri.q_len + (token - ri.token0) + 1;
-  const int parts = parts_for(limit);
-  if (parts <= 1) return;
-  const size_t base = (static_cast<size_t>(token) * s.num_q_heads + head) * s.p_stride;
-  float mx = -INFINITY;
-  for (int p = lane; p < parts; p += 32) mx = fmaxf(mx, part_lse[base + p]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  constexpr int kPer = D / 32;  // dims per lane
-  float acc[kPer];
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  for (int p0 = 0; p0 < parts; p0 += 32) {
-    const int p = p0 + lane;
-    const float w = p < parts ? exp2f(part_lse[base + p] - mx) : 0.f;
-    const int n = min(32, parts - p0);
-    for (int j = 0; j < n; ++j) {
-      const float wj = __shfl_sync(0xffffffffu, w, j);
-      wsum += wj;
-      const float* po = part_o + (base + p0 + j) * D + lane * kPer;
-      if constexpr (kPer == 4) {
-        const float4 a = *reinterpret_cast<const float4*>(po);
-        acc[0] += wj * a.x; acc[1] += wj * a.y; acc[2] += wj * a.z; acc[3] += wj * a.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) acc[e] += wj * po[e];
-      }
-    }
-  }
-  const float inv = 1.f / wsum;
-  T* o = out + (static_cast<size_t>(token) * s.num_q_heads + head) * D + lane * kPer;
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) o[e] = from_f32<T>(acc[e] * inv);
 }
 
 }  // namespace pa

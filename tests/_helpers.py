@@ -41,18 +41,26 @@ def gpu_cache_write(b: PagedBatch):
     return kc, vc
 
 
+def poisoned_workspace(nbytes: int, device) -> torch.Tensor:
+    """A workspace whose every byte is 0xFF (NaN as fp32, -1 as int32), so a
+    kernel that reads scratch before writing it in the same call shows it."""
+    ws = pa.alloc_workspace(nbytes, device)
+    ws.fill_(0xFF)
+    return ws
+
+
 def gpu_attention(b: PagedBatch, kc, vc, varlen: bool | None = None, out=None):
     varlen = (not b.is_decode) if varlen is None else varlen
     if out is None:
         out = torch.full_like(b.q, float("nan"))
     if varlen:
-        ws = pa.alloc_workspace(pa.pa_varlen_workspace_size(
+        ws = poisoned_workspace(pa.pa_varlen_workspace_size(
             b.num_seqs, b.total_q, b.num_q_heads, b.num_kv_heads, b.head_dim, b.max_query_len,
             b.max_seq_len), b.q.device)
         pa.pa_varlen(out, b.q, kc, vc, b.block_tables, b.query_start_loc, b.seq_lens,
                      b.max_query_len, b.max_seq_len, b.scale, ws)
     else:
-        ws = pa.alloc_workspace(pa.pa_decode_workspace_size(
+        ws = poisoned_workspace(pa.pa_decode_workspace_size(
             b.num_seqs, b.num_q_heads, b.num_kv_heads, b.head_dim, b.max_seq_len), b.q.device)
         pa.pa_decode(out, b.q, kc, vc, b.block_tables, b.seq_lens, b.max_seq_len, b.scale, ws)
     pa.pa_get_device_error()

@@ -76,16 +76,29 @@ def _a256(x):
     return (x + 255) // 256 * 256
 
 
+def _layout(S, T, hq, hkv, d, max_len, varlen):
+    """Mirror of the workspace layout documented in csrc/pa_api.cu."""
+    g = hq // hkv
+    ns = -(-g // 16)
+    p = -(-max_len // 512) if max_len > 0 else 1
+    off = _a256(16 + 2 * (S + 1) * 4)                 # schedule block + two row prefixes
+    if p > 1:
+        off = _a256(off + T * hq * p * 4)             # partial log-sum-exp
+        off = _a256(off + T * hq * p * d * 4)         # partial outputs
+    return off
+
+
 def test_workspace_sizes(lib):
-    # one partition (<= 512 tokens): only the schedule, S+1 ints rounded to 256 B
-    assert pa.pa_decode_workspace_size(64, 32, 32, 128, 512) == _a256(65 * 4)
-    # S=8, Hq=64, 64 partitions of 512: LSE [8*64*64] fp32 + O [8*64*64*128] fp32
-    ws = pa.pa_decode_workspace_size(8, 64, 8, 128, 32768)
-    assert ws == _a256(9 * 4) + _a256(8 * 64 * 64 * 4) + _a256(8 * 64 * 64 * 128 * 4)
+    assert pa.pa_decode_workspace_size(64, 32, 32, 128, 512) == _layout(64, 64, 32, 32, 128, 512,
+                                                                        False)
+    assert pa.pa_decode_workspace_size(8, 64, 8, 128, 32768) == _layout(8, 8, 64, 8, 128, 32768,
+                                                                        False)
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 100) == 0
-    # varlen: total_q=10 rows x Hq=4 x 2 partitions
-    vs = pa.pa_varlen_workspace_size(3, 10, 4, 2, 64, 8, 1024)
-    assert vs == _a256(4 * 4) + _a256(10 * 4 * 2 * 4) + _a256(10 * 4 * 2 * 64 * 4)
+    assert pa.pa_varlen_workspace_size(3, 10, 4, 2, 64, 8, 1024) == _layout(3, 10, 4, 2, 64, 1024,
+                                                                            True)
+    # the split-K partials dominate: [T][Hq][P] lse + [T][Hq][P][D] outputs
+    big = pa.pa_decode_workspace_size(8, 64, 8, 128, 32768)
+    assert big >= 8 * 64 * 64 * 129 * 4
 
 
 def _decode(lib, **kw):
