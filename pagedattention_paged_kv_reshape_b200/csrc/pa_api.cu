@@ -15,6 +15,7 @@
 
 #include "pa_attn_mma.cuh"
 #include "pa_attn_simt.cuh"
+#include "pa_chunk_tc.cuh"
 #include "pa_reduce.cuh"
 #include "pa_reshape.cuh"
 #include "pa_sched.cuh"
@@ -172,12 +173,22 @@ constexpr int kStages = PA_STAGES;
 
 struct Plan {
   pa::Shape s;
-  size_t off_row_a, off_row_b, off_part_lse, off_part_o, bytes;
+  size_t off_row_a, off_row_b, off_chunk, off_part_lse, off_part_o, bytes;
   long long max_units;
+  int chunk_qt;         // query tokens per tcgen05 chunk tile (0: no chunk kernel possible)
+  long long chunk_cap;  // capacity of the chunk-tile list
 };
 
+// The tcgen05 chunk kernel tiles 128 rows = (128 / gs) query tokens x gs heads.
+int chunk_tile_tokens(int group) {
+  const int gs = group < pa::kRows ? group : pa::kRows;
+  return (gs == 1 || gs == 2 || gs == 4 || gs == 8 || gs == 16) ? pa::kTcRows / gs : 0;
+}
+
 // Workspace layout: the schedule block (Sched), the two per-row unit prefixes,
-// then the split-K partials (only when some context can exceed one partition).
+// the chunk-tile list (varlen batches whose head grouping the tcgen05 kernel
+// supports), then the split-K partials (only when some context can exceed
+// one partition).
 Plan make_plan(int num_seqs, int total_q, int hq, int hkv, int d, int max_len, bool varlen) {
   Plan p{};
   pa::Shape& s = p.s;
@@ -191,10 +202,18 @@ Plan make_plan(int num_seqs, int total_q, int hq, int hkv, int d, int max_len, b
   s.head_dim = d;
   s.total_q = total_q;
   s.p_stride = max_len > 0 ? (max_len + pa::kPart - 1) / pa::kPart : 1;
+  s.chunk_qt = 0;
+  s.chunk_cap = 0;
   const size_t rows = static_cast<size_t>(num_seqs) + 1;
   p.off_row_a = sizeof(pa::Sched);
   p.off_row_b = p.off_row_a + rows * 4;
   size_t off = align256(p.off_row_b + rows * 4);
+  p.off_chunk = off;
+  p.chunk_qt = varlen ? chunk_tile_tokens(s.group) : 0;
+  if (p.chunk_qt > 0) {  // a chunk row of q_len tokens yields ceil(q_len / qt) <= 2 q_len / qt tiles
+    p.chunk_cap = 2LL * ((total_q + p.chunk_qt - 1) / p.chunk_qt) + 1;
+    off = align256(off + static_cast<size_t>(p.chunk_cap) * sizeof(int2));
+  }
   p.off_part_lse = off;
   p.off_part_o = off;
   if (s.p_stride > 1) {
@@ -218,6 +237,7 @@ pa::Work carve(void* workspace, const Plan& p) {
   w.sched = reinterpret_cast<pa::Sched*>(ws);
   w.row_a = reinterpret_cast<int*>(ws + p.off_row_a);
   w.row_b = reinterpret_cast<int*>(ws + p.off_row_b);
+  w.chunk_list = reinterpret_cast<int2*>(ws + p.off_chunk);
   w.part_lse = reinterpret_cast<float*>(ws + p.off_part_lse);
   w.part_o = reinterpret_cast<float*>(ws + p.off_part_o);
   return w;
@@ -316,6 +336,32 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   return PA_OK;
 }
 
+template <typename T, int D>
+pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
+  using L = pa::TcLayout<D>;
+  auto kern = pa::chunk_tc_kernel<T, D>;
+  int occ = 0;
+  cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk kernel set-up");
+  CUtensorMap tk, tv, tq;
+  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * pa::kBlock;
+  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, pa::kBlock);
+  if (st != PA_OK) return st;
+  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, pa::kBlock);
+  if (st != PA_OK) return st;
+  st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.chunk_qt);
+  if (st != PA_OK) return st;
+  long long grid = sm_count();
+  const long long items = p.chunk_cap * a.num_kv_heads * p.s.ns;
+  if (items < grid) grid = items;
+  if (grid < 1) grid = 1;
+  e = launch_pdl(kern, static_cast<unsigned>(grid), L::kThreads, L::kSmem, a.stream, tk, tv, tq,
+                 p.s, static_cast<T*>(a.out), a.block_tables, a.qsl, a.seq_lens, w,
+                 static_cast<float>(a.scale * M_LOG2E));
+  if (e != cudaSuccess) return cuda_fail(e, "chunk kernel launch");
+  return PA_OK;
+}
+
 template <typename T>
 pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   const pa::Work w = carve(a.workspace, p);
@@ -332,7 +378,14 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   } else {
     st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, w) : launch_simt<T, 64>(a, p, w);
   }
-  if (st != PA_OK || p.s.p_stride <= 1) return st;
+  if (st != PA_OK) return st;
+  if constexpr (sizeof(T) == 2) {
+    if (p.s.chunk_qt > 0) {
+      st = a.head_dim == 128 ? launch_chunk<T, 128>(a, p, w) : launch_chunk<T, 64>(a, p, w);
+      if (st != PA_OK) return st;
+    }
+  }
+  if (p.s.p_stride <= 1) return PA_OK;
   const long long warps = static_cast<long long>(a.total_q) * a.num_q_heads;
   const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
   e = a.head_dim == 128
@@ -369,6 +422,13 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
       return fail(PA_ERR_UNSUPPORTED, "tensor-core path needs bf16 or f16 (got fp32)");
   }
   const bool use_mma = sixteen && path != PA_PATH_SIMT;
+  // Prefill-chunk rows (q_len >= one 128-row tile) go to the tcgen05 kernel
+  // unless a family without it was forced.
+  p.s.chunk_qt = (use_mma && path != PA_PATH_MMA && p.chunk_qt > 0 &&
+                  a.max_query_len >= p.chunk_qt)
+                     ? p.chunk_qt
+                     : 0;
+  p.s.chunk_cap = static_cast<int>(p.chunk_cap);
   switch (a.dtype) {
     case PA_BF16: return run_typed<__nv_bfloat16>(a, p, use_mma);
     case PA_F16: return run_typed<__half>(a, p, use_mma);

@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(256) reduce_kernel(Shape s, const int* __restr
     row = lo;
   }
   const RowInfo ri = load_row(s, qsl, seq_lens, row);
-  if (!ri.ok || ri.q_len == 0) return;
+  if (!ri.ok || ri.q_len == 0 || is_chunk_row(s, ri)) return;  // chunk rows: written directly
   const int parts = parts_for(ri.seq_len - ri.q_len + (token - ri.token0) + 1);
   if (parts <= 1) return;
   const size_t base = (static_cast<size_t>(token) * s.num_q_heads + head) * s.p_stride;

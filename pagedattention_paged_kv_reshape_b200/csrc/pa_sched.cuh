@@ -45,14 +45,17 @@ struct Shape {
   int max_query_len;
   int total_q;
   int p_stride;     // partitions per (token, head) in the workspace
+  int chunk_qt;     // > 0: rows with q_len >= chunk_qt go to the tcgen05 chunk kernel
+                    // as tiles of chunk_qt query tokens (128 / gs)
+  int chunk_cap;    // capacity of the chunk-tile list
 };
 
 // Schedule block at the start of the workspace.
 struct Sched {
-  int next;      // next unit index to claim
-  int total_a;   // class-A units
-  int total_b;   // class-B units
-  int pad;
+  int next;         // next unit index to claim
+  int total_a;      // class-A units
+  int total_b;      // class-B units
+  int chunk_count;  // entries of the chunk-tile list
 };
 
 // Pointers into the workspace.
@@ -60,6 +63,7 @@ struct Work {
   Sched* sched;
   int* row_a;       // [num_seqs + 1] prefix of class-A units
   int* row_b;       // [num_seqs + 1] prefix of class-B units
+  int2* chunk_list; // (row, first query) of every tcgen05 chunk tile
   float* part_lse;  // [total_q][Hq][p_stride]
   float* part_o;    // [total_q][Hq][p_stride][D]
 };
@@ -93,9 +97,13 @@ __device__ __forceinline__ RowInfo load_row(const Shape& s, const int* __restric
 __device__ __forceinline__ int head_units(const Shape& s) { return s.num_kv_heads * s.ns; }
 
 // Units of each class in a row.
+__device__ __forceinline__ bool is_chunk_row(const Shape& s, const RowInfo& ri) {
+  return s.chunk_qt > 0 && ri.q_len >= s.chunk_qt;
+}
+
 __device__ __forceinline__ void row_units(const Shape& s, const RowInfo& ri, int& a, int& b) {
   a = b = 0;
-  if (!ri.ok || ri.q_len == 0) return;
+  if (!ri.ok || ri.q_len == 0 || is_chunk_row(s, ri)) return;
   const int items = ceil_div(ri.q_len, s.qpt);
   const int parts = ceil_div(ri.seq_len, kPart);
   b = items * head_units(s);
@@ -224,7 +232,8 @@ __device__ __forceinline__ int locate_unit_thread(const Shape& s, const Work& w,
 
 // ---------------------------------------------------------------------------
 // Prep kernel: validate rows, write the two prefix sums and the totals, zero
-// the claim counter, zero the output rows of empty decode requests.  One CTA of 1024 threads.  It lets the attention kernel
+// the claim counter, list the tiles of chunk rows for the tcgen05 kernel,
+// zero the output rows of empty decode requests.  One CTA of 1024 threads.  It lets the attention kernel
 // launch at once (programmatic dependent launch); that kernel waits for this
 // grid to complete before it reads any of the above.
 // ---------------------------------------------------------------------------
@@ -238,6 +247,7 @@ __global__ void __launch_bounds__(1024) schedule_kernel(Shape s, const int* __re
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
     carry_s[0] = carry_s[1] = 0;
+    w.sched->chunk_count = 0;
     if (qsl && (qsl[0] != 0 || qsl[s.num_seqs] != s.total_q))
       report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, -1, qsl[s.num_seqs]);
   }
@@ -249,6 +259,15 @@ __global__ void __launch_bounds__(1024) schedule_kernel(Shape s, const int* __re
       const RowInfo ri = load_row(s, qsl, seq_lens, r);
       if (!ri.ok) report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, r, ri.seq_len);
       row_units(s, ri, va, vb);
+      if (ri.ok && is_chunk_row(s, ri)) {
+        const int n = ceil_div(ri.q_len, s.chunk_qt);
+        const int at = atomicAdd(&w.sched->chunk_count, n);
+        if (at + n <= s.chunk_cap) {
+          for (int j = 0; j < n; ++j) w.chunk_list[at + j] = make_int2(r, j * s.chunk_qt);
+        } else {  // rows overlap in query_start_loc: more tiles than tokens allow
+          report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, r, at + n);
+        }
+      }
       if (ri.ok && qsl == nullptr && ri.seq_len == 0) {
         T* o = out + static_cast<size_t>(r) * s.num_q_heads * s.head_dim;
         for (int i = 0; i < s.num_q_heads * s.head_dim; ++i) o[i] = from_f32<T>(0.f);
@@ -299,6 +318,8 @@ __global__ void __launch_bounds__(1024) schedule_kernel(Shape s, const int* __re
     w.sched->total_a = carry_s[0];
     w.sched->total_b = carry_s[1];
   }
+  __syncthreads();
+  if (tid == 0 && w.sched->chunk_count > s.chunk_cap) w.sched->chunk_count = s.chunk_cap;
 }
 
 // ---------------------------------------------------------------------------

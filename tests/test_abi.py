@@ -82,6 +82,10 @@ def _layout(S, T, hq, hkv, d, max_len, varlen):
     ns = -(-g // 16)
     p = -(-max_len // 512) if max_len > 0 else 1
     off = _a256(16 + 2 * (S + 1) * 4)                 # schedule block + two row prefixes
+    gs = min(g, 16)
+    if varlen and gs in (1, 2, 4, 8, 16):             # tcgen05 chunk-tile list, int2 entries
+        qt = 128 // gs
+        off = _a256(off + (2 * -(-T // qt) + 1) * 8)
     if p > 1:
         off = _a256(off + T * hq * p * 4)             # partial log-sum-exp
         off = _a256(off + T * hq * p * d * 4)         # partial outputs

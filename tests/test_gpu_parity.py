@@ -140,26 +140,49 @@ def test_decode_empty_context_is_zero_row():
 # ---------------------------------------------------------------------------
 
 VARLEN_CASES = [
-    # (seq_len, q_len) rows, hq, hkv, d, dtype
+    # (seq_len, q_len) rows, hq, hkv, d, dtype.  With the default path, rows of
+    # at least 128 / min(group, 16) new tokens run on the tcgen05 chunk kernel.
     ([(700, 37), (1, 1), (33, 1), (64, 64), (2000, 1), (530, 0), (1300, 300)], 32, 8, 128, "bf16"),
     ([(1, 1), (600, 600), (90, 5)], 8, 8, 64, "f16"),
     ([(2048, 512), (100, 1), (4096, 1)], 16, 2, 128, "bf16"),
-    ([(45, 45), (1100, 13), (3, 1)], 6, 2, 128, "bf16"),
+    ([(45, 45), (1100, 13), (3, 1)], 6, 2, 128, "bf16"),          # group 3: no tcgen05 tiles
     ([(520, 20), (17, 17), (2, 1)], 4, 4, 64, "f32"),
+    ([(300, 40), (1000, 129), (200, 200), (5, 1)], 32, 8, 64, "bf16"),  # ragged chunk tiles
+    ([(1000, 129), (129, 129), (77, 1)], 4, 4, 128, "f16"),        # MHA: 128-token tiles
+    ([(600, 70), (64, 1), (900, 9)], 64, 2, 128, "bf16"),          # group 32: 16-head slices
+    ([(2500, 256), (300, 1)], 16, 2, 64, "f16"),                   # group 8, head_dim 64
 ]
 
 
-@pytest.mark.parametrize("path", ["auto", "simt"])
+@pytest.mark.parametrize("path", ["auto", "mma", "simt"])
 @pytest.mark.parametrize("case", range(len(VARLEN_CASES)))
 def test_varlen_matches_oracle(case, path):
     rows, hq, hkv, d, dtype = VARLEN_CASES[case]
     if path == "simt":
         pa.pa_set_path(pa.Path.SIMT)
+    elif path == "mma":
+        if dtype == "f32":
+            pytest.skip("tensor-core paths need 16-bit inputs")
+        pa.pa_set_path(pa.Path.MMA)
     b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
                       head_dim=d, dtype=dtype, seed=100 + case, device=DEV, pool_factor=1.2)
     out, _, _ = gpu_step(b, varlen=True)
     ref, _, _ = oracle_step(b, varlen=True)
     assert_close(out, ref, dtype, f"varlen case {case} ({path})")
+
+
+def test_chunk_kernel_agrees_with_decode_kernel_tiles():
+    """The tcgen05 chunk tiles and the decode kernel's 16-row tiles compute the
+    same rows; both are within tolerance of each other as well as the oracle."""
+    b = W.build_batch([W.Request(s, q) for s, q in [(1536 + 512, 512), (800, 1)]],
+                      num_q_heads=32, num_kv_heads=8, head_dim=128, dtype="bf16", seed=7,
+                      device=DEV, pool_factor=1.1)
+    kc, vc = gpu_cache_write(b)
+    tc = gpu_attention(b, kc, vc, varlen=True)
+    pa.pa_set_path(pa.Path.MMA)
+    mma = gpu_attention(b, kc, vc, varlen=True)
+    assert_close(tc, f64(mma), "bf16", "tcgen05 vs mma tiles")
+    assert torch.equal(tc[-1], mma[-1])   # the decode row takes the same kernel on both
 
 
 def test_varlen_decode_rows_equal_decode():
