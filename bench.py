@@ -53,6 +53,9 @@ def parse_args():
     return ap.parse_args()
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -61,6 +64,14 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak() -> float:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return FALLBACK_BF16_TFLOPS
 
 
 # Sources the attention kernel is compiled from (its traffic record is keyed to them).
@@ -437,8 +448,9 @@ def run_ours(args):
     }
 
     if not args.no_per_config:
+        tensor_peak = measured_tensor_peak()
         per = {}
-        for name in ("gqa_bs256", "long_32k", "mixed_2048"):
+        for name in ("gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512"):
             if name == args.workload:
                 continue
             del b
@@ -456,6 +468,13 @@ def run_ours(args):
             if name == "mixed_2048":
                 ent["unique_vs_logical_kv"] = [a2["kv_unique"], a2["kv_logical"]]
                 ent["chunk_gflop"] = round(A.chunk_flops(b) / 1e9, 2)
+            if name == "prefill_16x512":   # dense causal chunks: a tensor-core roofline
+                tflops = A.chunk_flops(b) / (attn / 1e3) / 1e12
+                ent = {"chunk_tflops": round(tflops, 1),
+                       "pct_of_bf16_peak": round(100 * tflops / tensor_peak, 1),
+                       "attention_ms": round(attn, 4), "chunk_gflop": round(A.chunk_flops(b) / 1e9, 1),
+                       "peak_kind": "measured bf16_tflops (burst)",
+                       "tokens_per_s": round(b.total_q / (attn / 1e3), 1)}
             per[name] = ent
         result["per_config"] = per
 

@@ -386,13 +386,28 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
     }
   }
   if (p.s.p_stride <= 1) return PA_OK;
-  const long long warps = static_cast<long long>(a.total_q) * a.num_q_heads;
-  const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+  // one CTA per (request, 16-token slice, 8 heads) of the rows the attention kernels split
+  int max_q = a.qsl ? a.max_query_len : 1;
+  if (p.s.chunk_qt > 0 && max_q >= p.s.chunk_qt) max_q = p.s.chunk_qt - 1;
+  const int slices = (max_q + pa::kReduceTokens - 1) / pa::kReduceTokens;
+  const dim3 grid(static_cast<unsigned>(a.num_seqs),
+                  static_cast<unsigned>(slices < 65535 ? slices : 65535),
+                  static_cast<unsigned>((a.num_q_heads + 7) / 8));
+  if (grid.y == 0) return PA_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   e = a.head_dim == 128
-          ? launch_pdl(pa::reduce_kernel<T, 128>, blocks, 256, 0, a.stream, p.s, a.qsl,
-                       a.seq_lens, w, static_cast<T*>(a.out))
-          : launch_pdl(pa::reduce_kernel<T, 64>, blocks, 256, 0, a.stream, p.s, a.qsl,
-                       a.seq_lens, w, static_cast<T*>(a.out));
+          ? cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 128>, p.s, a.qsl, a.seq_lens, w,
+                               static_cast<T*>(a.out))
+          : cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 64>, p.s, a.qsl, a.seq_lens, w,
+                               static_cast<T*>(a.out));
   if (e != cudaSuccess) return cuda_fail(e, "reduce kernel launch");
   return PA_OK;
 }

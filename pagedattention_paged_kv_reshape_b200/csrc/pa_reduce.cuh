@@ -3,18 +3,24 @@
 //   M = max_p lse_p,  w_p = 2^(lse_p - M),  out = sum_p w_p o_p / sum_p w_p
 // (lse_p in log2 units, o_p already normalised by its partition's sum).
 //
-// One warp per (query token, head); each lane owns D/32 consecutive dims.  The
+// One CTA per (request, slice of kReduceTokens query tokens, group of eight
+// query heads; CTAs stride over the slices of longer rows): it reads the
+// request's metadata once; each warp merges one head for the slice's tokens,
+// each lane owning D/32 dims.  The
 // loop over partitions is unrolled so that eight partitions' loads are in
-// flight at once: at 64 partitions (32K-token contexts) a loop that waited on
-// each load in turn would be bound by L2 latency.  The kernel is launched
-// behind the attention kernel with programmatic dependent launch (its CTAs may
-// be scheduled as attention CTAs retire) and waits for that grid to complete
-// before reading the partials.
+// flight at once (32K-token contexts have 64 partitions).  Rows handled by the
+// tcgen05 chunk kernel are skipped: that kernel writes them directly.
+//
+// The kernel is launched behind the attention kernels with programmatic
+// dependent launch (its CTAs may be scheduled as attention CTAs retire) and
+// waits for those grids to complete before reading the partials.
 #pragma once
 
 #include "pa_sched.cuh"
 
 namespace pa {
+
+constexpr int kReduceTokens = 16;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) reduce_kernel(Shape s, const int* __restrict__ qsl,
@@ -23,70 +29,63 @@ __global__ void __launch_bounds__(256) reduce_kernel(Shape s, const int* __restr
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kPer = D / 32;  // dims per lane
   constexpr int kUnroll = 8;
-  const int lane = threadIdx.x & 31;
-  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int token = static_cast<int>(gw / s.num_q_heads);
-  const int head = static_cast<int>(gw % s.num_q_heads);
-  if (token >= s.total_q) return;
-  int row = token;
-  if (qsl) {  // the request owning this token
-    int lo = 0, hi = s.num_seqs - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (__ldg(qsl + mid) <= token)
-        lo = mid;
-      else
-        hi = mid - 1;
-    }
-    row = lo;
-  }
+  const int row = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const RowInfo ri = load_row(s, qsl, seq_lens, row);
-  if (!ri.ok || ri.q_len == 0 || is_chunk_row(s, ri)) return;  // chunk rows: written directly
-  const int parts = parts_for(ri.seq_len - ri.q_len + (token - ri.token0) + 1);
-  if (parts <= 1) return;
-  const size_t base = (static_cast<size_t>(token) * s.num_q_heads + head) * s.p_stride;
-  const float* lse = w.part_lse + base;
-  float mx = -INFINITY;
-  for (int p = lane; p < parts; p += 32) mx = fmaxf(mx, lse[p]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float acc[kPer];
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  const float* po = w.part_o + base * D + lane * kPer;
-  for (int p0 = 0; p0 < parts; p0 += 32) {
-    const int n = min(32, parts - p0);
-    const float wl = lane < n ? exp2f(lse[p0 + lane] - mx) : 0.f;  // weight of partition p0+lane
-    for (int j0 = 0; j0 < n; j0 += kUnroll) {
-      float v[kUnroll][kPer];
-#pragma unroll
-      for (int j = 0; j < kUnroll; ++j) {  // issue every load first
-        const int jj = min(j0 + j, n - 1);
-        const float* src = po + static_cast<size_t>(p0 + jj) * D;
-        if constexpr (kPer == 4) {
-          const float4 a = *reinterpret_cast<const float4*>(src);
-          v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
-        } else {
-          const float2 a = *reinterpret_cast<const float2*>(src);
-          v[j][0] = a.x; v[j][1] = a.y;
+  if (!ri.ok || ri.q_len == 0 || is_chunk_row(s, ri)) return;
+  const int head = blockIdx.z * 8 + warp;
+  if (head >= s.num_q_heads) return;
+  for (int t0 = blockIdx.y * kReduceTokens; t0 < ri.q_len; t0 += gridDim.y * kReduceTokens) {
+    const int nt = min(kReduceTokens, ri.q_len - t0);
+    for (int ti = t0; ti < t0 + nt; ++ti) {
+      const int parts = parts_for(ri.seq_len - ri.q_len + ti + 1);
+      if (parts <= 1) continue;  // written directly by the attention kernel
+      const int token = ri.token0 + ti;
+      const size_t base = (static_cast<size_t>(token) * s.num_q_heads + head) * s.p_stride;
+      const float* lse = w.part_lse + base;
+      float mx = -INFINITY;
+      for (int p = lane; p < parts; p += 32) mx = fmaxf(mx, lse[p]);
+  #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float acc[kPer];
+  #pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+      float wsum = 0.f;
+      const float* po = w.part_o + base * D + lane * kPer;
+      for (int p0 = 0; p0 < parts; p0 += 32) {
+        const int n = min(32, parts - p0);
+        const float wl = lane < n ? exp2f(lse[p0 + lane] - mx) : 0.f;  // weight of partition p0+lane
+        for (int j0 = 0; j0 < n; j0 += kUnroll) {
+          float v[kUnroll][kPer];
+  #pragma unroll
+          for (int j = 0; j < kUnroll; ++j) {  // issue every load first
+            const int jj = min(j0 + j, n - 1);
+            const float* src = po + static_cast<size_t>(p0 + jj) * D;
+            if constexpr (kPer == 4) {
+              const float4 a = *reinterpret_cast<const float4*>(src);
+              v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
+            } else {
+              const float2 a = *reinterpret_cast<const float2*>(src);
+              v[j][0] = a.x; v[j][1] = a.y;
+            }
+          }
+  #pragma unroll
+          for (int j = 0; j < kUnroll; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, wl, (j0 + j) & 31);
+            if (j0 + j < n) {
+              wsum += wj;
+  #pragma unroll
+              for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wj, v[j][e], acc[e]);
+            }
+          }
         }
       }
-#pragma unroll
-      for (int j = 0; j < kUnroll; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, wl, (j0 + j) & 31);
-        if (j0 + j < n) {
-          wsum += wj;
-#pragma unroll
-          for (int e = 0; e < kPer; ++e) acc[e] = fmaf(wj, v[j][e], acc[e]);
-        }
-      }
+      const float inv = 1.f / wsum;
+      T* o = out + (static_cast<size_t>(token) * s.num_q_heads + head) * D + lane * kPer;
+  #pragma unroll
+      for (int e = 0; e < kPer; ++e) o[e] = from_f32<T>(acc[e] * inv);
     }
   }
-  const float inv = 1.f / wsum;
-  T* o = out + (static_cast<size_t>(token) * s.num_q_heads + head) * D + lane * kPer;
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) o[e] = from_f32<T>(acc[e] * inv);
 }
 
 }  // namespace pa

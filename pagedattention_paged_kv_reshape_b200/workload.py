@@ -263,6 +263,13 @@ def mixed_requests(seed, decode_rows=1536, chunk_q=512, chunk_cached=1536, lo=64
     return [chunk] + reqs if chunk_first else reqs + [chunk]
 
 
+def prefill_requests(seed, rows=16, chunk_q=512, cached=1536):
+    """A prefill-heavy scheduler iteration: ``rows`` requests each running a
+    512-token causal chunk on 1536 cached tokens (chunked prefill of long
+    prompts); every row goes to the tensor-core chunk path."""
+    return [Request(cached + chunk_q, chunk_q) for _ in range(rows)]
+
+
 CONFIGS = {
     "tiny": dict(requests=tiny_requests, num_q_heads=4, num_kv_heads=4, head_dim=64,
                  dtype="f32", pool_blocks=64, kind="decode",
@@ -285,6 +292,10 @@ CONFIGS = {
                        about="2048-token budget: 512-query causal chunk on 1536 cached tokens + "
                              "1536 decode rows (ctx U[64,4096], half share a 512-token prefix), "
                              "32/8 heads, head_dim 128, bf16"),
+    "prefill_16x512": dict(requests=prefill_requests, num_q_heads=32, num_kv_heads=8,
+                           head_dim=128, dtype="bf16", pool_factor=1.0, kind="varlen",
+                           about="16 causal prefill chunks of 512 tokens on 1536 cached tokens, "
+                                 "32/8 heads, head_dim 128, bf16 (tensor-core chunk kernel)"),
 }
 
 
