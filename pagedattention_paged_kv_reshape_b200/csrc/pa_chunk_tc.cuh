@@ -9,11 +9,13 @@
 // * work item = (chunk row, tile of 128/gs query tokens x gs query heads =
 //   128 tile rows, KV head slice); a persistent grid walks the items listed
 //   by the prep kernel;
-// * Q (one 3-D TMA box) and K/V (eight 16-token TMA boxes per 128-key tile,
-//   a two-stage ring) land in shared memory with 128-byte swizzling, which is
-//   exactly the canonical K-major layout (Q, K, P) and MN-major layout (V) the
-//   tcgen05 shared-memory descriptors describe;
-// * one thread issues S = Q K^T (M=128, N=128, K=16 steps) into TMEM;
+// * Q (one 3-D TMA box) and K, V (eight 16-token TMA boxes per 128-key tile;
+//   a three-stage K ring and a two-stage V ring) land in shared memory with
+//   128-byte swizzling, which is exactly the canonical K-major layout (Q, K,
+//   P) and MN-major layout (V) the tcgen05 shared-memory descriptors describe;
+// * one thread issues S = Q K^T (M=128, N=128, K=16 steps) into one of two
+//   TMEM score buffers, two tiles ahead of the softmax, so the tensor core
+//   computes the next scores while the softmax warps work;
 // * four softmax warps read S with tcgen05.ld, one tile row per thread, apply
 //   the causal mask (key <= position) and the online softmax in the log2
 //   domain, and write P (rounded to the input type) to shared memory;
@@ -21,7 +23,7 @@
 //   softmax threads fold it into their fp32 row accumulators with the
 //   running rescale, and write the output row at the end.
 //
-// Every wait is bounded.  TMEM (256 columns) is freed on every path, after a
+// Every wait is bounded.  TMEM (512 columns) is freed on every path, after a
 // final commit has drained the MMAs this CTA issued.  The kernel is launched
 // behind the decode kernel with programmatic dependent launch so that it
 // fills that kernel's tail; it reads nothing the decode kernel writes, and it
@@ -36,31 +38,35 @@
 
 namespace pa {
 
-constexpr int kTcRows = 128;  // tile rows = TMEM lanes
-constexpr int kTcKeys = 128;  // keys per KV tile = 8 blocks
-constexpr int kTcStages = 2;
+constexpr int kTcRows = 128;   // tile rows = TMEM lanes
+constexpr int kTcKeys = 128;   // keys per KV tile = 8 blocks
+constexpr int kTcKStages = 3;  // K ring: a K tile is free once its QK^T has run
+constexpr int kTcVStages = 2;  // V ring: a V tile is free once its PV has run
 
 template <int D>
 struct TcLayout {
   static constexpr int kHalves = D / 64;           // 128-byte swizzle rows per token row
   static constexpr int kHalfBytes = 128 * 128;     // 128 rows x 128 B
   static constexpr int kQBytes = kHalves * kHalfBytes;
-  static constexpr int kKVBytes = kHalves * kHalfBytes;
+  static constexpr int kKVBytes = kHalves * kHalfBytes;  // one K or V tile
   static constexpr int kPBytes = 2 * kHalfBytes;   // 128 rows x 128 keys x 2 B
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kTcStages * kKVBytes;
-  static constexpr int kOffP = kOffV + kTcStages * kKVBytes;
+  static constexpr int kOffV = kOffK + kTcKStages * kKVBytes;
+  static constexpr int kOffP = kOffV + kTcVStages * kKVBytes;
   static constexpr int kOffBar = kOffP + kPBytes;
-  // qfull, qfree, kvfull[2], kvempty[2], sfull, pfull, pvfull, drain
-  static constexpr int kNumBars = 10;
+  // qfull, qfree, kfull[3], kempty[3], vfull[2], vempty[2], sfull[2], pfull, pvfull, drain
+  static constexpr int kNumBars = 2 + 2 * kTcKStages + 2 * kTcVStages + 2 + 3;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 12;
-  static constexpr int kSmem = kBytes + 1024;
+  // at least ~114 KB, so that a single CTA fits per SM and its TMEM
+  // allocation can never wait for another CTA's
+  static constexpr int kSmem = (kBytes + 1024) > 116 * 1024 ? (kBytes + 1024) : 116 * 1024;
   static constexpr int kThreads = 160;             // 4 softmax warps + 1 TMA/MMA warp
-  static constexpr uint32_t kTmemCols = 256;       // S in [0,128), O in [128, 128 + D)
+  static constexpr uint32_t kTmemCols = 512;       // S0 [0,128), S1 [128,256), O [256, 256 + D)
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "1 KB alignment");
+  static_assert(kBytes + 1024 <= 232448, "shared memory budget");
 };
 
 template <typename T, int D>
@@ -80,9 +86,13 @@ __global__ void __launch_bounds__(160, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + L::kOffBar;
   const uint32_t qfull = bar0, qfree = bar0 + 8;
-  auto kvfull = [&](int st) { return bar0 + 16u + 8u * st; };
-  auto kvempty = [&](int st) { return bar0 + 32u + 8u * st; };
-  const uint32_t sfull = bar0 + 48, pfull = bar0 + 56, pvfull = bar0 + 64, drain = bar0 + 72;
+  auto kfull = [&](int st) { return bar0 + 16u + 8u * st; };
+  auto kempty = [&](int st) { return bar0 + 16u + 8u * (kTcKStages + st); };
+  auto vfull = [&](int st) { return bar0 + 16u + 8u * (2 * kTcKStages + st); };
+  auto vempty = [&](int st) { return bar0 + 16u + 8u * (2 * kTcKStages + kTcVStages + st); };
+  auto sfull = [&](int b) { return bar0 + 16u + 8u * (2 * kTcKStages + 2 * kTcVStages + b); };
+  const uint32_t pfull = bar0 + 16u + 8u * (2 * kTcKStages + 2 * kTcVStages + 2);
+  const uint32_t pvfull = pfull + 8, drain = pfull + 16;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
   const uint32_t q_smem = sbase + L::kOffQ;
@@ -94,11 +104,16 @@ __global__ void __launch_bounds__(160, 1)
   if (tid == 0) {
     mbar_init(qfull, 1);
     mbar_init(qfree, 1);
-    for (int st = 0; st < kTcStages; ++st) {
-      mbar_init(kvfull(st), 1);
-      mbar_init(kvempty(st), 1);
+    for (int st = 0; st < kTcKStages; ++st) {
+      mbar_init(kfull(st), 1);
+      mbar_init(kempty(st), 1);
     }
-    mbar_init(sfull, 1);
+    for (int st = 0; st < kTcVStages; ++st) {
+      mbar_init(vfull(st), 1);
+      mbar_init(vempty(st), 1);
+    }
+    mbar_init(sfull(0), 1);
+    mbar_init(sfull(1), 1);
     mbar_init(pfull, 4);
     mbar_init(pvfull, 1);
     mbar_init(drain, 1);
@@ -113,8 +128,8 @@ __global__ void __launch_bounds__(160, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t t_s = tbase;
-  const uint32_t t_o = tbase + kTcKeys;
+  auto t_s = [&](int b) { return tbase + static_cast<uint32_t>(b * kTcKeys); };  // S0, S1
+  const uint32_t t_o = tbase + 2 * kTcKeys;
 
   const int count = __ldcg(&w.sched->chunk_count);
   const int hun = head_units(s);
@@ -146,44 +161,82 @@ __global__ void __launch_bounds__(160, 1)
 
   if (warp == 4) {
     // ------------------------------------------------ TMA loads + MMA issue
-    int g = 0;  // KV tiles issued so far by this CTA (stage ring position)
+    // Tile t of the current item is this CTA's tile g + t: its K lands in K
+    // stage (g+t) % 3, its V in V stage (g+t) % 2, its scores in S buffer
+    // (g+t) % 2.  Steady state, per tile t: wait for P(t), issue PV(t), then
+    // S(t+2) (its S buffer was freed by P(t)), then refill K and V stages.
+    int g = 0;  // tiles of earlier items
     int k = 0;  // items so far
     bool ok = true;
-    // K/V tile t of `it` into stage (g + t) % 2: eight 16-token blocks.
-    auto issue_kv = [&](const Item& it, int t) -> bool {
+    // One lane per 16-token block issues that block's TMA boxes, so the eight
+    // blocks of a tile (16 boxes for K or V) go out in parallel instead of
+    // one after another from a single thread.
+    auto load_blocks = [&](const Item& it, int t, uint32_t dst, const CUtensorMap* map,
+                           uint32_t bar) {
+      const int first = t * (kTcKeys / kBlock);
+      const int nb = min(kTcKeys / kBlock, ceil_div(it.kv_end, kBlock) - first);
+      if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb * L::kHalves * 2048));
+      __syncwarp();
+      if (lane < nb) {
+        int pb = __ldg(block_tables + static_cast<size_t>(it.row) * s.table_stride + first + lane);
+        if (pb < 0 || pb >= s.num_blocks) {
+          report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, it.row, pb);
+          pb = 0;
+        }
+        const int y = (pb * s.num_kv_heads + it.kvh) * kBlock;
+#pragma unroll
+        for (int h = 0; h < L::kHalves; ++h)
+          tma_load_2d(dst + h * L::kHalfBytes + lane * 2048, map, bar, h * 64, y);
+      }
+      __syncwarp();
+    };
+    auto issue_k = [&](const Item& it, int t) -> bool {
+      const int gt = g + t, st = gt % kTcKStages;
+      bool r = true;
+      if (lane == 0)
+        r = mbar_wait(kempty(st), ((gt / kTcKStages) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r) load_blocks(it, t, k_smem(st), &tm_k, kfull(st));
+      return r;
+    };
+    auto issue_v = [&](const Item& it, int t) -> bool {
+      const int gt = g + t, st = gt % kTcVStages;
+      bool r = true;
+      if (lane == 0)
+        r = mbar_wait(vempty(st), ((gt / kTcVStages) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r) load_blocks(it, t, v_smem(st), &tm_v, vfull(st));
+      return r;
+    };
+    // S(t) = Q K(t)^T into S buffer (g+t) % 2.
+    auto issue_s = [&](const Item& it, int t) -> bool {
       bool r = true;
       if (lane == 0) {
-        const int gt = g + t;
-        const int st = gt % kTcStages;
-        r = mbar_wait(kvempty(st), ((gt / kTcStages) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+        const int gt = g + t, st = gt % kTcKStages;
+        r = mbar_wait(kfull(st), (gt / kTcKStages) & 1, kWhereWaitFull, abort_flag);
         if (r) {
-          const int first = t * (kTcKeys / kBlock);
-          const int nb = min(kTcKeys / kBlock, ceil_div(it.kv_end, kBlock) - first);
-          mbar_arrive_expect_tx(kvfull(st), static_cast<uint32_t>(nb * 2 * L::kHalves * 2048));
-          const int* table = block_tables + static_cast<size_t>(it.row) * s.table_stride + first;
-          for (int b = 0; b < nb; ++b) {
-            int pb = __ldg(table + b);
-            if (pb < 0 || pb >= s.num_blocks) {
-              report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, it.row, pb);
-              pb = 0;
-            }
-            const int y = (pb * s.num_kv_heads + it.kvh) * kBlock;
+          tc_fence_after();
 #pragma unroll
-            for (int h = 0; h < L::kHalves; ++h) {
-              tma_load_2d(k_smem(st) + h * L::kHalfBytes + b * 2048, &tm_k, kvfull(st), h * 64, y);
-              tma_load_2d(v_smem(st) + h * L::kHalfBytes + b * 2048, &tm_v, kvfull(st), h * 64, y);
-            }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
+            umma_ss(t_s(gt & 1), smem_desc_sw128(q_smem + off, 16, 1024),
+                    smem_desc_sw128(k_smem(st) + off, 16, 1024), kIdescS, kk > 0);
           }
+          umma_commit(sfull(gt & 1));
+          umma_commit(kempty(st));
+          if (t == it.nkt - 1) umma_commit(qfree);
         }
       }
       return __shfl_sync(0xffffffffu, r, 0);
     };
-    // Wait for tile t, zero V rows past the item's last key, issue S = Q K^T.
-    auto issue_s = [&](const Item& it, int t) -> bool {
-      const int gt = g + t;
-      const int st = gt % kTcStages;
+    // O_tile = P(t) V(t), once the softmax warps have written P(t).
+    auto issue_pv = [&](const Item& it, int t) -> bool {
+      const int gt = g + t, st = gt % kTcVStages;
       bool r = true;
-      if (lane == 0) r = mbar_wait(kvfull(st), (gt / kTcStages) & 1, kWhereWaitFull, abort_flag);
+      if (lane == 0) {
+        r = mbar_wait(pfull, gt & 1, kWhereWaitMma, abort_flag) &&
+            mbar_wait(vfull(st), (gt / kTcVStages) & 1, kWhereWaitFull, abort_flag);
+      }
       r = __shfl_sync(0xffffffffu, r, 0);
       if (!r) return false;
       const int valid = it.kv_end - t * kTcKeys;  // keys of this tile that exist
@@ -203,13 +256,13 @@ __global__ void __launch_bounds__(160, 1)
       if (lane == 0) {
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
-          umma_ss(t_s, smem_desc_sw128(q_smem + off, 16, 1024),
-                  smem_desc_sw128(k_smem(st) + off, 16, 1024), kIdescS, kk > 0);
+        for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+          umma_ss(t_o,
+                  smem_desc_sw128(p_smem + (kk >> 2) * L::kHalfBytes + (kk & 3) * 32, 16, 1024),
+                  smem_desc_sw128(v_smem(st) + kk * 2048, L::kHalfBytes, 1024), kIdescPV, kk > 0);
         }
-        umma_commit(sfull);
-        if (t == it.nkt - 1) umma_commit(qfree);
+        umma_commit(pvfull);
+        umma_commit(vempty(st));
       }
       return true;
     };
@@ -225,30 +278,18 @@ __global__ void __launch_bounds__(160, 1)
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      for (int t = 0; t < min(kTcStages, it.nkt) && ok; ++t) ok = issue_kv(it, t);
+      for (int t = 0; t < min(kTcKStages, it.nkt) && ok; ++t) ok = issue_k(it, t);
+      for (int t = 0; t < min(kTcVStages, it.nkt) && ok; ++t) ok = issue_v(it, t);
       if (ok && lane == 0) ok = mbar_wait(qfull, k & 1, kWhereWaitQ, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (ok) ok = issue_s(it, 0);
+      for (int t = 0; t < min(2, it.nkt) && ok; ++t) ok = issue_s(it, t);
       for (int t = 0; t < it.nkt && ok; ++t) {
-        const int st = (g + t) % kTcStages;
-        if (lane == 0) {
-          ok = mbar_wait(pfull, (g + t) & 1, kWhereWaitMma, abort_flag);
-          if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kTcKeys / 16; ++kk) {
-              umma_ss(t_o,
-                      smem_desc_sw128(p_smem + (kk >> 2) * L::kHalfBytes + (kk & 3) * 32, 16, 1024),
-                      smem_desc_sw128(v_smem(st) + kk * 2048, L::kHalfBytes, 1024), kIdescPV,
-                      kk > 0);
-            }
-            umma_commit(pvfull);
-            umma_commit(kvempty(st));
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok && t + 1 < it.nkt) ok = issue_s(it, t + 1);
-        if (ok && t + kTcStages < it.nkt) ok = issue_kv(it, t + kTcStages);
+        // K stage of tile t was freed by S(t), issued two steps ago: refill it
+        // first so the load has the most time to land before S(t+3) needs it
+        if (t + kTcKStages < it.nkt) ok = issue_k(it, t + kTcKStages);
+        if (ok) ok = issue_pv(it, t);
+        if (ok && t + 2 < it.nkt) ok = issue_s(it, t + 2);
+        if (ok && t + kTcVStages < it.nkt) ok = issue_v(it, t + kTcVStages);
       }
       g += it.nkt;
     }
@@ -273,20 +314,31 @@ __global__ void __launch_bounds__(160, 1)
       for (int d = 0; d < D; ++d) o[d] = 0.f;
       float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
       for (int t = 0; t < it.nkt && ok; ++t) {
-        ok = __all_sync(0xffffffffu, mbar_wait(sfull, (g + t) & 1, kWhereWaitMma, abort_flag));
+        const int gt = g + t;
+        const uint32_t sb = t_s(gt & 1) + lane_base;  // this tile's S buffer, this warp's lanes
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(sfull(gt & 1), (gt >> 1) & 1, kWhereWaitMma, abort_flag));
         if (!ok) break;
         tc_fence_after();
         const int key0 = t * kTcKeys;
         float v[32];
-        // pass 1: the row maximum of this tile
-        float mx = -INFINITY;
+        // pass 1: the row maximum of this tile (4 independent chains; the
+        // causal mask is applied only to chunks that cross this row's limit)
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
         for (int c = 0; c < kTcKeys / 32; ++c) {
-          tmem_ld32(t_s + lane_base + c * 32, v);
+          tmem_ld32(sb + c * 32, v);
+          const int kb = key0 + c * 32;
+          if (kb + 32 <= lim) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            mx = fmaxf(mx, key0 + c * 32 + j < lim ? v[j] * scale_log2 : -INFINITY);
+            for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], v[j] * scale_log2);
+          } else if (kb < lim) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (kb + j < lim) m4[j & 3] = fmaxf(m4[j & 3], v[j] * scale_log2);
+          }
         }
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         const float mn = fmaxf(m, mx);
         const float mu = mn == -INFINITY ? 0.f : mn;
         const float alpha = exp2f(m - mu);
@@ -304,19 +356,31 @@ __global__ void __launch_bounds__(160, 1)
           }
         }
         // pass 2: P = 2^(x - m), rounded to the input type, into shared memory
-        float psum = 0.f;
+        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float nmu = -mu;
 #pragma unroll 1
         for (int c = 0; c < kTcKeys / 32; ++c) {
-          tmem_ld32(t_s + lane_base + c * 32, v);
+          tmem_ld32(sb + c * 32, v);
+          const int kb = key0 + c * 32;
           uint32_t pk[16];
+          if (kb + 32 <= lim) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int key = key0 + c * 32 + 2 * j;
-            const float x0 = key < lim ? v[2 * j] * scale_log2 : -INFINITY;
-            const float x1 = key + 1 < lim ? v[2 * j + 1] * scale_log2 : -INFINITY;
-            pk[j] = pack2<T>(exp2f(x0 - mu), exp2f(x1 - mu));
+            for (int j = 0; j < 16; ++j)
+              pk[j] = pack2<T>(exp2f(fmaf(v[2 * j], scale_log2, nmu)),
+                               exp2f(fmaf(v[2 * j + 1], scale_log2, nmu)));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float p0 = kb + 2 * j < lim ? exp2f(fmaf(v[2 * j], scale_log2, nmu)) : 0.f;
+              const float p1 =
+                  kb + 2 * j + 1 < lim ? exp2f(fmaf(v[2 * j + 1], scale_log2, nmu)) : 0.f;
+              pk[j] = pack2<T>(p0, p1);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {  // sum the same rounded weights P.V uses
             const float2 f = unpack2<T>(pk[j]);
-            psum += f.x + f.y;
+            ps4[j & 3] += f.x + f.y;
           }
           const int half = c >> 1;
 #pragma unroll
@@ -331,6 +395,7 @@ __global__ void __launch_bounds__(160, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pfull);
+        const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
         l = l * alpha + psum;
         m = mn;
         alpha_prev = alpha;
