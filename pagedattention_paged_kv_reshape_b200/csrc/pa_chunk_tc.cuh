@@ -9,19 +9,23 @@
 // * work item = (chunk row, tile of 128/gs query tokens x gs query heads =
 //   128 tile rows, KV head slice); a persistent grid walks the items listed
 //   by the prep kernel;
-// * Q (one 3-D TMA box) and K, V (eight 16-token TMA boxes per 128-key tile;
-//   a three-stage K ring and a two-stage V ring) land in shared memory with
-//   128-byte swizzling, which is exactly the canonical K-major layout (Q, K,
-//   P) and MN-major layout (V) the tcgen05 shared-memory descriptors describe;
+// * Q (one 3-D TMA box) and K, V (eight 16-token TMA boxes per 128-key tile,
+//   in K and V rings) land in shared memory with 128-byte swizzling, which is
+//   exactly the canonical K-major layout (Q, K, P) and MN-major layout (V) the
+//   tcgen05 shared-memory descriptors describe;
 // * one thread issues S = Q K^T (M=128, N=128, K=16 steps) into one of two
 //   TMEM score buffers, two tiles ahead of the softmax, so the tensor core
 //   computes the next scores while the softmax warps work;
-// * four softmax warps read S with tcgen05.ld, one tile row per thread, apply
-//   the causal mask (key <= position) and the online softmax in the log2
-//   domain, and write P (rounded to the input type) to shared memory;
-// * the same thread issues O_tile = P V into a second TMEM region; the
-//   softmax threads fold it into their fp32 row accumulators with the
-//   running rescale, and write the output row at the end.
+// * four softmax warps read a tile's scores with one round of tcgen05.ld (a
+//   whole 128-key row per thread), apply the causal mask (key <= position)
+//   and the online softmax in the log2 domain, and write P (rounded to the
+//   input type) into one of two shared-memory P buffers;
+// * the same thread issues O += P V into a TMEM accumulator that lives for
+//   the whole work item.  The running maximum that P is taken against is
+//   raised only when a row's maximum grows by more than 2^8 (P then stays
+//   below 256); only then is the row's O brought to the new reference point,
+//   through TMEM, between two PV steps.  The epilogue reads O once and
+//   divides by the row sum.
 //
 // Every wait is bounded.  TMEM (512 columns) is freed on every path, after a
 // final commit has drained the MMAs this CTA issued.  The kernel is launched
@@ -38,25 +42,36 @@
 
 namespace pa {
 
-constexpr int kTcRows = 128;   // tile rows = TMEM lanes
-constexpr int kTcKeys = 128;   // keys per KV tile = 8 blocks
-constexpr int kTcKStages = 3;  // K ring: a K tile is free once its QK^T has run
-constexpr int kTcVStages = 2;  // V ring: a V tile is free once its PV has run
+constexpr int kTcRows = 128;        // tile rows = TMEM lanes
+constexpr int kTcKeys = 128;        // keys per KV tile = 8 blocks
+constexpr int kTcVStages = 2;       // V ring: a V tile is free once its PV has run
+constexpr float kTcRescale = 8.f;   // raise the reference maximum past this (log2 units)
 
 template <int D>
 struct TcLayout {
+  // K ring: a K tile is free once its QK^T has run
+  static constexpr int kKStages = D == 64 ? 3 : 2;
   static constexpr int kHalves = D / 64;           // 128-byte swizzle rows per token row
   static constexpr int kHalfBytes = 128 * 128;     // 128 rows x 128 B
   static constexpr int kQBytes = kHalves * kHalfBytes;
   static constexpr int kKVBytes = kHalves * kHalfBytes;  // one K or V tile
-  static constexpr int kPBytes = 2 * kHalfBytes;   // 128 rows x 128 keys x 2 B
+  static constexpr int kPBytes = 2 * kHalfBytes;   // one P buffer: 128 rows x 128 keys x 2 B
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kTcKStages * kKVBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
   static constexpr int kOffP = kOffV + kTcVStages * kKVBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
-  // qfull, qfree, kfull[3], kempty[3], vfull[2], vempty[2], sfull[2], pfull, pvfull, drain
-  static constexpr int kNumBars = 2 + 2 * kTcKStages + 2 * kTcVStages + 2 + 3;
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  // barrier indexes: qfull, qfree, kfull[KS], kempty[KS], vfull[VS], vempty[VS],
+  // sfull[2], pfull[2], pfree[2], drain
+  static constexpr int kBarQFull = 0, kBarQFree = 1, kBarKFull = 2;
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;
+  static constexpr int kBarVEmpty = kBarVFull + kTcVStages;
+  static constexpr int kBarSFull = kBarVEmpty + kTcVStages;
+  static constexpr int kBarPFull = kBarSFull + 2;
+  static constexpr int kBarPFree = kBarPFull + 2;
+  static constexpr int kBarDrain = kBarPFree + 2;
+  static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 12;
@@ -77,6 +92,7 @@ __global__ void __launch_bounds__(160, 1)
                     const int* __restrict__ block_tables, const int* __restrict__ qsl,
                     const int* __restrict__ seq_lens, Work w, float scale_log2) {
   using L = TcLayout<D>;
+  constexpr int KS = L::kKStages, VS = kTcVStages;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescS = instr_desc_f16(kBf16, false, false, kTcRows, kTcKeys);
   constexpr uint32_t kIdescPV = instr_desc_f16(kBf16, false, true, kTcRows, D);
@@ -84,39 +100,26 @@ __global__ void __launch_bounds__(160, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + L::kOffBar;
-  const uint32_t qfull = bar0, qfree = bar0 + 8;
-  auto kfull = [&](int st) { return bar0 + 16u + 8u * st; };
-  auto kempty = [&](int st) { return bar0 + 16u + 8u * (kTcKStages + st); };
-  auto vfull = [&](int st) { return bar0 + 16u + 8u * (2 * kTcKStages + st); };
-  auto vempty = [&](int st) { return bar0 + 16u + 8u * (2 * kTcKStages + kTcVStages + st); };
-  auto sfull = [&](int b) { return bar0 + 16u + 8u * (2 * kTcKStages + 2 * kTcVStages + b); };
-  const uint32_t pfull = bar0 + 16u + 8u * (2 * kTcKStages + 2 * kTcVStages + 2);
-  const uint32_t pvfull = pfull + 8, drain = pfull + 16;
+  auto bar = [&](int i) { return sbase + static_cast<uint32_t>(L::kOffBar + 8 * i); };
+  const uint32_t qfull = bar(L::kBarQFull), qfree = bar(L::kBarQFree), drain = bar(L::kBarDrain);
+  auto kfull = [&](int st) { return bar(L::kBarKFull + st); };
+  auto kempty = [&](int st) { return bar(L::kBarKEmpty + st); };
+  auto vfull = [&](int st) { return bar(L::kBarVFull + st); };
+  auto vempty = [&](int st) { return bar(L::kBarVEmpty + st); };
+  auto sfull = [&](int b) { return bar(L::kBarSFull + b); };  // S(b) written
+  auto pfull = [&](int b) { return bar(L::kBarPFull + b); };  // P(b) written (4 warps)
+  auto pfree = [&](int b) { return bar(L::kBarPFree + b); };  // PV from P(b) done
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
   const uint32_t q_smem = sbase + L::kOffQ;
-  const uint32_t p_smem = sbase + L::kOffP;
   auto k_smem = [&](int st) { return sbase + L::kOffK + st * L::kKVBytes; };
   auto v_smem = [&](int st) { return sbase + L::kOffV + st * L::kKVBytes; };
+  auto p_smem = [&](int b) { return sbase + L::kOffP + b * L::kPBytes; };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
-    mbar_init(qfull, 1);
-    mbar_init(qfree, 1);
-    for (int st = 0; st < kTcKStages; ++st) {
-      mbar_init(kfull(st), 1);
-      mbar_init(kempty(st), 1);
-    }
-    for (int st = 0; st < kTcVStages; ++st) {
-      mbar_init(vfull(st), 1);
-      mbar_init(vempty(st), 1);
-    }
-    mbar_init(sfull(0), 1);
-    mbar_init(sfull(1), 1);
-    mbar_init(pfull, 4);
-    mbar_init(pvfull, 1);
-    mbar_init(drain, 1);
+    for (int i = 0; i < L::kNumBars; ++i)  // P(b) is written by the four softmax warps
+      mbar_init(bar(i), (i == L::kBarPFull || i == L::kBarPFull + 1) ? 4 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -161,10 +164,11 @@ __global__ void __launch_bounds__(160, 1)
 
   if (warp == 4) {
     // ------------------------------------------------ TMA loads + MMA issue
-    // Tile t of the current item is this CTA's tile g + t: its K lands in K
-    // stage (g+t) % 3, its V in V stage (g+t) % 2, its scores in S buffer
-    // (g+t) % 2.  Steady state, per tile t: wait for P(t), issue PV(t), then
-    // S(t+2) (its S buffer was freed by P(t)), then refill K and V stages.
+    // Tile t of the current item is this CTA's tile gt = g + t: its K lands
+    // in K stage gt % KS, its V in V stage gt % VS, its scores in S buffer
+    // gt % 2 and its P in P buffer gt % 2.  Steady state, per tile t: refill
+    // the K stage S(t) has freed, wait for P(t), issue PV(t), then S(t+2)
+    // (its S buffer was read before P(t) was written), then refill V.
     int g = 0;  // tiles of earlier items
     int k = 0;  // items so far
     bool ok = true;
@@ -172,10 +176,11 @@ __global__ void __launch_bounds__(160, 1)
     // blocks of a tile (16 boxes for K or V) go out in parallel instead of
     // one after another from a single thread.
     auto load_blocks = [&](const Item& it, int t, uint32_t dst, const CUtensorMap* map,
-                           uint32_t bar) {
+                           uint32_t bar_full) {
       const int first = t * (kTcKeys / kBlock);
       const int nb = min(kTcKeys / kBlock, ceil_div(it.kv_end, kBlock) - first);
-      if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nb * L::kHalves * 2048));
+      if (lane == 0)
+        mbar_arrive_expect_tx(bar_full, static_cast<uint32_t>(nb * L::kHalves * 2048));
       __syncwarp();
       if (lane < nb) {
         int pb = __ldg(block_tables + static_cast<size_t>(it.row) * s.table_stride + first + lane);
@@ -186,34 +191,32 @@ __global__ void __launch_bounds__(160, 1)
         const int y = (pb * s.num_kv_heads + it.kvh) * kBlock;
 #pragma unroll
         for (int h = 0; h < L::kHalves; ++h)
-          tma_load_2d(dst + h * L::kHalfBytes + lane * 2048, map, bar, h * 64, y);
+          tma_load_2d(dst + h * L::kHalfBytes + lane * 2048, map, bar_full, h * 64, y);
       }
       __syncwarp();
     };
     auto issue_k = [&](const Item& it, int t) -> bool {
-      const int gt = g + t, st = gt % kTcKStages;
+      const int gt = g + t, st = gt % KS;
       bool r = true;
-      if (lane == 0)
-        r = mbar_wait(kempty(st), ((gt / kTcKStages) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+      if (lane == 0) r = mbar_wait(kempty(st), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
       r = __shfl_sync(0xffffffffu, r, 0);
       if (r) load_blocks(it, t, k_smem(st), &tm_k, kfull(st));
       return r;
     };
     auto issue_v = [&](const Item& it, int t) -> bool {
-      const int gt = g + t, st = gt % kTcVStages;
+      const int gt = g + t, st = gt % VS;
       bool r = true;
-      if (lane == 0)
-        r = mbar_wait(vempty(st), ((gt / kTcVStages) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+      if (lane == 0) r = mbar_wait(vempty(st), ((gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
       r = __shfl_sync(0xffffffffu, r, 0);
       if (r) load_blocks(it, t, v_smem(st), &tm_v, vfull(st));
       return r;
     };
-    // S(t) = Q K(t)^T into S buffer (g+t) % 2.
+    // S(t) = Q K(t)^T into S buffer gt % 2.
     auto issue_s = [&](const Item& it, int t) -> bool {
       bool r = true;
       if (lane == 0) {
-        const int gt = g + t, st = gt % kTcKStages;
-        r = mbar_wait(kfull(st), (gt / kTcKStages) & 1, kWhereWaitFull, abort_flag);
+        const int gt = g + t, st = gt % KS;
+        r = mbar_wait(kfull(st), (gt / KS) & 1, kWhereWaitFull, abort_flag);
         if (r) {
           tc_fence_after();
 #pragma unroll
@@ -229,13 +232,14 @@ __global__ void __launch_bounds__(160, 1)
       }
       return __shfl_sync(0xffffffffu, r, 0);
     };
-    // O_tile = P(t) V(t), once the softmax warps have written P(t).
+    // O (+)= P(t) V(t), once the softmax warps have written P(t) (and, where
+    // a row's reference maximum moved, rescaled its O).
     auto issue_pv = [&](const Item& it, int t) -> bool {
-      const int gt = g + t, st = gt % kTcVStages;
+      const int gt = g + t, st = gt % VS, b = gt & 1;
       bool r = true;
       if (lane == 0) {
-        r = mbar_wait(pfull, gt & 1, kWhereWaitMma, abort_flag) &&
-            mbar_wait(vfull(st), (gt / kTcVStages) & 1, kWhereWaitFull, abort_flag);
+        r = mbar_wait(pfull(b), (gt >> 1) & 1, kWhereWaitMma, abort_flag) &&
+            mbar_wait(vfull(st), (gt / VS) & 1, kWhereWaitFull, abort_flag);
       }
       r = __shfl_sync(0xffffffffu, r, 0);
       if (!r) return false;
@@ -258,10 +262,11 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
         for (int kk = 0; kk < kTcKeys / 16; ++kk) {
           umma_ss(t_o,
-                  smem_desc_sw128(p_smem + (kk >> 2) * L::kHalfBytes + (kk & 3) * 32, 16, 1024),
-                  smem_desc_sw128(v_smem(st) + kk * 2048, L::kHalfBytes, 1024), kIdescPV, kk > 0);
+                  smem_desc_sw128(p_smem(b) + (kk >> 2) * L::kHalfBytes + (kk & 3) * 32, 16, 1024),
+                  smem_desc_sw128(v_smem(st) + kk * 2048, L::kHalfBytes, 1024), kIdescPV,
+                  (t > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(pvfull);
+        umma_commit(pfree(b));
         umma_commit(vempty(st));
       }
       return true;
@@ -278,18 +283,16 @@ __global__ void __launch_bounds__(160, 1)
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      for (int t = 0; t < min(kTcKStages, it.nkt) && ok; ++t) ok = issue_k(it, t);
-      for (int t = 0; t < min(kTcVStages, it.nkt) && ok; ++t) ok = issue_v(it, t);
+      for (int t = 0; t < min(KS, it.nkt) && ok; ++t) ok = issue_k(it, t);
+      for (int t = 0; t < min(VS, it.nkt) && ok; ++t) ok = issue_v(it, t);
       if (ok && lane == 0) ok = mbar_wait(qfull, k & 1, kWhereWaitQ, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       for (int t = 0; t < min(2, it.nkt) && ok; ++t) ok = issue_s(it, t);
       for (int t = 0; t < it.nkt && ok; ++t) {
-        // K stage of tile t was freed by S(t), issued two steps ago: refill it
-        // first so the load has the most time to land before S(t+3) needs it
-        if (t + kTcKStages < it.nkt) ok = issue_k(it, t + kTcKStages);
+        if (t + KS < it.nkt) ok = issue_k(it, t + KS);  // into the stage S(t) has freed
         if (ok) ok = issue_pv(it, t);
         if (ok && t + 2 < it.nkt) ok = issue_s(it, t + 2);
-        if (ok && t + kTcVStages < it.nkt) ok = issue_v(it, t + kTcVStages);
+        if (ok && t + VS < it.nkt) ok = issue_v(it, t + VS);
       }
       g += it.nkt;
     }
@@ -302,6 +305,10 @@ __global__ void __launch_bounds__(160, 1)
     // ------------------------------------------------------- softmax warps
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int r = tid;  // tile row = TMEM lane
+    // Scores enter as x = s * |scale| after a sign flip of s for a negative
+    // scale, so that the row maximum is always a max.
+    const bool neg = scale_log2 < 0.f;
+    const float sc = fabsf(scale_log2);
     int g = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
@@ -309,117 +316,127 @@ __global__ void __launch_bounds__(160, 1)
       const int i = r / s.gs, gi = r % s.gs;
       const bool valid = i < it.nq && gi < it.rows;
       const int lim = it.pos0 + i + 1;  // keys visible to this row
-      float o[D];
-#pragma unroll
-      for (int d = 0; d < D; ++d) o[d] = 0.f;
-      float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+      float m = -INFINITY;              // reference maximum P is taken against (log2 units)
+      float l = 0.f;                    // sum of P against that reference
       for (int t = 0; t < it.nkt && ok; ++t) {
-        const int gt = g + t;
-        const uint32_t sb = t_s(gt & 1) + lane_base;  // this tile's S buffer, this warp's lanes
+        const int gt = g + t, b = gt & 1;
+        // scores of this tile, and P buffer b free (PV two tiles back done)
         ok = __all_sync(0xffffffffu,
-                        mbar_wait(sfull(gt & 1), (gt >> 1) & 1, kWhereWaitMma, abort_flag));
+                        mbar_wait(sfull(b), (gt >> 1) & 1, kWhereWaitMma, abort_flag) &&
+                            mbar_wait(pfree(b), ((gt >> 1) & 1) ^ 1, kWhereWaitMma, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        const int key0 = t * kTcKeys;
-        float v[32];
-        // pass 1: the row maximum of this tile (4 independent chains; the
-        // causal mask is applied only to chunks that cross this row's limit)
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int c = 0; c < kTcKeys / 32; ++c) {
-          tmem_ld32(sb + c * 32, v);
-          const int kb = key0 + c * 32;
-          if (kb + 32 <= lim) {
+        uint32_t ra[64], rb[64];
+        tmem_ld64_issue(t_s(b) + lane_base, ra);
+        tmem_ld64_issue(t_s(b) + lane_base + 64, rb);
+        tmem_ld_wait(ra);
+        reg_tie(rb);
+        float x[kTcKeys];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], v[j] * scale_log2);
-          } else if (kb < lim) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (kb + j < lim) m4[j & 3] = fmaxf(m4[j & 3], v[j] * scale_log2);
-          }
+        for (int j = 0; j < 64; ++j) {
+          x[j] = __uint_as_float(ra[j]);
+          x[64 + j] = __uint_as_float(rb[j]);
         }
-        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        const float mn = fmaxf(m, mx);
-        const float mu = mn == -INFINITY ? 0.f : mn;
-        const float alpha = exp2f(m - mu);
-        // the previous tile's P V: fold it in, which also frees P and O
-        if (t > 0) {
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(pvfull, (g + t - 1) & 1, kWhereWaitMma, abort_flag));
+        if (neg) {
+#pragma unroll
+          for (int j = 0; j < kTcKeys; ++j) x[j] = -x[j];
+        }
+        const int nvis = lim - t * kTcKeys;  // keys of this tile this row may see
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (nvis >= kTcKeys) {
+#pragma unroll
+          for (int j = 0; j < kTcKeys; ++j) m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < kTcKeys; ++j)
+            if (j < nvis) m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+        }
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
+        // raise the reference maximum only when the row maximum has grown by
+        // more than 2^kTcRescale (always on the first visible keys)
+        const bool raise = mx > m + kTcRescale;
+        float alpha = 1.f;
+        if (raise) {
+          alpha = ex2_approx(m - mx);  // 0 when m = -inf
+          m = mx;
+        }
+        if (t > 0 && __any_sync(0xffffffffu, raise)) {
+          // O holds PV of tiles 0 .. t-1: once PV(t-1) is done, scale it
+          ok = __all_sync(0xffffffffu, mbar_wait(pfree((gt - 1) & 1), ((gt - 1) >> 1) & 1,
+                                                 kWhereWaitMma, abort_flag));
           if (!ok) break;
           tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t ro[64];
+            tmem_ld64_issue(t_o + lane_base + c * 64, ro);
+            tmem_ld_wait(ro);
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32(t_o + lane_base + c * 32, v);
+            for (int j = 0; j < 64; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
+            tmem_st64(t_o + lane_base + c * 64, ro);
+          }
+          tmem_st_wait();
+        }
+        l *= alpha;
+        // P = 2^(x - m), rounded to the input type, into P buffer b
+        const float nm = m == -INFINITY ? 0.f : -m;
+        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[kTcKeys / 2];
+        if (nvis >= kTcKeys) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[c * 32 + j] = fmaf(o[c * 32 + j], alpha_prev, v[j]);
+          for (int j = 0; j < kTcKeys / 2; ++j) {
+            const float p0 = ex2_approx(fmaf(x[2 * j], sc, nm));
+            const float p1 = ex2_approx(fmaf(x[2 * j + 1], sc, nm));
+            ps4[j & 3] += p0 + p1;
+            pk[j] = pack2<T>(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < kTcKeys / 2; ++j) {
+            const float p0 = 2 * j < nvis ? ex2_approx(fmaf(x[2 * j], sc, nm)) : 0.f;
+            const float p1 = 2 * j + 1 < nvis ? ex2_approx(fmaf(x[2 * j + 1], sc, nm)) : 0.f;
+            ps4[j & 3] += p0 + p1;
+            pk[j] = pack2<T>(p0, p1);
           }
         }
-        // pass 2: P = 2^(x - m), rounded to the input type, into shared memory
-        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
-        const float nmu = -mu;
-#pragma unroll 1
-        for (int c = 0; c < kTcKeys / 32; ++c) {
-          tmem_ld32(sb + c * 32, v);
-          const int kb = key0 + c * 32;
-          uint32_t pk[16];
-          if (kb + 32 <= lim) {
+        // keys 64c .. 64c+63 are one 128-byte row of P half c
+        const uint32_t prow = L::kOffP + b * L::kPBytes + r * 128;
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              pk[j] = pack2<T>(exp2f(fmaf(v[2 * j], scale_log2, nmu)),
-                               exp2f(fmaf(v[2 * j + 1], scale_log2, nmu)));
-          } else {
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float p0 = kb + 2 * j < lim ? exp2f(fmaf(v[2 * j], scale_log2, nmu)) : 0.f;
-              const float p1 =
-                  kb + 2 * j + 1 < lim ? exp2f(fmaf(v[2 * j + 1], scale_log2, nmu)) : 0.f;
-              pk[j] = pack2<T>(p0, p1);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {  // sum the same rounded weights P.V uses
-            const float2 f = unpack2<T>(pk[j]);
-            ps4[j & 3] += f.x + f.y;
-          }
-          const int half = c >> 1;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int ch = (c & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
-            *reinterpret_cast<uint4*>(smem + L::kOffP + half * L::kHalfBytes + r * 128 +
-                                      ((ch ^ (r & 7)) << 4)) =
-                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          for (int q8 = 0; q8 < 8; ++q8) {
+            const int j = c * 32 + q8 * 4;
+            *reinterpret_cast<uint4*>(smem + prow + c * L::kHalfBytes + ((q8 ^ (r & 7)) << 4)) =
+                make_uint4(pk[j], pk[j + 1], pk[j + 2], pk[j + 3]);
           }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(pfull);
-        const float psum = (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-        l = l * alpha + psum;
-        m = mn;
-        alpha_prev = alpha;
+        if (lane == 0) mbar_arrive(pfull(b));
+        l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
       }
-      if (ok && it.nkt > 0) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(pvfull, (g + it.nkt - 1) & 1, kWhereWaitMma, abort_flag));
+      if (ok) {
+        // the item's last PV done: O is final
+        const int gl = g + it.nkt - 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(pfree(gl & 1), (gl >> 1) & 1, kWhereWaitMma,
+                                               abort_flag));
         if (ok) {
           tc_fence_after();
-          float v[32];
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t ro[64];
+            tmem_ld64_issue(t_o + lane_base + c * 64, ro);
+            tmem_ld_wait(ro);
+            if (valid) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32(t_o + lane_base + c * 32, v);
+              for (int q = 0; q < 8; ++q) {
+                float a[8];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[c * 32 + j] = fmaf(o[c * 32 + j], alpha_prev, v[j]);
-          }
-          if (valid) {
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-              float a[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) a[e] = o[c * 8 + e];
-              store_row8<T, D>(s, out, it.token0 + i, it.head0 + gi, c, a, inv);
+                for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(ro[q * 8 + e]);
+                store_row8<T, D>(s, out, it.token0 + i, it.head0 + gi, c * 8 + q, a, inv);
+              }
             }
           }
         }

@@ -171,6 +171,24 @@ def test_varlen_matches_oracle(case, path):
     assert_close(out, ref, dtype, f"varlen case {case} ({path})")
 
 
+@pytest.mark.parametrize("scale", [1.0, -0.3, 0.0])
+def test_varlen_other_scales(scale):
+    """Scales other than 1/sqrt(head_dim).  With 1.0 the scores of N(0,1) data
+    have a standard deviation of about 11, so a row's running maximum climbs by
+    many powers of two across the context and the chunk kernel has to move the
+    reference point of its TMEM accumulator several times; a negative scale
+    reverses the order of the scores; zero is the plain mean of the visible
+    values.  f16, so that the near one-hot outputs of the large scale (|o| up to
+    about 5) still round to within the 1e-2 bound."""
+    rows = [(1500, 300), (700, 129), (40, 1), (900, 1)]
+    b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=32, num_kv_heads=8,
+                      head_dim=128, dtype="f16", seed=55, device=DEV, pool_factor=1.2)
+    b.scale = scale
+    out, _, _ = gpu_step(b, varlen=True)
+    ref, _, _ = oracle_step(b, varlen=True)
+    assert_close(out, ref, "f16", f"varlen scale {scale}")
+
+
 def test_chunk_kernel_agrees_with_decode_kernel_tiles():
     """The tcgen05 chunk tiles and the decode kernel's 16-row tiles compute the
     same rows; both are within tolerance of each other as well as the oracle."""
