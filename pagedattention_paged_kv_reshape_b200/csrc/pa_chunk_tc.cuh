@@ -8,24 +8,26 @@
 //
 // * work item = (chunk row, tile of 128/gs query tokens x gs query heads =
 //   128 tile rows, KV head slice); a persistent grid walks the items listed
-//   by the prep kernel;
-// * Q (one 3-D TMA box) and K, V (eight 16-token TMA boxes per 128-key tile,
-//   in K and V rings) land in shared memory with 128-byte swizzling, which is
-//   exactly the canonical K-major layout (Q, K, P) and MN-major layout (V) the
-//   tcgen05 shared-memory descriptors describe;
-// * one thread issues S = Q K^T (M=128, N=128, K=16 steps) into one of two
-//   TMEM score buffers, two tiles ahead of the softmax, so the tensor core
-//   computes the next scores while the softmax warps work;
+//   by the prep kernel, each CTA its items one after another;
+// * a load warp brings Q (one 3-D TMA box, two buffers) and K, V (eight
+//   16-token TMA boxes per 128-key tile, in K and V rings) into shared memory
+//   with 128-byte swizzling, which is exactly the canonical K-major layout
+//   (Q, K) and MN-major layout (V) the tcgen05 shared-memory descriptors
+//   describe.  It runs ahead of the tensor core as far as the rings allow,
+//   and hands each item's metadata to the other warps through shared memory;
+// * an MMA warp walks the CTA's tiles as one sequence across items: S = Q K^T
+//   (M=128, N=128, K=16 steps) into one of two TMEM score buffers, two tiles
+//   ahead of O += P V, so the tensor core computes the next scores while the
+//   softmax warps work, also across the boundary between two items;
 // * four softmax warps read a tile's scores with one round of tcgen05.ld (a
 //   whole 128-key row per thread), apply the causal mask (key <= position)
 //   and the online softmax in the log2 domain, and write P (rounded to the
-//   input type) into one of two shared-memory P buffers;
-// * the same thread issues O += P V into a TMEM accumulator that lives for
-//   the whole work item.  The running maximum that P is taken against is
-//   raised only when a row's maximum grows by more than 2^8 (P then stays
-//   below 256); only then is the row's O brought to the new reference point,
-//   through TMEM, between two PV steps.  The epilogue reads O once and
-//   divides by the row sum.
+//   input type) back into TMEM, where the PV MMA reads it as its A operand;
+// * O lives in TMEM for the whole item.  The running maximum that P is taken
+//   against is raised only when a row's maximum grows by more than 2^8 (P then
+//   stays below 256); only then is the row's O brought to the new reference
+//   point, through TMEM, between two PV steps.  The epilogue reads O once and
+//   divides by the row sum (of the rounded P that the PV MMA used).
 //
 // Every wait is bounded.  TMEM (512 columns) is freed on every path, after a
 // final commit has drained the MMAs this CTA issued.  The kernel is launched
@@ -44,55 +46,62 @@ namespace pa {
 
 constexpr int kTcRows = 128;        // tile rows = TMEM lanes
 constexpr int kTcKeys = 128;        // keys per KV tile = 8 blocks
-constexpr int kTcVStages = 2;       // V ring: a V tile is free once its PV has run
 constexpr float kTcRescale = 8.f;   // raise the reference maximum past this (log2 units)
+constexpr int kTcItemSlots = 4;     // item metadata handed from the load warp
 
 template <int D>
 struct TcLayout {
-  // K ring: a K tile is free once its QK^T has run
-  static constexpr int kKStages = D == 64 ? 3 : 2;
-  static constexpr int kHalves = D / 64;           // 128-byte swizzle rows per token row
-  static constexpr int kHalfBytes = 128 * 128;     // 128 rows x 128 B
-  static constexpr int kQBytes = kHalves * kHalfBytes;
-  static constexpr int kKVBytes = kHalves * kHalfBytes;  // one K or V tile
-  static constexpr int kPBytes = 2 * kHalfBytes;   // one P buffer: 128 rows x 128 keys x 2 B
+  static constexpr int kQStages = 2;
+  static constexpr int kKStages = D == 64 ? 4 : 3;  // a K tile is free once its QK^T has run
+  static constexpr int kVStages = D == 64 ? 4 : 2;  // a V tile is free once its PV has run
+  static constexpr int kHalves = D / 64;            // 128-byte swizzle rows per token row
+  static constexpr int kHalfBytes = 128 * 128;      // 128 rows x 128 B
+  static constexpr int kTileBytes = kHalves * kHalfBytes;  // one Q, K or V tile
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
-  static constexpr int kOffP = kOffV + kTcVStages * kKVBytes;
-  static constexpr int kOffBar = kOffP + 2 * kPBytes;
-  // barrier indexes: qfull, qfree, kfull[KS], kempty[KS], vfull[VS], vempty[VS],
-  // sfull[2], pfull[2], pfree[2], drain
-  static constexpr int kBarQFull = 0, kBarQFree = 1, kBarKFull = 2;
+  static constexpr int kOffK = kOffQ + kQStages * kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  // barrier indexes
+  static constexpr int kBarQFull = 0;
+  static constexpr int kBarQFree = kBarQFull + kQStages;
+  static constexpr int kBarKFull = kBarQFree + kQStages;
   static constexpr int kBarKEmpty = kBarKFull + kKStages;
   static constexpr int kBarVFull = kBarKEmpty + kKStages;
-  static constexpr int kBarVEmpty = kBarVFull + kTcVStages;
-  static constexpr int kBarSFull = kBarVEmpty + kTcVStages;
-  static constexpr int kBarPFull = kBarSFull + 2;
-  static constexpr int kBarPFree = kBarPFull + 2;
+  static constexpr int kBarVEmpty = kBarVFull + kVStages;
+  static constexpr int kBarSFull = kBarVEmpty + kVStages;  // S(b) written
+  static constexpr int kBarPFull = kBarSFull + 2;          // P(b) written (4 warps)
+  static constexpr int kBarPFree = kBarPFull + 2;          // the PV that read P(b) done
   static constexpr int kBarDrain = kBarPFree + 2;
   static constexpr int kNumBars = kBarDrain + 1;
-  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kOffItems = kOffBar + kNumBars * 8;
+  static constexpr int kItemBytes = 48;
+  static constexpr int kOffTmem = kOffItems + kTcItemSlots * kItemBytes;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 12;
   // at least ~114 KB, so that a single CTA fits per SM and its TMEM
   // allocation can never wait for another CTA's
   static constexpr int kSmem = (kBytes + 1024) > 116 * 1024 ? (kBytes + 1024) : 116 * 1024;
-  static constexpr int kThreads = 160;             // 4 softmax warps + 1 TMA/MMA warp
-  static constexpr uint32_t kTmemCols = 512;       // S0 [0,128), S1 [128,256), O [256, 256 + D)
-  static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "1 KB alignment");
+  static constexpr int kThreads = 192;  // 4 softmax warps, 1 load warp, 1 MMA warp
+  // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256 + D), P0 [384,448), P1 [448,512)
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffBar % 1024 == 0, "1 KB alignment");
   static_assert(kBytes + 1024 <= 232448, "shared memory budget");
 };
 
+// One work item, as every warp of the CTA sees it.
+struct TcItem {
+  int row, token0, nq, kvh, head0, rows, pos0, kv_end, nkt;
+};
+
 template <typename T, int D>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(192, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, Shape s, T* __restrict__ out,
                     const int* __restrict__ block_tables, const int* __restrict__ qsl,
                     const int* __restrict__ seq_lens, Work w, float scale_log2) {
   using L = TcLayout<D>;
-  constexpr int KS = L::kKStages, VS = kTcVStages;
+  constexpr int QS = L::kQStages, KS = L::kKStages, VS = L::kVStages;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescS = instr_desc_f16(kBf16, false, false, kTcRows, kTcKeys);
   constexpr uint32_t kIdescPV = instr_desc_f16(kBf16, false, true, kTcRows, D);
@@ -101,20 +110,26 @@ __global__ void __launch_bounds__(160, 1)
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) { return sbase + static_cast<uint32_t>(L::kOffBar + 8 * i); };
-  const uint32_t qfull = bar(L::kBarQFull), qfree = bar(L::kBarQFree), drain = bar(L::kBarDrain);
+  auto qfull = [&](int qb) { return bar(L::kBarQFull + qb); };
+  auto qfree = [&](int qb) { return bar(L::kBarQFree + qb); };
   auto kfull = [&](int st) { return bar(L::kBarKFull + st); };
   auto kempty = [&](int st) { return bar(L::kBarKEmpty + st); };
   auto vfull = [&](int st) { return bar(L::kBarVFull + st); };
   auto vempty = [&](int st) { return bar(L::kBarVEmpty + st); };
-  auto sfull = [&](int b) { return bar(L::kBarSFull + b); };  // S(b) written
-  auto pfull = [&](int b) { return bar(L::kBarPFull + b); };  // P(b) written (4 warps)
-  auto pfree = [&](int b) { return bar(L::kBarPFree + b); };  // PV from P(b) done
+  auto sfull = [&](int b) { return bar(L::kBarSFull + b); };
+  auto pfull = [&](int b) { return bar(L::kBarPFull + b); };
+  auto pfree = [&](int b) { return bar(L::kBarPFree + b); };
+  const uint32_t drain = bar(L::kBarDrain);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
-  const uint32_t q_smem = sbase + L::kOffQ;
-  auto k_smem = [&](int st) { return sbase + L::kOffK + st * L::kKVBytes; };
-  auto v_smem = [&](int st) { return sbase + L::kOffV + st * L::kKVBytes; };
-  auto p_smem = [&](int b) { return sbase + L::kOffP + b * L::kPBytes; };
+  auto q_smem = [&](int qb) { return sbase + L::kOffQ + qb * L::kTileBytes; };
+  auto k_smem = [&](int st) { return sbase + L::kOffK + st * L::kTileBytes; };
+  auto v_smem = [&](int st) { return sbase + L::kOffV + st * L::kTileBytes; };
+  // item k's metadata: written by the load warp before it arms qfull(k % 2),
+  // read by the other warps after that phase has completed
+  auto item_slot = [&](int k) {
+    return reinterpret_cast<TcItem*>(smem + L::kOffItems + (k % kTcItemSlots) * L::kItemBytes);
+  };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
@@ -131,128 +146,169 @@ __global__ void __launch_bounds__(160, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  auto t_s = [&](int b) { return tbase + static_cast<uint32_t>(b * kTcKeys); };  // S0, S1
+  auto t_s = [&](int b) { return tbase + static_cast<uint32_t>(b * kTcKeys); };
   const uint32_t t_o = tbase + 2 * kTcKeys;
+  auto t_p = [&](int b) { return tbase + static_cast<uint32_t>(3 * kTcKeys + b * kTcKeys / 2); };
 
   const int count = __ldcg(&w.sched->chunk_count);
-  const int hun = head_units(s);
-  const int items = count * hun;
-  const int qt = kTcRows / s.gs;
-
-  // Everything about one item, computed identically by every thread.
-  struct Item {
-    int row, token0, nq, kvh, head0, rows, pos0, kv_end, nkt;
-  };
-  auto load_item = [&](int item) {
-    Item it;
-    const int e = item % count;
-    const int hu = item / count;
-    const int2 ent = __ldcg(w.chunk_list + e);
-    const RowInfo ri = load_row(s, qsl, seq_lens, ent.x);
-    it.row = ent.x;
-    it.kvh = hu / s.ns;
-    const int slice = hu % s.ns;
-    it.head0 = it.kvh * s.group + slice * 16;
-    it.rows = min(s.gs, s.group - slice * 16);
-    it.nq = min(qt, ri.q_len - ent.y);
-    it.token0 = ri.token0 + ent.y;
-    it.pos0 = ri.seq_len - ri.q_len + ent.y;
-    it.kv_end = it.pos0 + it.nq;
-    it.nkt = ceil_div(it.kv_end, kTcKeys);
-    return it;
-  };
+  const int items = count * head_units(s);
+  // the k-th item of this CTA is blockIdx.x + k * gridDim.x
+  const int my_items = static_cast<int>(blockIdx.x) < items
+                           ? (items - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                           : 0;
 
   if (warp == 4) {
-    // ------------------------------------------------ TMA loads + MMA issue
-    // Tile t of the current item is this CTA's tile gt = g + t: its K lands
-    // in K stage gt % KS, its V in V stage gt % VS, its scores in S buffer
-    // gt % 2 and its P in P buffer gt % 2.  Steady state, per tile t: refill
-    // the K stage S(t) has freed, wait for P(t), issue PV(t), then S(t+2)
-    // (its S buffer was read before P(t) was written), then refill V.
+    // ---------------------------------------------------------- TMA loads
+    const int qt = kTcRows / s.gs;
     int g = 0;  // tiles of earlier items
-    int k = 0;  // items so far
     bool ok = true;
-    // One lane per 16-token block issues that block's TMA boxes, so the eight
-    // blocks of a tile (16 boxes for K or V) go out in parallel instead of
-    // one after another from a single thread.
-    auto load_blocks = [&](const Item& it, int t, uint32_t dst, const CUtensorMap* map,
-                           uint32_t bar_full) {
-      const int first = t * (kTcKeys / kBlock);
-      const int nb = min(kTcKeys / kBlock, ceil_div(it.kv_end, kBlock) - first);
-      if (lane == 0)
-        mbar_arrive_expect_tx(bar_full, static_cast<uint32_t>(nb * L::kHalves * 2048));
-      __syncwarp();
-      if (lane < nb) {
-        int pb = __ldg(block_tables + static_cast<size_t>(it.row) * s.table_stride + first + lane);
-        if (pb < 0 || pb >= s.num_blocks) {
-          report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, it.row, pb);
-          pb = 0;
-        }
-        const int y = (pb * s.num_kv_heads + it.kvh) * kBlock;
-#pragma unroll
-        for (int h = 0; h < L::kHalves; ++h)
-          tma_load_2d(dst + h * L::kHalfBytes + lane * 2048, map, bar_full, h * 64, y);
+    for (int k = 0; k < my_items && ok; ++k) {
+      TcItem it;
+      {
+        const int item = blockIdx.x + k * gridDim.x;
+        const int e = item % count;
+        const int hu = item / count;
+        const int2 ent = __ldcg(w.chunk_list + e);
+        const RowInfo ri = load_row(s, qsl, seq_lens, ent.x);
+        const int slice = hu % s.ns;
+        it.row = ent.x;
+        it.kvh = hu / s.ns;
+        it.head0 = it.kvh * s.group + slice * 16;
+        it.rows = min(s.gs, s.group - slice * 16);
+        it.nq = min(qt, ri.q_len - ent.y);
+        it.token0 = ri.token0 + ent.y;
+        it.pos0 = ri.seq_len - ri.q_len + ent.y;
+        it.kv_end = it.pos0 + it.nq;
+        it.nkt = ceil_div(it.kv_end, kTcKeys);
       }
-      __syncwarp();
+      const int qb = k % QS;
+      if (lane == 0) {
+        // Q buffer qb was last read by the S MMAs of item k - 2
+        ok = mbar_wait(qfree(qb), ((k / QS) & 1) ^ 1, kWhereWaitQ, abort_flag);
+        if (ok) {
+          *item_slot(k) = it;
+          mbar_arrive_expect_tx(qfull(qb), static_cast<uint32_t>(L::kTileBytes));
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_3d(q_smem(qb) + h * L::kHalfBytes, &tm_q, qfull(qb), h * 64, it.head0,
+                        it.token0);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      for (int t = 0; t < it.nkt && ok; ++t) {
+        const int gt = g + t, ks = gt % KS, vs = gt % VS;
+        // one lane per 16-token block of the tile: its id, then its K and V boxes
+        const int first = t * (kTcKeys / kBlock);
+        const int nb = min(kTcKeys / kBlock, ceil_div(it.kv_end, kBlock) - first);
+        int y = 0;
+        if (lane < nb) {
+          int pb = __ldg(block_tables + static_cast<size_t>(it.row) * s.table_stride + first + lane);
+          if (pb < 0 || pb >= s.num_blocks) {
+            report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, it.row, pb);
+            pb = 0;
+          }
+          y = (pb * s.num_kv_heads + it.kvh) * kBlock;
+        }
+        const uint32_t tx = static_cast<uint32_t>(nb * L::kHalves * 2048);
+        bool r = true;
+        if (lane == 0) {
+          r = mbar_wait(kempty(ks), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+          if (r) mbar_arrive_expect_tx(kfull(ks), tx);
+        }
+        ok = __shfl_sync(0xffffffffu, r, 0);
+        if (!ok) break;
+        if (lane < nb) {
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_2d(k_smem(ks) + h * L::kHalfBytes + lane * 2048, &tm_k, kfull(ks), h * 64,
+                        y);
+        }
+        if (lane == 0) {
+          r = mbar_wait(vempty(vs), ((gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+          if (r) mbar_arrive_expect_tx(vfull(vs), tx);
+        }
+        ok = __shfl_sync(0xffffffffu, r, 0);
+        if (!ok) break;
+        if (lane < nb) {
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h)
+            tma_load_2d(v_smem(vs) + h * L::kHalfBytes + lane * 2048, &tm_v, vfull(vs), h * 64,
+                        y);
+        }
+      }
+      g += it.nkt;
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issue
+    // The CTA's tiles form one sequence gt = 0, 1, 2, ... across its items.
+    // S(gt + 2) is issued right after PV(gt): by then the softmax warps have
+    // read S buffer gt % 2 (they wrote P(gt) after reading it).  Two cursors
+    // walk the sequence, the S cursor two tiles ahead of the PV cursor.
+    struct Cursor {
+      int k, t, g0, nkt, kv_end;
     };
-    auto issue_k = [&](const Item& it, int t) -> bool {
-      const int gt = g + t, st = gt % KS;
+    // enter item c.k: wait until its Q has landed (its metadata with it)
+    auto enter = [&](Cursor& c, bool wait_q) -> bool {
+      if (c.k >= my_items) return true;
       bool r = true;
-      if (lane == 0) r = mbar_wait(kempty(st), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+      int nkt = 0, kv_end = 0;
+      if (lane == 0) {  // the lane that observed qfull reads the slot
+        if (wait_q) r = mbar_wait(qfull(c.k % QS), (c.k / QS) & 1, kWhereWaitQ, abort_flag);
+        if (r) {
+          nkt = item_slot(c.k)->nkt;
+          kv_end = item_slot(c.k)->kv_end;
+        }
+      }
       r = __shfl_sync(0xffffffffu, r, 0);
-      if (r) load_blocks(it, t, k_smem(st), &tm_k, kfull(st));
+      c.nkt = __shfl_sync(0xffffffffu, nkt, 0);
+      c.kv_end = __shfl_sync(0xffffffffu, kv_end, 0);
       return r;
     };
-    auto issue_v = [&](const Item& it, int t) -> bool {
-      const int gt = g + t, st = gt % VS;
-      bool r = true;
-      if (lane == 0) r = mbar_wait(vempty(st), ((gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-      r = __shfl_sync(0xffffffffu, r, 0);
-      if (r) load_blocks(it, t, v_smem(st), &tm_v, vfull(st));
-      return r;
+    auto advance = [&](Cursor& c) {  // true when it moved on to the next item
+      if (++c.t < c.nkt) return false;
+      c.g0 += c.nkt;
+      c.t = 0;
+      ++c.k;
+      return true;
     };
-    // S(t) = Q K(t)^T into S buffer gt % 2.
-    auto issue_s = [&](const Item& it, int t) -> bool {
+    auto issue_s = [&](const Cursor& c) -> bool {
+      const int gt = c.g0 + c.t, ks = gt % KS, qb = c.k % QS;
       bool r = true;
       if (lane == 0) {
-        const int gt = g + t, st = gt % KS;
-        r = mbar_wait(kfull(st), (gt / KS) & 1, kWhereWaitFull, abort_flag);
+        r = mbar_wait(kfull(ks), (gt / KS) & 1, kWhereWaitFull, abort_flag);
         if (r) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
-            umma_ss(t_s(gt & 1), smem_desc_sw128(q_smem + off, 16, 1024),
-                    smem_desc_sw128(k_smem(st) + off, 16, 1024), kIdescS, kk > 0);
+            umma_ss(t_s(gt & 1), smem_desc_sw128(q_smem(qb) + off, 16, 1024),
+                    smem_desc_sw128(k_smem(ks) + off, 16, 1024), kIdescS, kk > 0);
           }
           umma_commit(sfull(gt & 1));
-          umma_commit(kempty(st));
-          if (t == it.nkt - 1) umma_commit(qfree);
+          umma_commit(kempty(ks));
+          if (c.t == c.nkt - 1) umma_commit(qfree(qb));
         }
       }
       return __shfl_sync(0xffffffffu, r, 0);
     };
-    // O (+)= P(t) V(t), once the softmax warps have written P(t) (and, where
-    // a row's reference maximum moved, rescaled its O).
-    auto issue_pv = [&](const Item& it, int t) -> bool {
-      const int gt = g + t, st = gt % VS, b = gt & 1;
+    auto issue_pv = [&](const Cursor& c) -> bool {
+      const int gt = c.g0 + c.t, vs = gt % VS, b = gt & 1;
       bool r = true;
       if (lane == 0) {
         r = mbar_wait(pfull(b), (gt >> 1) & 1, kWhereWaitMma, abort_flag) &&
-            mbar_wait(vfull(st), (gt / VS) & 1, kWhereWaitFull, abort_flag);
+            mbar_wait(vfull(vs), (gt / VS) & 1, kWhereWaitFull, abort_flag);
       }
       r = __shfl_sync(0xffffffffu, r, 0);
       if (!r) return false;
-      const int valid = it.kv_end - t * kTcKeys;  // keys of this tile that exist
+      const int valid = c.kv_end - c.t * kTcKeys;  // keys of this tile that exist
       if (valid < kTcKeys) {
         // padding rows may hold anything (NaN included), and 0 * NaN is NaN
         const int nchunks = (kTcKeys - valid) * L::kHalves * 8;
-        for (int c = lane; c < nchunks; c += 32) {
-          const int row = valid + c / (L::kHalves * 8);
-          const int h = (c / 8) % L::kHalves;
-          const int ch = c % 8;
-          *reinterpret_cast<uint4*>(smem + L::kOffV + st * L::kKVBytes + h * L::kHalfBytes +
-                                    row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        for (int ch = lane; ch < nchunks; ch += 32) {
+          const int row = valid + ch / (L::kHalves * 8);
+          const int h = (ch / 8) % L::kHalves;
+          *reinterpret_cast<uint4*>(smem + L::kOffV + vs * L::kTileBytes + h * L::kHalfBytes +
+                                    row * 128 + (ch % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
@@ -261,40 +317,29 @@ __global__ void __launch_bounds__(160, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTcKeys / 16; ++kk) {
-          umma_ss(t_o,
-                  smem_desc_sw128(p_smem(b) + (kk >> 2) * L::kHalfBytes + (kk & 3) * 32, 16, 1024),
-                  smem_desc_sw128(v_smem(st) + kk * 2048, L::kHalfBytes, 1024), kIdescPV,
-                  (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(t_o, t_p(b) + kk * 8,
+                  smem_desc_sw128(v_smem(vs) + kk * 2048, L::kHalfBytes, 1024), kIdescPV,
+                  (c.t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(pfree(b));
-        umma_commit(vempty(st));
+        umma_commit(vempty(vs));
       }
       return true;
     };
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
-      const Item it = load_item(item);
-      if (lane == 0) {
-        if (k > 0) ok = mbar_wait(qfree, (k - 1) & 1, kWhereWaitQ, abort_flag);
-        if (ok) {
-          mbar_arrive_expect_tx(qfull, static_cast<uint32_t>(L::kQBytes));
-#pragma unroll
-          for (int h = 0; h < L::kHalves; ++h)
-            tma_load_3d(q_smem + h * L::kHalfBytes, &tm_q, qfull, h * 64, it.head0, it.token0);
-        }
+    Cursor cs{0, 0, 0, 0, 0}, cp{0, 0, 0, 0, 0};
+    bool ok = enter(cs, true);
+    for (int j = 0; j < 2 && ok && cs.k < my_items; ++j) {
+      ok = issue_s(cs);
+      if (ok && advance(cs)) ok = enter(cs, true);
+    }
+    if (ok) ok = enter(cp, false);  // the S cursor has waited for item 0's Q
+    while (ok && cp.k < my_items) {
+      ok = issue_pv(cp);
+      if (ok && advance(cp)) ok = enter(cp, false);  // the S cursor is past it already
+      if (ok && cs.k < my_items) {
+        ok = issue_s(cs);
+        if (ok && advance(cs)) ok = enter(cs, true);
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      for (int t = 0; t < min(KS, it.nkt) && ok; ++t) ok = issue_k(it, t);
-      for (int t = 0; t < min(VS, it.nkt) && ok; ++t) ok = issue_v(it, t);
-      if (ok && lane == 0) ok = mbar_wait(qfull, k & 1, kWhereWaitQ, abort_flag);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      for (int t = 0; t < min(2, it.nkt) && ok; ++t) ok = issue_s(it, t);
-      for (int t = 0; t < it.nkt && ok; ++t) {
-        if (t + KS < it.nkt) ok = issue_k(it, t + KS);  // into the stage S(t) has freed
-        if (ok) ok = issue_pv(it, t);
-        if (ok && t + 2 < it.nkt) ok = issue_s(it, t + 2);
-        if (ok && t + VS < it.nkt) ok = issue_v(it, t + VS);
-      }
-      g += it.nkt;
     }
     if (lane == 0) {  // no MMA of this CTA may still run when TMEM is freed
       umma_commit(drain);
@@ -311,16 +356,19 @@ __global__ void __launch_bounds__(160, 1)
     const float sc = fabsf(scale_log2);
     int g = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
-      const Item it = load_item(item);
+    for (int k = 0; k < my_items && ok; ++k) {
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(qfull(k % QS), (k / QS) & 1, kWhereWaitQ, abort_flag));
+      if (!ok) break;
+      const TcItem it = *item_slot(k);
       const int i = r / s.gs, gi = r % s.gs;
       const bool valid = i < it.nq && gi < it.rows;
       const int lim = it.pos0 + i + 1;  // keys visible to this row
       float m = -INFINITY;              // reference maximum P is taken against (log2 units)
-      float l = 0.f;                    // sum of P against that reference
+      float l = 0.f;                    // sum of the rounded P against that reference
       for (int t = 0; t < it.nkt && ok; ++t) {
         const int gt = g + t, b = gt & 1;
-        // scores of this tile, and P buffer b free (PV two tiles back done)
+        // scores of this tile, and P buffer b free (the PV two tiles back done)
         ok = __all_sync(0xffffffffu,
                         mbar_wait(sfull(b), (gt >> 1) & 1, kWhereWaitMma, abort_flag) &&
                             mbar_wait(pfree(b), ((gt >> 1) & 1) ^ 1, kWhereWaitMma, abort_flag));
@@ -375,42 +423,32 @@ __global__ void __launch_bounds__(160, 1)
             for (int j = 0; j < 64; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
             tmem_st64(t_o + lane_base + c * 64, ro);
           }
-          tmem_st_wait();
         }
         l *= alpha;
         // P = 2^(x - m), rounded to the input type, into P buffer b
         const float nm = m == -INFINITY ? 0.f : -m;
-        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[kTcKeys / 2];
         if (nvis >= kTcKeys) {
 #pragma unroll
-          for (int j = 0; j < kTcKeys / 2; ++j) {
-            const float p0 = ex2_approx(fmaf(x[2 * j], sc, nm));
-            const float p1 = ex2_approx(fmaf(x[2 * j + 1], sc, nm));
-            ps4[j & 3] += p0 + p1;
-            pk[j] = pack2<T>(p0, p1);
-          }
+          for (int j = 0; j < kTcKeys / 2; ++j)
+            pk[j] = pack2<T>(ex2_approx(fmaf(x[2 * j], sc, nm)),
+                             ex2_approx(fmaf(x[2 * j + 1], sc, nm)));
         } else {
 #pragma unroll
           for (int j = 0; j < kTcKeys / 2; ++j) {
             const float p0 = 2 * j < nvis ? ex2_approx(fmaf(x[2 * j], sc, nm)) : 0.f;
             const float p1 = 2 * j + 1 < nvis ? ex2_approx(fmaf(x[2 * j + 1], sc, nm)) : 0.f;
-            ps4[j & 3] += p0 + p1;
             pk[j] = pack2<T>(p0, p1);
           }
         }
-        // keys 64c .. 64c+63 are one 128-byte row of P half c
-        const uint32_t prow = L::kOffP + b * L::kPBytes + r * 128;
+        tmem_st64(t_p(b) + lane_base, pk);
+        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-          for (int q8 = 0; q8 < 8; ++q8) {
-            const int j = c * 32 + q8 * 4;
-            *reinterpret_cast<uint4*>(smem + prow + c * L::kHalfBytes + ((q8 ^ (r & 7)) << 4)) =
-                make_uint4(pk[j], pk[j + 1], pk[j + 2], pk[j + 3]);
-          }
+        for (int j = 0; j < kTcKeys / 2; ++j) {  // sum the same rounded weights P.V uses
+          const float2 f = unpack2<T>(pk[j]);
+          ps4[j & 3] += f.x + f.y;
         }
-        fence_proxy_async_smem();
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pfull(b));
