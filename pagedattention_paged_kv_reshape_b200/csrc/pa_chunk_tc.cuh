@@ -13,21 +13,25 @@
 //   16-token TMA boxes per 128-key tile, in K and V rings) into shared memory
 //   with 128-byte swizzling, which is exactly the canonical K-major layout
 //   (Q, K) and MN-major layout (V) the tcgen05 shared-memory descriptors
-//   describe.  It runs ahead of the tensor core as far as the rings allow,
-//   and hands each item's metadata to the other warps through shared memory;
-// * an MMA warp walks the CTA's tiles as one sequence across items: S = Q K^T
-//   (M=128, N=128, K=16 steps) into one of two TMEM score buffers, two tiles
-//   ahead of O += P V, so the tensor core computes the next scores while the
-//   softmax warps work, also across the boundary between two items;
-// * four softmax warps read a tile's scores with one round of tcgen05.ld (a
-//   whole 128-key row per thread), apply the causal mask (key <= position)
-//   and the online softmax in the log2 domain, and write P (rounded to the
-//   input type) back into TMEM, where the PV MMA reads it as its A operand;
+//   describe.  It walks the CTA's tiles as one sequence, K one tile ahead of
+//   V, runs ahead of the tensor core as far as the rings allow, fetches item
+//   metadata one to two items ahead, and hands it to the other warps through
+//   shared memory;
+// * an MMA warp walks the same sequence: S = Q K^T (M=128, N=128, K=16 steps)
+//   into one of two TMEM score buffers, two tiles ahead of O += P V, so the
+//   tensor core computes the next scores while the softmax warps work, also
+//   across the boundary between two items;
+// * eight softmax warps, two threads per tile row: each reads the row's 128
+//   scores with one round of tcgen05.ld and takes the row maximum under the
+//   causal mask (key <= position), then exponentiates its half of the keys
+//   (online softmax in the log2 domain) and writes P, rounded to the input
+//   type, into TMEM, where the PV MMA reads it as its A operand;
 // * O lives in TMEM for the whole item.  The running maximum that P is taken
 //   against is raised only when a row's maximum grows by more than 2^8 (P then
 //   stays below 256); only then is the row's O brought to the new reference
-//   point, through TMEM, between two PV steps.  The epilogue reads O once and
-//   divides by the row sum (of the rounded P that the PV MMA used).
+//   point, through TMEM, between two PV steps.  The epilogue adds the two
+//   halves of the row sum (of the rounded P the PV MMA used), reads O once
+//   and divides.
 //
 // Every wait is bounded.  TMEM (512 columns) is freed on every path, after a
 // final commit has drained the MMAs this CTA issued.  The kernel is launched
@@ -69,19 +73,21 @@ struct TcLayout {
   static constexpr int kBarVFull = kBarKEmpty + kKStages;
   static constexpr int kBarVEmpty = kBarVFull + kVStages;
   static constexpr int kBarSFull = kBarVEmpty + kVStages;  // S(b) written
-  static constexpr int kBarPFull = kBarSFull + 2;          // P(b) written (4 warps)
+  static constexpr int kBarPFull = kBarSFull + 2;          // P(b) written (8 warps)
   static constexpr int kBarPFree = kBarPFull + 2;          // the PV that read P(b) done
-  static constexpr int kBarDrain = kBarPFree + 2;
+  static constexpr int kBarPair = kBarPFree + 2;           // the two warps of a row quarter
+  static constexpr int kBarDrain = kBarPair + 4;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffItems = kOffBar + kNumBars * 8;
   static constexpr int kItemBytes = 48;
-  static constexpr int kOffTmem = kOffItems + kTcItemSlots * kItemBytes;
+  static constexpr int kOffLsum = kOffItems + kTcItemSlots * kItemBytes;  // [2 halves][128 rows]
+  static constexpr int kOffTmem = kOffLsum + 2 * kTcRows * 4;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 12;
   // at least ~114 KB, so that a single CTA fits per SM and its TMEM
   // allocation can never wait for another CTA's
   static constexpr int kSmem = (kBytes + 1024) > 116 * 1024 ? (kBytes + 1024) : 116 * 1024;
-  static constexpr int kThreads = 192;  // 4 softmax warps, 1 load warp, 1 MMA warp
+  static constexpr int kThreads = 320;  // 8 softmax warps, 1 load warp, 1 MMA warp
   // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256 + D), P0 [384,448), P1 [448,512)
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffBar % 1024 == 0, "1 KB alignment");
@@ -94,7 +100,7 @@ struct TcItem {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, Shape s, T* __restrict__ out,
@@ -119,6 +125,7 @@ __global__ void __launch_bounds__(192, 1)
   auto sfull = [&](int b) { return bar(L::kBarSFull + b); };
   auto pfull = [&](int b) { return bar(L::kBarPFull + b); };
   auto pfree = [&](int b) { return bar(L::kBarPFree + b); };
+  auto pairbar = [&](int quad) { return bar(L::kBarPair + quad); };
   const uint32_t drain = bar(L::kBarDrain);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
@@ -133,8 +140,12 @@ __global__ void __launch_bounds__(192, 1)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
-    for (int i = 0; i < L::kNumBars; ++i)  // P(b) is written by the four softmax warps
-      mbar_init(bar(i), (i == L::kBarPFull || i == L::kBarPFull + 1) ? 4 : 1);
+    for (int i = 0; i < L::kNumBars; ++i) {
+      int n = 1;
+      if (i == L::kBarPFull || i == L::kBarPFull + 1) n = 8;  // the eight softmax warps
+      if (i >= L::kBarPair && i < L::kBarPair + 4) n = 2;     // the two warps of a pair
+      mbar_init(bar(i), n);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -157,35 +168,45 @@ __global__ void __launch_bounds__(192, 1)
                            ? (items - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
                            : 0;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------- TMA loads
     const int qt = kTcRows / s.gs;
-    int g = 0;  // tiles of earlier items
-    bool ok = true;
-    for (int k = 0; k < my_items && ok; ++k) {
+    // Item metadata is fetched ahead: the chunk-list entry of item k + 2 and
+    // the row data of item k + 1 are in flight while item k is issued.
+    auto entry_of = [&](int k) -> int2 {
+      return k < my_items ? __ldcg(w.chunk_list + (blockIdx.x + k * gridDim.x) % count)
+                          : make_int2(0, 0);
+    };
+    auto row_data = [&](int k, int2 ent) -> int3 {  // (qsl[row], qsl[row + 1], seq_lens[row])
+      return k < my_items ? make_int3(__ldcg(qsl + ent.x), __ldcg(qsl + ent.x + 1),
+                                      __ldcg(seq_lens + ent.x))
+                          : make_int3(0, 0, 0);
+    };
+    auto make_item = [&](int k, int2 ent, int3 rd) {
       TcItem it;
-      {
-        const int item = blockIdx.x + k * gridDim.x;
-        const int e = item % count;
-        const int hu = item / count;
-        const int2 ent = __ldcg(w.chunk_list + e);
-        const RowInfo ri = load_row(s, qsl, seq_lens, ent.x);
-        const int slice = hu % s.ns;
-        it.row = ent.x;
-        it.kvh = hu / s.ns;
-        it.head0 = it.kvh * s.group + slice * 16;
-        it.rows = min(s.gs, s.group - slice * 16);
-        it.nq = min(qt, ri.q_len - ent.y);
-        it.token0 = ri.token0 + ent.y;
-        it.pos0 = ri.seq_len - ri.q_len + ent.y;
-        it.kv_end = it.pos0 + it.nq;
-        it.nkt = ceil_div(it.kv_end, kTcKeys);
-      }
+      const int hu = (blockIdx.x + k * gridDim.x) / count;
+      const int slice = hu % s.ns;
+      const int q_len = rd.y - rd.x;
+      it.row = ent.x;
+      it.kvh = hu / s.ns;
+      it.head0 = it.kvh * s.group + slice * 16;
+      it.rows = min(s.gs, s.group - slice * 16);
+      it.nq = min(qt, q_len - ent.y);
+      it.token0 = rd.x + ent.y;
+      it.pos0 = rd.z - q_len + ent.y;
+      it.kv_end = it.pos0 + it.nq;
+      it.nkt = ceil_div(it.kv_end, kTcKeys);
+      return it;
+    };
+    bool ok = true;
+    // make item k current: publish its metadata and load its Q
+    auto publish = [&](int k, const TcItem& it) -> bool {
       const int qb = k % QS;
+      bool r = true;
       if (lane == 0) {
         // Q buffer qb was last read by the S MMAs of item k - 2
-        ok = mbar_wait(qfree(qb), ((k / QS) & 1) ^ 1, kWhereWaitQ, abort_flag);
-        if (ok) {
+        r = mbar_wait(qfree(qb), ((k / QS) & 1) ^ 1, kWhereWaitQ, abort_flag);
+        if (r) {
           *item_slot(k) = it;
           mbar_arrive_expect_tx(qfull(qb), static_cast<uint32_t>(L::kTileBytes));
 #pragma unroll
@@ -194,10 +215,45 @@ __global__ void __launch_bounds__(192, 1)
                         it.token0);
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      return __shfl_sync(0xffffffffu, r, 0);
+    };
+    // V of a tile reuses the block ids its K looked up; at most two tiles
+    // wait for their V (the older one is issued right after a new K).
+    struct Pending {
+      int y, nb, gt;
+    };
+    Pending va{0, 0, 0}, vb{0, 0, 0};
+    int npend = 0;
+    auto issue_v = [&](const Pending& p) -> bool {
+      const int vs = p.gt % VS;
+      bool r = true;
+      if (lane == 0) {
+        r = mbar_wait(vempty(vs), ((p.gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+        if (r) mbar_arrive_expect_tx(vfull(vs), static_cast<uint32_t>(p.nb * L::kHalves * 2048));
+      }
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r && lane < p.nb) {
+#pragma unroll
+        for (int h = 0; h < L::kHalves; ++h)
+          tma_load_2d(v_smem(vs) + h * L::kHalfBytes + lane * 2048, &tm_v, vfull(vs), h * 64,
+                      p.y);
+      }
+      return r;
+    };
+    int2 ent1 = entry_of(1);
+    TcItem it;
+    if (my_items > 0) {
+      const int2 ent0 = entry_of(0);
+      it = make_item(0, ent0, row_data(0, ent0));
+    }
+    int3 rd1 = row_data(1, ent1);
+    int2 ent2 = entry_of(2);
+    if (my_items > 0) ok = publish(0, it);
+    int g = 0;  // tiles of earlier items
+    for (int k = 0; k < my_items && ok;) {
       for (int t = 0; t < it.nkt && ok; ++t) {
-        const int gt = g + t, ks = gt % KS, vs = gt % VS;
-        // one lane per 16-token block of the tile: its id, then its K and V boxes
+        const int gt = g + t, ks = gt % KS;
+        // one lane per 16-token block of the tile: its id, then its K boxes
         const int first = t * (kTcKeys / kBlock);
         const int nb = min(kTcKeys / kBlock, ceil_div(it.kv_end, kBlock) - first);
         int y = 0;
@@ -209,11 +265,10 @@ __global__ void __launch_bounds__(192, 1)
           }
           y = (pb * s.num_kv_heads + it.kvh) * kBlock;
         }
-        const uint32_t tx = static_cast<uint32_t>(nb * L::kHalves * 2048);
         bool r = true;
         if (lane == 0) {
           r = mbar_wait(kempty(ks), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-          if (r) mbar_arrive_expect_tx(kfull(ks), tx);
+          if (r) mbar_arrive_expect_tx(kfull(ks), static_cast<uint32_t>(nb * L::kHalves * 2048));
         }
         ok = __shfl_sync(0xffffffffu, r, 0);
         if (!ok) break;
@@ -223,22 +278,27 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_2d(k_smem(ks) + h * L::kHalfBytes + lane * 2048, &tm_k, kfull(ks), h * 64,
                         y);
         }
-        if (lane == 0) {
-          r = mbar_wait(vempty(vs), ((gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-          if (r) mbar_arrive_expect_tx(vfull(vs), tx);
-        }
-        ok = __shfl_sync(0xffffffffu, r, 0);
-        if (!ok) break;
-        if (lane < nb) {
-#pragma unroll
-          for (int h = 0; h < L::kHalves; ++h)
-            tma_load_2d(v_smem(vs) + h * L::kHalfBytes + lane * 2048, &tm_v, vfull(vs), h * 64,
-                        y);
+        // queue this tile's V; issue the previous tile's
+        if (npend == 0) {
+          va = Pending{y, nb, gt};
+          npend = 1;
+        } else {
+          vb = Pending{y, nb, gt};
+          ok = issue_v(va);
+          va = vb;
         }
       }
       g += it.nkt;
+      if (++k < my_items && ok) {
+        it = make_item(k, ent1, rd1);
+        ent1 = ent2;
+        rd1 = row_data(k + 1, ent1);
+        ent2 = entry_of(k + 2);
+        ok = publish(k, it);
+      }
     }
-  } else if (warp == 5) {
+    if (ok && npend == 1) issue_v(va);  // the last tile's V
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issue
     // The CTA's tiles form one sequence gt = 0, 1, 2, ... across its items.
     // S(gt + 2) is issued right after PV(gt): by then the softmax warps have
@@ -348,12 +408,19 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------- softmax warps
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int r = tid;  // tile row = TMEM lane
+    // Warps q and q + 4 share TMEM lanes 32q .. 32q + 31 (tile rows): both
+    // take the row maximum over all 128 keys of a tile, warp q exponentiates
+    // keys 0 .. 63, warp q + 4 keys 64 .. 127, and O's columns are split the
+    // same way.
+    const int quad = warp & 3, h = warp >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int r = quad * 32 + lane;  // tile row = TMEM lane
+    float* lsum = reinterpret_cast<float*>(smem + L::kOffLsum);  // [2][128]
     // Scores enter as x = s * |scale| after a sign flip of s for a negative
     // scale, so that the row maximum is always a max.
     const bool neg = scale_log2 < 0.f;
     const float sc = fabsf(scale_log2);
+    constexpr int kHalfD = D / 2;
     int g = 0;
     bool ok = true;
     for (int k = 0; k < my_items && ok; ++k) {
@@ -365,7 +432,7 @@ __global__ void __launch_bounds__(192, 1)
       const bool valid = i < it.nq && gi < it.rows;
       const int lim = it.pos0 + i + 1;  // keys visible to this row
       float m = -INFINITY;              // reference maximum P is taken against (log2 units)
-      float l = 0.f;                    // sum of the rounded P against that reference
+      float l = 0.f;                    // this half's sum of the rounded P
       for (int t = 0; t < it.nkt && ok; ++t) {
         const int gt = g + t, b = gt & 1;
         // scores of this tile, and P buffer b free (the PV two tiles back done)
@@ -374,30 +441,41 @@ __global__ void __launch_bounds__(192, 1)
                             mbar_wait(pfree(b), ((gt >> 1) & 1) ^ 1, kWhereWaitMma, abort_flag));
         if (!ok) break;
         tc_fence_after();
+        // x: this thread's half of the keys (h*64 ..), y: the other half
         uint32_t ra[64], rb[64];
-        tmem_ld64_issue(t_s(b) + lane_base, ra);
-        tmem_ld64_issue(t_s(b) + lane_base + 64, rb);
+        tmem_ld64_issue(t_s(b) + lane_base + h * 64, ra);
+        tmem_ld64_issue(t_s(b) + lane_base + (h ^ 1) * 64, rb);
         tmem_ld_wait(ra);
         reg_tie(rb);
-        float x[kTcKeys];
+        float x[64], y[64];
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
           x[j] = __uint_as_float(ra[j]);
-          x[64 + j] = __uint_as_float(rb[j]);
+          y[j] = __uint_as_float(rb[j]);
         }
         if (neg) {
 #pragma unroll
-          for (int j = 0; j < kTcKeys; ++j) x[j] = -x[j];
+          for (int j = 0; j < 64; ++j) {
+            x[j] = -x[j];
+            y[j] = -y[j];
+          }
         }
         const int nvis = lim - t * kTcKeys;  // keys of this tile this row may see
+        const int hv = nvis - h * 64;        // ... of this thread's half
+        const int ov = nvis - (h ^ 1) * 64;  // ... of the other half
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (nvis >= kTcKeys) {
 #pragma unroll
-          for (int j = 0; j < kTcKeys; ++j) m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+          for (int j = 0; j < 64; j += 2) {
+            m4[(j >> 1) & 1] = fmax3(m4[(j >> 1) & 1], x[j], x[j + 1]);
+            m4[2 + ((j >> 1) & 1)] = fmax3(m4[2 + ((j >> 1) & 1)], y[j], y[j + 1]);
+          }
         } else {
 #pragma unroll
-          for (int j = 0; j < kTcKeys; ++j)
-            if (j < nvis) m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+          for (int j = 0; j < 64; ++j) {
+            if (j < hv) m4[j & 1] = fmaxf(m4[j & 1], x[j]);
+            if (j < ov) m4[2 + (j & 1)] = fmaxf(m4[2 + (j & 1)], y[j]);
+          }
         }
         const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
         // raise the reference maximum only when the row maximum has grown by
@@ -409,63 +487,72 @@ __global__ void __launch_bounds__(192, 1)
           m = mx;
         }
         if (t > 0 && __any_sync(0xffffffffu, raise)) {
-          // O holds PV of tiles 0 .. t-1: once PV(t-1) is done, scale it
+          // O holds PV of tiles 0 .. t-1: once PV(t-1) is done, scale this
+          // thread's half of the row
           ok = __all_sync(0xffffffffu, mbar_wait(pfree((gt - 1) & 1), ((gt - 1) >> 1) & 1,
                                                  kWhereWaitMma, abort_flag));
           if (!ok) break;
           tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < D / 64; ++c) {
+          if constexpr (kHalfD == 64) {
             uint32_t ro[64];
-            tmem_ld64_issue(t_o + lane_base + c * 64, ro);
+            tmem_ld64_issue(t_o + lane_base + h * kHalfD, ro);
             tmem_ld_wait(ro);
 #pragma unroll
             for (int j = 0; j < 64; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
-            tmem_st64(t_o + lane_base + c * 64, ro);
+            tmem_st64(t_o + lane_base + h * kHalfD, ro);
+          } else {
+            uint32_t ro[32];
+            tmem_ld32_issue(t_o + lane_base + h * kHalfD, ro);
+            tmem_ld_wait(ro);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
+            tmem_st32(t_o + lane_base + h * kHalfD, ro);
           }
         }
         l *= alpha;
-        // P = 2^(x - m), rounded to the input type, into P buffer b
+        // P = 2^(x - m) for this half, rounded to the input type, into P(b)
         const float nm = m == -INFINITY ? 0.f : -m;
-        uint32_t pk[kTcKeys / 2];
-        if (nvis >= kTcKeys) {
+        const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(nm, nm);
+        uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < kTcKeys / 2; ++j)
-            pk[j] = pack2<T>(ex2_approx(fmaf(x[2 * j], sc, nm)),
-                             ex2_approx(fmaf(x[2 * j + 1], sc, nm)));
-        } else {
-#pragma unroll
-          for (int j = 0; j < kTcKeys / 2; ++j) {
-            const float p0 = 2 * j < nvis ? ex2_approx(fmaf(x[2 * j], sc, nm)) : 0.f;
-            const float p1 = 2 * j + 1 < nvis ? ex2_approx(fmaf(x[2 * j + 1], sc, nm)) : 0.f;
-            pk[j] = pack2<T>(p0, p1);
+        for (int j = 0; j < 32; ++j) {
+          const float2 a = ffma2(make_float2(x[2 * j], x[2 * j + 1]), sc2, nm2);
+          float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y);
+          if (hv < 64) {
+            p0 = 2 * j < hv ? p0 : 0.f;
+            p1 = 2 * j + 1 < hv ? p1 : 0.f;
           }
+          pk[j] = pack2<T>(p0, p1);
         }
-        tmem_st64(t_p(b) + lane_base, pk);
-        float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+        tmem_st32(t_p(b) + lane_base + h * 32, pk);
+        float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int j = 0; j < kTcKeys / 2; ++j) {  // sum the same rounded weights P.V uses
-          const float2 f = unpack2<T>(pk[j]);
-          ps4[j & 3] += f.x + f.y;
-        }
+        for (int j = 0; j < 32; ++j)  // sum the same rounded weights P.V uses
+          ps[j & 1] = fadd2(ps[j & 1], unpack2<T>(pk[j]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pfull(b));
-        l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+        l += (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y);
       }
       if (ok) {
+        // both halves of the row sum, through shared memory
+        lsum[h * kTcRows + r] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pairbar(quad));
+        ok = __all_sync(0xffffffffu, mbar_wait(pairbar(quad), k & 1, kWhereWaitMma, abort_flag));
+        const float lt = l + lsum[(h ^ 1) * kTcRows + r];
         // the item's last PV done: O is final
         const int gl = g + it.nkt - 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(pfree(gl & 1), (gl >> 1) & 1, kWhereWaitMma,
-                                               abort_flag));
+        if (ok)
+          ok = __all_sync(0xffffffffu, mbar_wait(pfree(gl & 1), (gl >> 1) & 1, kWhereWaitMma,
+                                                 abort_flag));
         if (ok) {
           tc_fence_after();
-          const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll 1
-          for (int c = 0; c < D / 64; ++c) {
+          const float inv = lt > 0.f ? 1.f / lt : 0.f;
+          if constexpr (kHalfD == 64) {
             uint32_t ro[64];
-            tmem_ld64_issue(t_o + lane_base + c * 64, ro);
+            tmem_ld64_issue(t_o + lane_base + h * kHalfD, ro);
             tmem_ld_wait(ro);
             if (valid) {
 #pragma unroll
@@ -473,7 +560,20 @@ __global__ void __launch_bounds__(192, 1)
                 float a[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(ro[q * 8 + e]);
-                store_row8<T, D>(s, out, it.token0 + i, it.head0 + gi, c * 8 + q, a, inv);
+                store_row8<T, D>(s, out, it.token0 + i, it.head0 + gi, h * 8 + q, a, inv);
+              }
+            }
+          } else {
+            uint32_t ro[32];
+            tmem_ld32_issue(t_o + lane_base + h * kHalfD, ro);
+            tmem_ld_wait(ro);
+            if (valid) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                float a[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(ro[q * 8 + e]);
+                store_row8<T, D>(s, out, it.token0 + i, it.head0 + gi, h * 4 + q, a, inv);
               }
             }
           }
