@@ -362,6 +362,52 @@ def combine_over_ranks(local_ms: float, local_bytes: float, local_tokens: float,
     return max_ms, nb.item() / (max_ms / 1e3) / 1e9, tok.item() / (max_ms / 1e3)
 
 
+def measure_block_ops(torch, pa, dev, peak) -> dict:
+    """Copy-on-write copies inside the device pool and swaps to / from a pinned
+    host pool, each on 2048 / 1024 blocks of 8 KV heads x 16 x 128 bf16
+    (64 KB of K+V per block; 256 MB of HBM traffic per copy call, more than
+    the L2).  GB/s count the bytes each call reads plus writes (copy) or
+    moves (swap)."""
+    nb, hkv, d = 6144, 8, 128
+    g = torch.Generator(device=dev).manual_seed(1234)
+    k = torch.randn(nb, hkv, 16, d, generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn(nb, hkv, 16, d, generator=g, device=dev).to(torch.bfloat16)
+    block_bytes = 2 * hkv * 16 * d * 2
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(1234))
+    n_copy, n_swap = 2048, 1024
+    cmap = torch.stack([perm[:n_copy], perm[n_copy:2 * n_copy]], 1).int().to(dev)
+    host_k = torch.empty(n_swap, hkv, 16, d, dtype=torch.bfloat16).pin_memory()
+    host_v = torch.empty_like(host_k).pin_memory()
+    omap = torch.stack([perm[:n_swap], torch.arange(n_swap)], 1).int().to(dev)
+    imap = torch.stack([torch.arange(n_swap), perm[2 * n_copy:2 * n_copy + n_swap]], 1).int().to(dev)
+
+    def timed(fn, iters=10):
+        for _ in range(3):
+            fn()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        s.record()
+        for _ in range(iters):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / iters
+
+    copy_ms = timed(lambda: pa.pa_copy_blocks(k, v, cmap))
+    out_ms = timed(lambda: pa.pa_swap_blocks(k, v, host_k, host_v, omap))
+    in_ms = timed(lambda: pa.pa_swap_blocks(host_k, host_v, k, v, imap))
+    pa.pa_get_device_error()
+    copy_gbs = 2 * n_copy * block_bytes / (copy_ms / 1e3) / 1e9
+    return {"copy_blocks": {"pairs": n_copy, "ms": round(copy_ms, 4),
+                            "gbs_read_plus_write": round(copy_gbs, 1),
+                            "pct_of_hbm_peak": round(100 * copy_gbs / peak, 1)},
+            "swap_out": {"blocks": n_swap, "ms": round(out_ms, 4),
+                         "gbs": round(n_swap * block_bytes / (out_ms / 1e3) / 1e9, 1)},
+            "swap_in": {"blocks": n_swap, "ms": round(in_ms, 4),
+                        "gbs": round(n_swap * block_bytes / (in_ms / 1e3) / 1e9, 1)},
+            "blocks": "8 KV heads x 16 tokens x 128 dims, bf16, K and V"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -477,6 +523,7 @@ def run_ours(args):
                        "tokens_per_s": round(b.total_q / (attn / 1e3), 1)}
             per[name] = ent
         result["per_config"] = per
+        result["block_ops"] = measure_block_ops(torch, pa, dev, peak)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         del b

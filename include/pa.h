@@ -17,12 +17,16 @@
  *      ("vLLM 深度拆解" §4.3 chunked prefill; "vLLM 架构源码解析" §3.2 unified
  *      token budget and §3.3.2 query_start_loc / positions / seq_lens).
  *
+ * and the block operations next to it: pa_copy_blocks (copy-on-write) and
+ * pa_swap_blocks (swap-out / swap-in between the device and a host pool).
+ *
  * Attention is softmax(q . K^T * scale) . V ("vLLM 深度拆解" §2.2).
  *
  * Conventions shared by every call
  * --------------------------------
  * - Every pointer argument except the returned strings is a DEVICE pointer on
- *   the current CUDA device, owned by the caller.  The library keeps no
+ *   the current CUDA device, owned by the caller (pa_swap_blocks also takes
+ *   page-locked host memory).  The library keeps no
  *   pointer after the call returns and allocates no device memory: scratch
  *   space is the caller's `workspace`, sized by the *_workspace_size query
  *   (pa_decode_static uses a fixed array built into the library instead).
@@ -120,6 +124,56 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
                                const int32_t* slot_mapping, int num_tokens, int num_kv_heads,
                                int head_dim, int block_size, int num_blocks, pa_dtype dtype,
                                void* stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copies inside one pool.
+ *
+ * Blocks are shared by reference count ("2. 核心思想" §核心抽象: ref_cnt
+ * supports copy-on-write and sharing across requests; "vLLM 架构源码解析"
+ * §4.3.2: parallel samples share the prompt's blocks).  Before a request
+ * writes into a block that another request still references, the engine
+ * gives it a private copy; this call makes those copies.
+ *
+ *   k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim]
+ *   block_mapping     int32 [num_pairs][2] = (src, dst), device memory: block
+ *                     dst of both caches becomes a byte copy of block src
+ *                     (every KV head, every slot)
+ *
+ * Pairs must be independent: no dst may be another pair's src or dst (the
+ * order among pairs is unspecified).  src == dst is a no-op.  A pair with an
+ * id outside [0, num_blocks) is skipped and recorded as PA_ERR_DEVICE_BOUNDS.
+ * num_pairs == 0 is a no-op.
+ */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, void* stream);
+
+/*
+ * pa_swap_blocks -- move blocks between two pools, e.g. the device pool and
+ * a pool in host memory.
+ *
+ * The v0 scheduler preempts a request by swapping its KV cache out to CPU
+ * memory and swaps it back into the GPU pool when the request resumes
+ * ("vLLM 架构源码解析" §1, the preemption table: v0 (Swap)).
+ *
+ *   src_k, src_v  [src_num_blocks, num_kv_heads, block_size, head_dim]
+ *   dst_k, dst_v  [dst_num_blocks, num_kv_heads, block_size, head_dim]
+ *   block_mapping int32 [num_pairs][2] = (src, dst): block dst of (dst_k,
+ *                 dst_v) becomes a byte copy of block src of (src_k, src_v)
+ *
+ * Unlike every other call, the pools and block_mapping may each be device
+ * memory or page-locked host memory (cudaHostAlloc / cudaHostRegister, e.g.
+ * torch's pin_memory()); the kernel reads and writes host memory through
+ * its device-visible address, so a swap is one launch however many blocks
+ * it moves.  Pageable host memory is refused (PA_ERR_INVALID_ARG).  The
+ * caller keeps the host buffers alive and unmodified until the stream has
+ * passed the call.  Pair rules and errors as for pa_copy_blocks (ids are
+ * checked against the pool each side of the pair belongs to).
+ */
+pa_status pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                         const int32_t* block_mapping, int num_pairs, int num_kv_heads,
+                         int head_dim, int block_size, int src_num_blocks, int dst_num_blocks,
+                         pa_dtype dtype, void* stream);
 
 /*
  * Workspace (bytes) pa_decode needs for these sizes.  Includes the split-K

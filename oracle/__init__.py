@@ -35,3 +35,4 @@ from .paged_attention import (  # noqa: F401
     paged_varlen,
     default_scale,
 )
+from .block_ops import copy_blocks, swap_blocks  # noqa: F401,E402

@@ -7,7 +7,9 @@ kernels, and this thin Python binding of it:
 * :func:`pa_reshape_and_cache` -- scatter new K/V rows into 16-token blocks;
 * :func:`pa_decode` -- block-table-indirected decode attention (GQA, online
   softmax, split-K with a log-sum-exp reduce);
-* :func:`pa_varlen` -- mixed batches of decode rows and causal prefill chunks.
+* :func:`pa_varlen` -- mixed batches of decode rows and causal prefill chunks;
+* :func:`pa_copy_blocks` / :func:`pa_swap_blocks` -- copy-on-write copies
+  inside a pool, swap-out / swap-in between the device and a host pool.
 
 PyTorch provides device memory and streams only.  The seeded workload
 generator lives in :mod:`.workload`; byte/flop accounting in :mod:`.accounting`.
@@ -21,6 +23,7 @@ from ._binding import (  # noqa: F401
     alloc_workspace,
     lib,
     STATIC_WORKSPACE_BYTES,
+    pa_copy_blocks,
     pa_decode,
     pa_decode_static,
     pa_decode_workspace_size,
@@ -28,6 +31,7 @@ from ._binding import (  # noqa: F401
     pa_reshape_and_cache,
     pa_set_path,
     pa_status_string,
+    pa_swap_blocks,
     pa_varlen,
     pa_varlen_workspace_size,
     pa_version,

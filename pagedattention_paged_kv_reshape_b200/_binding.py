@@ -45,6 +45,10 @@ DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 _SIGNATURES = {
     "pa_reshape_and_cache": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                                       _c_int, _c_int, _vp]),
+    "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                _vp]),
+    "pa_swap_blocks": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                _c_int, _c_int, _vp]),
     "pa_decode_workspace_size": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "pa_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int, _c_int,
                            _c_int, _c_int, _c_int, _c_float, _vp, _c_size, _c_int, _vp]),
@@ -136,6 +140,48 @@ def pa_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None) -> N
         _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), k.shape[0],
         k.shape[1], k.shape[2], k_cache.shape[2], k_cache.shape[0], _dtype_code(k),
         _stream(stream)))
+
+
+def _pool_pair(k_pool, v_pool, what: str):
+    _require(k_pool.shape == v_pool.shape and k_pool.dim() == 4, f"{what} pools must be 4-D")
+    _require(k_pool.dtype == v_pool.dtype, f"{what} dtypes must match")
+    _require(k_pool.is_contiguous() and v_pool.is_contiguous(), f"{what} pools must be dense")
+
+
+def _block_mapping(block_mapping) -> int:
+    _require(block_mapping.dtype == torch.int32 and block_mapping.dim() == 2
+             and block_mapping.shape[1] == 2 and block_mapping.is_contiguous(),
+             "block_mapping must be a dense int32 [num_pairs, 2]")
+    return block_mapping.shape[0]
+
+
+def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
+    """Copy-on-write: for each row (src, dst) of ``block_mapping``, block ``dst``
+    of both caches becomes a copy of block ``src``."""
+    _dense(k_cache, v_cache, block_mapping)
+    _pool_pair(k_cache, v_cache, "cache")
+    n = _block_mapping(block_mapping)
+    nb, hkv, bs, d = k_cache.shape
+    _check(lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), n, hkv, d, bs,
+                                nb, _dtype_code(k_cache), _stream(stream)))
+
+
+def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, stream=None) -> None:
+    """Swap out / in: for each row (src, dst) of ``block_mapping``, block ``dst``
+    of (``dst_k``, ``dst_v``) becomes a copy of block ``src`` of (``src_k``,
+    ``src_v``).  Each pool and the mapping may be on the device or in pinned
+    host memory."""
+    for t in (src_k, src_v, dst_k, dst_v, block_mapping):
+        _require(t.is_cuda or t.is_pinned(), "host tensors must be pinned (pin_memory())")
+    _pool_pair(src_k, src_v, "source")
+    _pool_pair(dst_k, dst_v, "destination")
+    _require(src_k.shape[1:] == dst_k.shape[1:] and src_k.dtype == dst_k.dtype,
+             "source and destination blocks must have the same shape and dtype")
+    n = _block_mapping(block_mapping)
+    _, hkv, bs, d = src_k.shape
+    _check(lib().pa_swap_blocks(_ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v),
+                                _ptr(block_mapping), n, hkv, d, bs, src_k.shape[0],
+                                dst_k.shape[0], _dtype_code(src_k), _stream(stream)))
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,

@@ -15,6 +15,7 @@
 
 #include "pa_attn_mma.cuh"
 #include "pa_attn_simt.cuh"
+#include "pa_blocks.cuh"
 #include "pa_chunk_tc.cuh"
 #include "pa_reduce.cuh"
 #include "pa_reshape.cuh"
@@ -512,6 +513,91 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
   return PA_OK;
 }
 
+// Device-visible address of a pointer the kernels may dereference: device
+// memory as is, page-locked host memory through its mapped address.  Pageable
+// host memory is refused.
+static pa_status device_address(const void* p, const void** out, const char* what) {
+  cudaPointerAttributes at{};
+  const cudaError_t e = cudaPointerGetAttributes(&at, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PA_ERR_INVALID_ARG, "%s: not a CUDA-visible pointer", what);
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+    *out = p;
+    return PA_OK;
+  }
+  if (at.type == cudaMemoryTypeHost && at.devicePointer) {
+    *out = at.devicePointer;
+    return PA_OK;
+  }
+  return fail(PA_ERR_INVALID_ARG, "%s: host memory must be page-locked (cudaHostAlloc/Register)",
+              what);
+}
+
+static pa_status launch_block_copy(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                                   const int32_t* block_mapping, int num_pairs, int num_kv_heads,
+                                   int head_dim, int block_size, int src_num_blocks,
+                                   int dst_num_blocks, pa_dtype dtype, void* stream,
+                                   bool allow_host) {
+  if (!valid_dtype(dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || src_num_blocks < 0 ||
+      dst_num_blocks < 0)
+    return fail(PA_ERR_INVALID_ARG, "bad sizes");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
+  if (block_size != pa::kBlock)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 16)", block_size);
+  if (num_pairs == 0) return PA_OK;
+  const void* in[] = {src_k, src_v, dst_k, dst_v, block_mapping};
+  const char* names[] = {"src_k", "src_v", "dst_k", "dst_v", "block_mapping"};
+  const void* dev[5];
+  for (int i = 0; i < 5; ++i) {
+    if (!in[i]) return fail(PA_ERR_INVALID_ARG, "%s is null", names[i]);
+    if (!aligned(in[i], i < 4 ? 16 : 4))
+      return fail(PA_ERR_INVALID_ARG, "%s is not %d-byte aligned", names[i], i < 4 ? 16 : 4);
+    if (allow_host) {
+      const pa_status st = device_address(in[i], &dev[i], names[i]);
+      if (st != PA_OK) return st;
+    } else {
+      dev[i] = in[i];
+    }
+  }
+  const long long block_bytes =
+      static_cast<long long>(num_kv_heads) * block_size * head_dim * elem_bytes(dtype);
+  if (block_bytes / 16 > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "block too large");
+  const int block_vecs = static_cast<int>(block_bytes / 16);
+  const int chunks = (block_vecs + pa::kCopyThreads * pa::kCopyUnroll - 1) /
+                     (pa::kCopyThreads * pa::kCopyUnroll);
+  const long long grid = static_cast<long long>(num_pairs) * chunks;
+  if (grid > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many pairs");
+  pa::copy_blocks_kernel<<<dim3(static_cast<unsigned>(grid), 2), pa::kCopyThreads, 0,
+                           static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(dev[0]), static_cast<const uint4*>(dev[1]),
+      static_cast<uint4*>(const_cast<void*>(dev[2])), static_cast<uint4*>(const_cast<void*>(dev[3])),
+      static_cast<const int*>(dev[4]), src_num_blocks, dst_num_blocks, block_vecs, chunks);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "block copy launch");
+  return PA_OK;
+}
+
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* block_mapping,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, void* stream) {
+  return launch_block_copy(k_cache, v_cache, k_cache, v_cache, block_mapping, num_pairs,
+                           num_kv_heads, head_dim, block_size, num_blocks, num_blocks, dtype,
+                           stream, false);
+}
+
+pa_status pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                         const int32_t* block_mapping, int num_pairs, int num_kv_heads,
+                         int head_dim, int block_size, int src_num_blocks, int dst_num_blocks,
+                         pa_dtype dtype, void* stream) {
+  return launch_block_copy(src_k, src_v, dst_k, dst_v, block_mapping, num_pairs, num_kv_heads,
+                           head_dim, block_size, src_num_blocks, dst_num_blocks, dtype, stream,
+                           true);
+}
+
 size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                 int max_context_len) {
   if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
@@ -589,8 +675,9 @@ pa_status pa_get_device_error(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
   static const char* where[] = {"?", "reshape_and_cache slot", "block-table entry",
                                 "row metadata", "wait for K/V tile", "wait for free stage",
-                                "wait for query tile", "tensor memory", "wait for MMA/barrier"};
-  const int w = rec.where >= 0 && rec.where <= 8 ? rec.where : 0;
+                                "wait for query tile", "tensor memory", "wait for MMA/barrier",
+                                "block copy pair"};
+  const int w = rec.where >= 0 && rec.where <= 9 ? rec.where : 0;
   return fail(static_cast<pa_status>(rec.code), "device: %s (%s; a=%lld b=%lld)",
               pa_status_string(static_cast<pa_status>(rec.code)), where[w], rec.a, rec.b);
 }

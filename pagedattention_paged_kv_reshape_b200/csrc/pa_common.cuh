@@ -47,6 +47,7 @@ enum ErrWhere : int {
   kWhereWaitQ = 6,
   kWhereTmem = 7,
   kWhereWaitMma = 8,
+  kWhereCopyPair = 9,
 };
 
 __device__ __forceinline__ void report_error(unsigned code, int where, long long a, long long b) {

@@ -185,3 +185,22 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_binding, "LIBRARY_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         _binding.lib()
+
+
+@cpu_only
+def test_block_ops_reject_bad_arguments(lib):
+    # pa_copy_blocks(k, v, map, num_pairs, Hkv, D, block_size, num_blocks, dtype, stream)
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 0, 8, 128, 16, 10, 1, None) == pa.Status.OK
+    assert lib.pa_copy_blocks(None, FAKE, FAKE, 3, 8, 128, 16, 10, 1, None) == \
+        pa.Status.INVALID_ARG
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 3, 8, 80, 16, 10, 1, None) == \
+        pa.Status.UNSUPPORTED
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, -1, 8, 128, 16, 10, 1, None) == \
+        pa.Status.INVALID_ARG
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 3, 8, 128, 16, 10, 7, None) == \
+        pa.Status.INVALID_ARG
+    # pa_swap_blocks(src_k, src_v, dst_k, dst_v, map, n, Hkv, D, bs, src_nb, dst_nb, dtype, s)
+    assert lib.pa_swap_blocks(FAKE, FAKE, FAKE, None, FAKE, 3, 8, 128, 16, 10, 10, 1, None) == \
+        pa.Status.INVALID_ARG
+    assert lib.pa_swap_blocks(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 16, 10, 10, 1, None) == \
+        pa.Status.OK
