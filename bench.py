@@ -496,7 +496,8 @@ def run_ours(args):
     if not args.no_per_config:
         tensor_peak = measured_tensor_peak()
         per = {}
-        for name in ("gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512"):
+        for name in ("gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512", "gqa_bs256_b8",
+                     "gqa_bs256_b32"):
             if name == args.workload:
                 continue
             del b

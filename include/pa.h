@@ -3,8 +3,8 @@
  *
  * The hot path of a paged-KV serving engine's attention layer:
  *
- *   1. pa_reshape_and_cache  -- scatter this step's new K/V rows into 16-token
- *      physical blocks through a per-token slot mapping
+ *   1. pa_reshape_and_cache  -- scatter this step's new K/V rows into
+ *      physical blocks (8, 16 or 32 tokens) through a per-token slot mapping
  *      ("vLLM 架构源码解析 | 第 1 篇" §3.3.3: reshape_and_cache(k, v, kv_cache,
  *      slot_mapping) runs before paged_attention in every attention layer).
  *   2. pa_decode             -- one query row per request attends to its
@@ -44,11 +44,12 @@
  *   [blocks, block_size, d_k] in "vLLM 架构源码解析" §4.2; this one keeps a
  *   token's head_dim values contiguous so that one 16-byte load carries eight
  *   16-bit values of one token.)
- * - block_size must be 16 ("vLLM 架构源码解析" §1.1 and §5.1, the default).
+ * - block_size is 8, 16 or 32 tokens ("vLLM 架构源码解析" §5.1 weighs 8, 16
+ *   and 32 and passes block_size=32; 16 is the default of §1.1).
  * - block_tables is int32 [num_seqs, block_table_stride]: entry [r][j] is the
- *   physical block holding tokens j*16 .. j*16+15 of request r
- *   ("vLLM 深度拆解" §3.3: block_tables[seq_id * stride + block_idx]).
- *   Entries past ceil(len/16) are never read.
+ *   physical block holding tokens j*block_size .. (j+1)*block_size-1 of
+ *   request r ("vLLM 深度拆解" §3.3: block_tables[seq_id * stride +
+ *   block_idx]).  Entries past ceil(len/block_size) are never read.
  * - Grouped-query attention: query head h reads KV head
  *   h / (num_q_heads / num_kv_heads).  num_q_heads % num_kv_heads == 0.
  * - head_dim is 64 or 128.  dtype: PA_F32, PA_BF16 or PA_F16; q, k, v, the

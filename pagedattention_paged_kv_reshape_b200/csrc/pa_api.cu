@@ -263,6 +263,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+bool supported_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32; }
+
 pa_status check_common(const AttnArgs& a) {
   if (!valid_dtype(a.dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", a.dtype);
   if (a.num_seqs < 0 || a.total_q < 0 || a.max_query_len < 0 || a.max_seq_len < 0 ||
@@ -273,10 +275,10 @@ pa_status check_common(const AttnArgs& a) {
                 a.num_q_heads, a.num_kv_heads);
   if (a.head_dim != 64 && a.head_dim != 128)
     return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", a.head_dim);
-  if (a.block_size != pa::kBlock)
-    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 16)", a.block_size);
+  if (!supported_block_size(a.block_size))
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", a.block_size);
   if (!(std::isfinite(a.scale))) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
-  if (static_cast<long long>(a.num_blocks) * a.num_kv_heads * pa::kBlock > 0x7fffffffLL)
+  if (static_cast<long long>(a.num_blocks) * a.num_kv_heads * a.block_size > 0x7fffffffLL)
     return fail(PA_ERR_UNSUPPORTED, "pool of %d blocks x %d heads exceeds 2^31 token rows",
                 a.num_blocks, a.num_kv_heads);
   if (static_cast<long long>(a.total_q) * a.num_q_heads > 0x7fffffffLL)
@@ -320,10 +322,12 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "mma kernel set-up");
   CUtensorMap tk, tv, tq;
-  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * pa::kBlock;
-  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, pa::kBlock);
+  // one box = 16 cache rows, or one whole 8-token block
+  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
+  const int box_rows = a.block_size < pa::kBlock ? a.block_size : pa::kBlock;
+  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, box_rows);
   if (st != PA_OK) return st;
-  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, pa::kBlock);
+  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, box_rows);
   if (st != PA_OK) return st;
   st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.qpt);
   if (st != PA_OK) return st;
@@ -345,10 +349,12 @@ pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "chunk kernel set-up");
   CUtensorMap tk, tv, tq;
-  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * pa::kBlock;
-  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, pa::kBlock);
+  // one box = 16 cache rows, or one whole 8-token block
+  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
+  const int box_rows = a.block_size < pa::kBlock ? a.block_size : pa::kBlock;
+  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, box_rows);
   if (st != PA_OK) return st;
-  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, pa::kBlock);
+  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, box_rows);
   if (st != PA_OK) return st;
   st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.chunk_qt);
   if (st != PA_OK) return st;
@@ -421,6 +427,7 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
   Plan p = make_plan(a.num_seqs, a.total_q, a.num_q_heads, a.num_kv_heads, a.head_dim, max_len,
                      varlen);
   p.s.table_stride = a.table_stride;
+  p.s.block_size = a.block_size;
   p.s.num_blocks = a.num_blocks;
   p.s.max_seq_len = a.max_seq_len;
   p.s.max_query_len = varlen ? a.max_query_len : 1;
@@ -489,8 +496,8 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
     return fail(PA_ERR_INVALID_ARG, "bad sizes");
   if (head_dim != 64 && head_dim != 128)
     return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
-  if (block_size != pa::kBlock)
-    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 16)", block_size);
+  if (!supported_block_size(block_size))
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", block_size);
   if (num_tokens == 0) return PA_OK;
   const void* ptrs[] = {k, v, k_cache, v_cache};
   for (const void* p : ptrs) {
@@ -506,8 +513,8 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
   pa::reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), 256, 0,
                                  static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, row_vecs,
-      static_cast<long long>(num_blocks) * pa::kBlock);
+      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, row_vecs, block_size,
+      static_cast<long long>(num_blocks) * block_size);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache launch");
   return PA_OK;
@@ -546,8 +553,8 @@ static pa_status launch_block_copy(const void* src_k, const void* src_v, void* d
     return fail(PA_ERR_INVALID_ARG, "bad sizes");
   if (head_dim != 64 && head_dim != 128)
     return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
-  if (block_size != pa::kBlock)
-    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 16)", block_size);
+  if (!supported_block_size(block_size))
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", block_size);
   if (num_pairs == 0) return PA_OK;
   const void* in[] = {src_k, src_v, dst_k, dst_v, block_mapping};
   const char* names[] = {"src_k", "src_v", "dst_k", "dst_v", "block_mapping"};

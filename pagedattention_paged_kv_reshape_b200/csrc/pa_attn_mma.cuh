@@ -9,9 +9,10 @@
 //   logical]) into a ring of shared-memory slots, running several units ahead
 //   so that the dependent global loads of that lookup never delay the stream.
 // * The TMA warp takes each slot and issues cp.async.bulk.tensor loads of the
-//   tile's query rows and of every (block, KV head) K tile and V tile --
-//   16 tokens x head_dim, 4 KB each at bf16 x 128 -- into a STAGES-deep ring of
-//   shared-memory stages completed on mbarriers.  The tensor maps use 128-byte
+//   tile's query rows and of every 16-key K tile and V tile of the unit --
+//   16 tokens x head_dim, 4 KB each at bf16 x 128; one box of a 16- or
+//   32-token block, or two 8-row boxes of two 8-token blocks -- into a
+//   STAGES-deep ring of shared-memory stages completed on mbarriers.  The tensor maps use 128-byte
 //   swizzling, so the ldmatrix reads below are free of bank conflicts.
 // * Consumer warp w takes the unit's blocks w, w+NCW, ...: S = Q K^T (16 tile
 //   rows x 16 tokens, m16n8k16 MMAs, fp32 accumulate), masking of keys past
@@ -29,10 +30,13 @@ namespace pa {
 
 constexpr int kMetaSlots = 4;
 
-// One scheduler-ring slot: a decoded unit and its partition's block ids.
+// One scheduler-ring slot: a decoded unit and, for each 16-key tile of its
+// partition, the cache row of the tile's first key (y0) and, with 8-token
+// blocks, of its ninth key (y1; -1 when the tile has no second block).
 struct MetaSlot {
   Unit u;
-  int pb[kPart / kBlock];
+  int y0[kPart / kBlock];
+  int y1[kPart / kBlock];
 };
 
 template <int D, int NCW, int STAGES>
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
         next = __shfl_sync(0xffffffffu, nx, 0);
       }
       Unit un;
-      int e = 0;
+      int e = 0, e1 = -1;
       if (!done) {
         int local, cls;
         const int row = locate_unit_warp(s, w, total_a, unit, cur_a, cur_b, local, cls);
@@ -150,12 +154,13 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
         if (un.kv_begin >= un.kv_end) continue;  // no key of this partition is visible
         const int nblk = ceil_div(un.kv_end - un.kv_begin, kBlock);
         if (lane < nblk) {
-          e = __ldg(block_tables + static_cast<size_t>(row) * s.table_stride +
-                    un.kv_begin / kBlock + lane);
-          if (e < 0 || e >= s.num_blocks) {
-            report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, row, e);
-            e = 0;
-          }
+          const int* table = block_tables + static_cast<size_t>(row) * s.table_stride;
+          const int key = un.kv_begin + lane * kBlock;
+          e = key_row(table, key, s.block_size, s.num_kv_heads, un.kvh, s.num_blocks, row);
+          if (s.block_size < kBlock)
+            e1 = key + 8 < un.kv_end ? key_row(table, key + 8, s.block_size, s.num_kv_heads,
+                                               un.kvh, s.num_blocks, row)
+                                     : -1;
         }
       } else {
         un.row = -1;
@@ -166,7 +171,8 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
                                     abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      meta[ms].pb[lane] = e;
+      meta[ms].y0[lane] = e;
+      meta[ms].y1[lane] = e1;
       if (lane == 0) meta[ms].u = un;
       __syncwarp();
       if (lane == 0) mbar_arrive(mfull_bar(ms));
@@ -203,18 +209,32 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
         tma_load_3d(qdst + h * (kRows * 128), &tm_q, qfull_bar(qs), h * 64, un.head0, un.token0);
       const int nblk = ceil_div(un.kv_end - un.kv_begin, kBlock);
       for (int jj = 0; jj < nblk; ++jj, ++n) {
-        const int pb = meta[ms].pb[jj];
+        const int y = meta[ms].y0[jj];
         const int st = n % STAGES;
         if (!(ok = mbar_wait(empty_bar(st), ((n / STAGES) & 1) ^ 1, kWhereWaitEmpty, abort_flag)))
           break;
         ++issued;
-        mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
-        const int y = (pb * s.num_kv_heads + un.kvh) * kBlock;
         const uint32_t kdst = sbase + st * L::kStageBytes;
+        if (s.block_size >= kBlock) {  // one 16-row box per half
+          mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
 #pragma unroll
-        for (int h = 0; h < L::kHalves; ++h) {
-          tma_load_2d(kdst + h * L::kHalfBytes, &tm_k, full_bar(st), h * 64, y);
-          tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes, &tm_v, full_bar(st), h * 64, y);
+          for (int h = 0; h < L::kHalves; ++h) {
+            tma_load_2d(kdst + h * L::kHalfBytes, &tm_k, full_bar(st), h * 64, y);
+            tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes, &tm_v, full_bar(st), h * 64, y);
+          }
+        } else {  // 8-token blocks: rows 0-7 and, if the tile has them, rows 8-15
+          const int y1 = meta[ms].y1[jj];
+          mbar_arrive_expect_tx(full_bar(st), y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
+#pragma unroll
+          for (int h = 0; h < L::kHalves; ++h) {
+            tma_load_2d(kdst + h * L::kHalfBytes, &tm_k, full_bar(st), h * 64, y);
+            tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes, &tm_v, full_bar(st), h * 64, y);
+            if (y1 >= 0) {
+              tma_load_2d(kdst + h * L::kHalfBytes + 1024, &tm_k, full_bar(st), h * 64, y1);
+              tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes + 1024, &tm_v, full_bar(st),
+                          h * 64, y1);
+            }
+          }
         }
       }
       mbar_arrive(mempty_bar(ms));

@@ -2,8 +2,9 @@
 //
 // Same work units as the tensor-core kernel (pa_sched.cuh), processed by a
 // persistent grid of 4-warp CTAs.  Inside a unit, warp w takes the unit's
-// 16-token blocks w, w+4, ... ; each block is found through the request's
-// block-table row ("vLLM 深度拆解" §3.3) and read with plain vector loads.
+// 16-key tiles w, w+4, ... ; each tile's rows are found through the request's
+// block-table row ("vLLM 深度拆解" §3.3; one 16-row run of a 16- or 32-token
+// block, or two 8-token blocks) and read with plain vector loads.
 // Each warp keeps an online softmax (running max m, sum l, unnormalised o)
 // per tile row in the log2 domain; the epilogue merges the four warps.
 //
@@ -101,14 +102,18 @@ __global__ void __launch_bounds__(128, 1)
     const int* table = block_tables + static_cast<size_t>(u.row) * s.table_stride;
     for (int j = warp; j < nblk; j += NW) {
       const int blk_start = u.kv_begin + j * kBlock;
-      int pb = __ldg(table + blk_start / kBlock);
-      if (pb < 0 || pb >= s.num_blocks) {
-        if (lane == 0) report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, u.row, pb);
-        pb = 0;
-      }
-      const size_t tile = (static_cast<size_t>(pb) * s.num_kv_heads + u.kvh) * kBlock;
+      // cache rows of keys 0-7 and 8-15 of this tile (two 8-token blocks, or
+      // one run of 16 rows of a 16- or 32-token block)
+      const int y0 = key_row(table, blk_start, s.block_size, s.num_kv_heads, u.kvh,
+                             s.num_blocks, u.row);
+      const int y1 = s.block_size >= kBlock ? y0 + 8
+                     : blk_start + 8 < u.kv_end
+                         ? key_row(table, blk_start + 8, s.block_size, s.num_kv_heads, u.kvh,
+                                   s.num_blocks, u.row)
+                         : y0;
+      auto row_of = [&](int t) { return static_cast<size_t>(t < 8 ? y0 + t : y1 + t - 8); };
       float kr[HALF];
-      load_half_row<T, D>(k_cache + (tile + tok) * D + half * HALF, kr);
+      load_half_row<T, D>(k_cache + row_of(tok) * D + half * HALF, kr);
       const int kidx = blk_start + tok;
 #pragma unroll
       for (int r = 0; r < kRows; ++r) {
@@ -137,13 +142,13 @@ __global__ void __launch_bounds__(128, 1)
         }
       }
       const int nvalid = u.kv_end - blk_start;  // V rows at or past this are padding
-      const T* vt = v_cache + tile * D;
 #pragma unroll 4
       for (int t2 = 0; t2 < kBlock; ++t2) {
+        const T* vt = v_cache + row_of(t2) * D;
         float vv[PER];
 #pragma unroll
         for (int e = 0; e < PER; ++e)
-          vv[e] = t2 < nvalid ? to_f32<T>(vt[t2 * D + lane + 32 * e]) : 0.f;
+          vv[e] = t2 < nvalid ? to_f32<T>(vt[lane + 32 * e]) : 0.f;
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
           if (r < nrows) {

@@ -9,8 +9,9 @@
 // * work item = (chunk row, tile of 128/gs query tokens x gs query heads =
 //   128 tile rows, KV head slice); a persistent grid walks the items listed
 //   by the prep kernel, each CTA its items one after another;
-// * a load warp brings Q (one 3-D TMA box, two buffers) and K, V (eight
-//   16-token TMA boxes per 128-key tile, in K and V rings) into shared memory
+// * a load warp brings Q (one 3-D TMA box, two buffers) and K, V (one TMA box
+//   of 16 rows per 16 keys, two of 8 rows with 8-token blocks; K and V
+//   rings of 128-key tiles) into shared memory
 //   with 128-byte swizzling, which is exactly the canonical K-major layout
 //   (Q, K) and MN-major layout (V) the tcgen05 shared-memory descriptors
 //   describe.  It walks the CTA's tiles as one sequence, K one tile ahead of
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 8) {
     // ---------------------------------------------------------- TMA loads
     const int qt = kTcRows / s.gs;
+    const int box_rows = min(s.block_size, kBlock);  // rows of one K/V TMA box
     // Item metadata is fetched ahead: the chunk-list entry of item k + 2 and
     // the row data of item k + 1 are in flight while item k is issued.
     auto entry_of = [&](int k) -> int2 {
@@ -229,14 +231,16 @@ __global__ void __launch_bounds__(320, 1)
       bool r = true;
       if (lane == 0) {
         r = mbar_wait(vempty(vs), ((p.gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-        if (r) mbar_arrive_expect_tx(vfull(vs), static_cast<uint32_t>(p.nb * L::kHalves * 2048));
+        if (r)
+          mbar_arrive_expect_tx(vfull(vs),
+                                static_cast<uint32_t>(p.nb * L::kHalves * box_rows * 128));
       }
       r = __shfl_sync(0xffffffffu, r, 0);
       if (r && lane < p.nb) {
 #pragma unroll
         for (int h = 0; h < L::kHalves; ++h)
-          tma_load_2d(v_smem(vs) + h * L::kHalfBytes + lane * 2048, &tm_v, vfull(vs), h * 64,
-                      p.y);
+          tma_load_2d(v_smem(vs) + h * L::kHalfBytes + lane * box_rows * 128, &tm_v, vfull(vs),
+                      h * 64, p.y);
       }
       return r;
     };
@@ -253,30 +257,29 @@ __global__ void __launch_bounds__(320, 1)
     for (int k = 0; k < my_items && ok;) {
       for (int t = 0; t < it.nkt && ok; ++t) {
         const int gt = g + t, ks = gt % KS;
-        // one lane per 16-token block of the tile: its id, then its K boxes
-        const int first = t * (kTcKeys / kBlock);
-        const int nb = min(kTcKeys / kBlock, ceil_div(it.kv_end, kBlock) - first);
+        // one lane per TMA box of the tile (box = 16 rows, or 8 rows with
+        // 8-token blocks): its cache row, then its K boxes
+        const int key0 = t * kTcKeys;
+        const int nb = min(kTcKeys / box_rows, ceil_div(it.kv_end - key0, box_rows));
         int y = 0;
-        if (lane < nb) {
-          int pb = __ldg(block_tables + static_cast<size_t>(it.row) * s.table_stride + first + lane);
-          if (pb < 0 || pb >= s.num_blocks) {
-            report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, it.row, pb);
-            pb = 0;
-          }
-          y = (pb * s.num_kv_heads + it.kvh) * kBlock;
-        }
+        if (lane < nb)
+          y = key_row(block_tables + static_cast<size_t>(it.row) * s.table_stride,
+                      key0 + lane * box_rows, s.block_size, s.num_kv_heads, it.kvh, s.num_blocks,
+                      it.row);
         bool r = true;
         if (lane == 0) {
           r = mbar_wait(kempty(ks), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-          if (r) mbar_arrive_expect_tx(kfull(ks), static_cast<uint32_t>(nb * L::kHalves * 2048));
+          if (r)
+            mbar_arrive_expect_tx(kfull(ks),
+                                  static_cast<uint32_t>(nb * L::kHalves * box_rows * 128));
         }
         ok = __shfl_sync(0xffffffffu, r, 0);
         if (!ok) break;
         if (lane < nb) {
 #pragma unroll
           for (int h = 0; h < L::kHalves; ++h)
-            tma_load_2d(k_smem(ks) + h * L::kHalfBytes + lane * 2048, &tm_k, kfull(ks), h * 64,
-                        y);
+            tma_load_2d(k_smem(ks) + h * L::kHalfBytes + lane * box_rows * 128, &tm_k, kfull(ks),
+                        h * 64, y);
         }
         // queue this tile's V; issue the previous tile's
         if (npend == 0) {

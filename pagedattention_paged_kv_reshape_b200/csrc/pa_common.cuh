@@ -17,6 +17,9 @@
 namespace pa {
 
 // Tokens per physical block ("vLLM 架构源码解析" §1.1: 16 tokens by default).
+// Keys are processed in tiles of kBlock = 16 consecutive tokens whatever the
+// physical block size: a 32-token block holds two such tiles, an 8-token
+// block half of one (key_row below finds a key's row in the cache).
 constexpr int kBlock = 16;
 // Tokens per split-K partition.  Contexts longer than this are cut into
 // partitions whose partial softmax states are merged by log-sum-exp.
@@ -122,6 +125,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int whe
     }
   }
   return true;
+}
+
+// Row of key `key` of a request, in the cache viewed as rows of head_dim
+// elements: physical block table[key / block_size], KV head kvh, slot
+// key % block_size ("vLLM 深度拆解" §3.3: block_tables[seq * stride +
+// block_idx]).  An entry outside [0, num_blocks) is recorded and replaced by
+// block 0, so the access stays inside the pool.
+__device__ __forceinline__ int key_row(const int* __restrict__ table, int key, int block_size,
+                                       int num_kv_heads, int kvh, int num_blocks, int row) {
+  const int shift = __ffs(block_size) - 1;  // block sizes are powers of two
+  int pb = __ldg(table + (key >> shift));
+  if (pb < 0 || pb >= num_blocks) {
+    report_error(PA_ERR_DEVICE_BOUNDS, kWhereBlockId, row, pb);
+    pb = 0;
+  }
+  return (pb * num_kv_heads + kvh) * block_size + (key & (block_size - 1));
 }
 
 // ---------------------------------------------------------------------------

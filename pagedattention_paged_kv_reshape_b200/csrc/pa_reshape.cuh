@@ -2,8 +2,8 @@
 //
 // "vLLM 架构源码解析 | 第 1 篇" §3.3.3: the attention layer calls
 // reshape_and_cache(k, v, kv_cache, slot_mapping) before paged_attention;
-// §3.3.2 builds slot_mapping per token.  Slot s names physical block s / 16,
-// offset s % 16; a negative slot marks a padding token.
+// §3.3.2 builds slot_mapping per token.  Slot s names physical block
+// s / block_size, offset s % block_size; a negative slot marks a padding token.
 //
 // One warp per (token, KV head).  The K row and the V row of that pair are
 // head_dim * elem bytes each (256 B for bf16 x 128); lanes move them as
@@ -19,7 +19,8 @@ __global__ void __launch_bounds__(256)
     reshape_and_cache_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                              uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                              const int* __restrict__ slot_mapping, int num_tokens,
-                             int num_kv_heads, int row_vecs, long long num_slots) {
+                             int num_kv_heads, int row_vecs, int block_size,
+                             long long num_slots) {
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= static_cast<long long>(num_tokens) * num_kv_heads) return;
@@ -31,9 +32,9 @@ __global__ void __launch_bounds__(256)
     if (lane == 0) report_error(PA_ERR_DEVICE_BOUNDS, kWhereReshapeSlot, t, slot);
     return;
   }
-  const long long blk = slot / kBlock, off = slot % kBlock;
+  const long long blk = slot / block_size, off = slot % block_size;
   const long long src = (static_cast<long long>(t) * num_kv_heads + h) * row_vecs;
-  const long long dst = ((blk * num_kv_heads + h) * kBlock + off) * row_vecs;
+  const long long dst = ((blk * num_kv_heads + h) * block_size + off) * row_vecs;
   // lanes [0, row_vecs) copy K, the next row_vecs lanes copy V, and so on
   for (int c = lane; c < 2 * row_vecs; c += 32) {
     if (c < row_vecs)

@@ -40,6 +40,7 @@ struct Shape {
   int qpt;          // query tokens per tile (1 for pa_decode)
   int head_dim;
   int table_stride;
+  int block_size;   // tokens per physical block: 8, 16 or 32
   int num_blocks;
   int max_seq_len;  // host bound on seq_lens / context_lens
   int max_query_len;
@@ -88,7 +89,7 @@ __device__ __forceinline__ RowInfo load_row(const Shape& s, const int* __restric
     ri.q_len = ri.seq_len > 0 ? 1 : 0;  // an empty decode context: a zero output row
   }
   ri.ok = ri.seq_len >= 0 && ri.seq_len <= s.max_seq_len &&
-          ri.seq_len <= s.table_stride * kBlock && ri.q_len >= 0 &&
+          ri.seq_len <= s.table_stride * s.block_size && ri.q_len >= 0 &&
           ri.q_len <= ri.seq_len && ri.token0 >= 0 && ri.token0 + ri.q_len <= s.total_q &&
           (qsl == nullptr || ri.q_len <= s.max_query_len);
   return ri;

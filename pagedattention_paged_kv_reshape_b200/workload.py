@@ -292,6 +292,12 @@ CONFIGS = {
                        about="2048-token budget: 512-query causal chunk on 1536 cached tokens + "
                              "1536 decode rows (ctx U[64,4096], half share a 512-token prefix), "
                              "32/8 heads, head_dim 128, bf16"),
+    "gqa_bs256_b8": dict(requests=gqa_requests, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                         dtype="bf16", pool_factor=1.25, kind="decode", block_size=8,
+                         about="gqa_bs256 with 8-token blocks (\"vLLM 架构源码解析\" §5.1)"),
+    "gqa_bs256_b32": dict(requests=gqa_requests, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                          dtype="bf16", pool_factor=1.25, kind="decode", block_size=32,
+                          about="gqa_bs256 with 32-token blocks (\"vLLM 架构源码解析\" §5.1)"),
     "prefill_16x512": dict(requests=prefill_requests, num_q_heads=32, num_kv_heads=8,
                            head_dim=128, dtype="bf16", pool_factor=1.0, kind="varlen",
                            about="16 causal prefill chunks of 512 tokens on 1536 cached tokens, "

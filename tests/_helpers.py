@@ -79,15 +79,16 @@ def gpu_step(b: PagedBatch, varlen: bool | None = None):
 def oracle_step(b: PagedBatch, varlen: bool | None = None, seqs=None):
     """Oracle cache write then attention, on host copies of the batch."""
     varlen = (not b.is_decode) if varlen is None else varlen
+    bs = b.block_size
     kc, vc = O.reshape_and_cache(host(b.k_cache), host(b.v_cache), host(b.k_new),
-                                 host(b.v_new), b.host_slots)
+                                 host(b.v_new), b.host_slots, block_size=bs)
     q = host(b.q)
     if varlen:
         out = O.paged_varlen(q, kc, vc, b.host_tables, b.host_qsl, b.host_seq_lens, b.scale,
-                             b.dtype, seqs=seqs)
+                             b.dtype, block_size=bs, seqs=seqs)
     else:
         out = O.paged_decode(q, kc, vc, b.host_tables, b.host_seq_lens, b.scale, b.dtype,
-                             seqs=seqs)
+                             block_size=bs, seqs=seqs)
     return out, kc, vc
 
 
@@ -123,11 +124,15 @@ def oracle_rows(b: PagedBatch, rows, varlen: bool | None = None):
     """Oracle output (float64) for the query tokens of requests ``rows``."""
     varlen = (not b.is_decode) if varlen is None else varlen
     c = compact(b, rows)
-    kc, vc = O.reshape_and_cache(c["kc"], c["vc"], c["k_new"], c["v_new"], c["slots"])
+    bs = b.block_size
+    kc, vc = O.reshape_and_cache(c["kc"], c["vc"], c["k_new"], c["v_new"], c["slots"],
+                                 block_size=bs)
     if varlen:
-        out = O.paged_varlen(c["q"], kc, vc, c["tables"], c["qsl"], c["lens"], b.scale, b.dtype)
+        out = O.paged_varlen(c["q"], kc, vc, c["tables"], c["qsl"], c["lens"], b.scale, b.dtype,
+                             block_size=bs)
     else:
-        out = O.paged_decode(c["q"], kc, vc, c["tables"], c["lens"], b.scale, b.dtype)
+        out = O.paged_decode(c["q"], kc, vc, c["tables"], c["lens"], b.scale, b.dtype,
+                             block_size=bs)
     return c["tokens"], out
 
 

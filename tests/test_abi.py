@@ -122,7 +122,8 @@ def _decode(lib, **kw):
     (dict(hq=6, hkv=4), pa.Status.INVALID_ARG),        # Hq % Hkv != 0
     (dict(hkv=0), pa.Status.INVALID_ARG),
     (dict(d=96), pa.Status.UNSUPPORTED),
-    (dict(bs=32), pa.Status.UNSUPPORTED),
+    (dict(bs=24), pa.Status.UNSUPPORTED),
+    (dict(bs=64), pa.Status.UNSUPPORTED),
     (dict(dt=7), pa.Status.INVALID_ARG),
     (dict(S=-1), pa.Status.INVALID_ARG),
     (dict(scale=float("nan")), pa.Status.INVALID_ARG),
@@ -150,7 +151,8 @@ def test_empty_batches_launch_nothing(lib):
     ((None, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 16, 10, 1), pa.Status.INVALID_ARG),
     ((FAKE, FAKE, FAKE, FAKE, None, 4, 8, 128, 16, 10, 1), pa.Status.INVALID_ARG),
     ((FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 80, 16, 10, 1), pa.Status.UNSUPPORTED),
-    ((FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 8, 10, 1), pa.Status.UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 12, 10, 1), pa.Status.UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 64, 10, 1), pa.Status.UNSUPPORTED),
     ((FAKE, FAKE, FAKE, FAKE, FAKE, -1, 8, 128, 16, 10, 1), pa.Status.INVALID_ARG),
     ((FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 128, 16, 10, 9), pa.Status.INVALID_ARG),
 ])

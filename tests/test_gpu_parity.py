@@ -39,11 +39,12 @@ def decode_batch(lengths, hq, hkv, d, dtype, seed=0, **kw):
 # reshape_and_cache: bit-exact against the oracle's copy
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128), ("f16", 64), ("bf16", 64)])
-def test_reshape_and_cache_bit_exact(dtype, d):
+@pytest.mark.parametrize("dtype,d,bs", [("f32", 64, 16), ("bf16", 128, 16), ("f16", 64, 16),
+                                        ("bf16", 64, 16), ("bf16", 128, 8), ("f32", 64, 32)])
+def test_reshape_and_cache_bit_exact(dtype, d, bs):
     b = W.build_batch([W.Request(L, q) for L, q in [(1, 1), (40, 7), (300, 300), (17, 1)]],
                       num_q_heads=4, num_kv_heads=4, head_dim=d, dtype=dtype, seed=3, device=DEV,
-                      pool_factor=1.3)
+                      pool_factor=1.3, block_size=bs)
     slots = b.slot_mapping.clone()
     slots[::5] = -1                      # padding tokens are skipped
     hslots = b.host_slots.copy()
@@ -52,7 +53,7 @@ def test_reshape_and_cache_bit_exact(dtype, d):
     pa.pa_reshape_and_cache(b.k_new, b.v_new, kc, vc, slots)
     pa.pa_get_device_error()
     ok, ov = O.reshape_and_cache(host(b.k_cache), host(b.v_cache), host(b.k_new), host(b.v_new),
-                                 hslots)
+                                 hslots, block_size=bs)
     # byte-for-byte, NaN payloads included
     assert np.array_equal(host(kc).view(np.uint8), ok.view(np.uint8))
     assert np.array_equal(host(vc).view(np.uint8), ov.view(np.uint8))
@@ -187,6 +188,44 @@ def test_varlen_other_scales(scale):
     out, _, _ = gpu_step(b, varlen=True)
     ref, _, _ = oracle_step(b, varlen=True)
     assert_close(out, ref, "f16", f"varlen scale {scale}")
+
+
+BLOCK_SIZE_CASES = [
+    # (rows (seq_len, q_len), hq, hkv, d, dtype, block_size): 8- and 32-token
+    # blocks through decode rows, split-K rows and tcgen05 chunk rows
+    ([(700, 37), (1, 1), (33, 1), (2000, 1), (1300, 300), (9, 9)], 32, 8, 128, "bf16", 8),
+    ([(700, 37), (1, 1), (33, 1), (2000, 1), (1300, 300), (9, 9)], 32, 8, 128, "bf16", 32),
+    ([(600, 600), (90, 5), (1100, 1)], 8, 8, 64, "f16", 8),
+    ([(520, 20), (17, 17), (2, 1)], 4, 4, 64, "f32", 32),
+    ([(2500, 256), (300, 1), (15, 1)], 16, 2, 64, "f16", 32),
+]
+
+
+@pytest.mark.parametrize("path", ["auto", "mma", "simt"])
+@pytest.mark.parametrize("case", range(len(BLOCK_SIZE_CASES)))
+def test_block_sizes_match_oracle(case, path):
+    rows, hq, hkv, d, dtype, bs = BLOCK_SIZE_CASES[case]
+    if path == "simt":
+        pa.pa_set_path(pa.Path.SIMT)
+    elif path == "mma":
+        if dtype == "f32":
+            pytest.skip("tensor-core paths need 16-bit inputs")
+        pa.pa_set_path(pa.Path.MMA)
+    b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
+                      head_dim=d, dtype=dtype, seed=300 + case, device=DEV, pool_factor=1.2,
+                      block_size=bs)
+    out, kc, vc = gpu_step(b, varlen=True)
+    ref, okc, ovc = oracle_step(b, varlen=True)
+    assert np.array_equal(host(kc).view(np.uint8), okc.view(np.uint8))
+    assert_close(out, ref, dtype, f"block_size {bs} case {case} ({path})")
+    dec = [r for r, (s_, q_) in enumerate(rows) if q_ == 1]
+    if dec:  # the decode entry point on the same cache, for rows of one new token
+        bd = W.build_batch([W.Request(rows[r][0]) for r in dec], num_q_heads=hq,
+                           num_kv_heads=hkv, head_dim=d, dtype=dtype, seed=400 + case,
+                           device=DEV, pool_factor=1.2, block_size=bs)
+        out_d, _, _ = gpu_step(bd, varlen=False)
+        ref_d, _, _ = oracle_step(bd, varlen=False)
+        assert_close(out_d, ref_d, dtype, f"decode block_size {bs} case {case} ({path})")
 
 
 def test_chunk_kernel_agrees_with_decode_kernel_tiles():
