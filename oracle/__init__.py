@@ -36,3 +36,7 @@ from .paged_attention import (  # noqa: F401
     default_scale,
 )
 from .block_ops import copy_blocks, swap_blocks  # noqa: F401,E402
+from .fp8 import (  # noqa: F401,E402
+    E4M3_MAX, e4m3_decode, e4m3_encode, dequantize, reshape_and_cache_fp8, paged_decode_fp8,
+    paged_varlen_fp8,
+)

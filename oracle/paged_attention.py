@@ -41,6 +41,8 @@ def to_f64(a: np.ndarray, dtype: str) -> np.ndarray:
         return np.asarray(a, dtype=np.float16).astype(np.float64)
     if dtype == "f32":
         return np.asarray(a, dtype=np.float32).astype(np.float64)
+    if dtype == "f64":  # values already decoded (e.g. a dequantized FP8 cache)
+        return np.asarray(a, dtype=np.float64)
     raise ValueError(f"unknown dtype {dtype!r}")
 
 
