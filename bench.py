@@ -245,20 +245,38 @@ def cpu_baseline(batch, seconds: float) -> dict:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def make_step(pa, b, out, ws):
-    varlen = not b.is_decode
+def cache_write(pa, b, k_new, v_new, slots):
+    """pa_reshape_and_cache (or its quantising FP8 form) into ``b``'s pool."""
+    if b.fp8:
+        pa.pa_reshape_and_cache_fp8(k_new, v_new, b.k_cache, b.v_cache, slots, b.k_scale,
+                                    b.v_scale)
+    else:
+        pa.pa_reshape_and_cache(k_new, v_new, b.k_cache, b.v_cache, slots)
 
+
+def attention(pa, b, out, q, tables, lens, qsl, ws):
+    """pa_decode / pa_varlen (or the FP8 forms) over ``b``'s pool."""
+    if not b.is_decode:
+        if b.fp8:
+            pa.pa_varlen_fp8(out, q, b.k_cache, b.v_cache, b.k_scale, b.v_scale, tables, qsl,
+                             lens, b.max_query_len, b.max_seq_len, b.scale, ws)
+        else:
+            pa.pa_varlen(out, q, b.k_cache, b.v_cache, tables, qsl, lens, b.max_query_len,
+                         b.max_seq_len, b.scale, ws)
+    elif b.fp8:
+        pa.pa_decode_fp8(out, q, b.k_cache, b.v_cache, b.k_scale, b.v_scale, tables, lens,
+                         b.max_seq_len, b.scale, ws)
+    else:
+        pa.pa_decode(out, q, b.k_cache, b.v_cache, tables, lens, b.max_seq_len, b.scale, ws)
+
+
+def make_step(pa, b, out, ws):
     def step():
-        pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, b.slot_mapping)
+        cache_write(pa, b, b.k_new, b.v_new, b.slot_mapping)
         attend()
 
     def attend():
-        if varlen:
-            pa.pa_varlen(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.query_start_loc,
-                         b.seq_lens, b.max_query_len, b.max_seq_len, b.scale, ws)
-        else:
-            pa.pa_decode(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens,
-                         b.max_seq_len, b.scale, ws)
+        attention(pa, b, out, b.q, b.block_tables, b.seq_lens, b.query_start_loc, ws)
 
     return step, attend
 
@@ -292,7 +310,7 @@ def time_steps(torch, pa, b, steps, warmup):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(steps):
-        pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, b.slot_mapping)
+        cache_write(pa, b, b.k_new, b.v_new, b.slot_mapping)
         ev[i][0].record(stream)
         attend()
         ev[i][1].record(stream)
@@ -312,20 +330,13 @@ def time_e2e(torch, pa, b, steps):
     out = torch.empty_like(b.q)
     out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     ws = workspace_for(pa, b)
-    varlen = not b.is_decode
 
     def step():
         for n in names:
             dev[n].copy_(host[n], non_blocking=True)
-        pa.pa_reshape_and_cache(dev["k_new"], dev["v_new"], b.k_cache, b.v_cache,
-                                dev["slot_mapping"])
-        if varlen:
-            pa.pa_varlen(out, dev["q"], b.k_cache, b.v_cache, dev["block_tables"],
-                         dev["query_start_loc"], dev["seq_lens"], b.max_query_len,
-                         b.max_seq_len, b.scale, ws)
-        else:
-            pa.pa_decode(out, dev["q"], b.k_cache, b.v_cache, dev["block_tables"],
-                         dev["seq_lens"], b.max_seq_len, b.scale, ws)
+        cache_write(pa, b, dev["k_new"], dev["v_new"], dev["slot_mapping"])
+        attention(pa, b, out, dev["q"], dev["block_tables"], dev["seq_lens"],
+                  dev["query_start_loc"], ws)
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(5):
@@ -497,7 +508,7 @@ def run_ours(args):
         tensor_peak = measured_tensor_peak()
         per = {}
         for name in ("gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512", "gqa_bs256_b8",
-                     "gqa_bs256_b32"):
+                     "gqa_bs256_b32", "gqa_bs256_fp8"):
             if name == args.workload:
                 continue
             del b

@@ -86,7 +86,12 @@ typedef enum {
   PA_ERR_TIMEOUT = 6        /* (device) a bounded wait inside a kernel gave up */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
+typedef enum {
+  PA_F32 = 0,
+  PA_BF16 = 1,
+  PA_F16 = 2,
+  PA_E4M3 = 3  /* FP8 cache codes: only the element type of a pool in the block copies */
+} pa_dtype;
 
 /*
  * Kernel family selection, for tests and measurements.  PA_PATH_AUTO picks
@@ -125,6 +130,53 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
                                const int32_t* slot_mapping, int num_tokens, int num_kv_heads,
                                int head_dim, int block_size, int num_blocks, pa_dtype dtype,
                                void* stream);
+
+/*
+ * FP8 KV cache ("vLLM 深度拆解" §10.1: native FP8 with calibrated scales is
+ * the engine's next step).  The reading implemented: k_cache and v_cache hold
+ * FP8 e4m3 codes (one byte per element, the OCP E4M3 "fn" format: bias 7, no
+ * infinity, largest finite 448) in the layout above, and each KV head h has an
+ * fp32 scale for K, k_scale[h], and for V, v_scale[h] (device arrays
+ * [num_kv_heads], chosen by the caller's calibration).  A cached element
+ * stands for decode(code) * scale.  Halving the KV bytes halves what decode
+ * attention streams.
+ *
+ * pa_reshape_and_cache_fp8 -- the quantising write: element x (of `dtype`) of
+ * KV head h becomes the e4m3 code of float(x) / scale[h], the quotient
+ * correctly rounded in fp32, then rounded to nearest even and saturated to
+ * +-448.  Slots and errors as for pa_reshape_and_cache.
+ */
+pa_status pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                                   const int32_t* slot_mapping, const float* k_scale,
+                                   const float* v_scale, int num_tokens, int num_kv_heads,
+                                   int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                                   void* stream);
+
+/*
+ * pa_decode_fp8 / pa_varlen_fp8 -- pa_decode / pa_varlen over an FP8 cache:
+ * the same arguments plus k_scale and v_scale; q and out have `dtype`
+ * (PA_BF16, PA_F16 or PA_F32).  The result is attention over the dequantized
+ * cache.  On the tensor-core path the codes become f16 (every e4m3 value is
+ * exact in f16) and q is converted to f16 for the MMAs; the K scale folds into
+ * the softmax scale and the V scale into the output.  Workspace sizes are
+ * those of pa_decode_workspace_size / pa_varlen_workspace_size.
+ */
+pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale,
+                        const int32_t* block_tables, int block_table_stride,
+                        const int32_t* context_lens, int num_seqs, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        int max_context_len, float scale, void* workspace,
+                        size_t workspace_bytes, pa_dtype dtype, void* stream);
+
+pa_status pa_varlen_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale,
+                        const int32_t* block_tables, int block_table_stride,
+                        const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
+                        int total_q, int max_query_len, int max_seq_len, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        float scale, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                        void* stream);
 
 /*
  * pa_copy_blocks -- copy-on-write block copies inside one pool.

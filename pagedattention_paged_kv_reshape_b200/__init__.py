@@ -9,7 +9,10 @@ kernels, and this thin Python binding of it:
   softmax, split-K with a log-sum-exp reduce);
 * :func:`pa_varlen` -- mixed batches of decode rows and causal prefill chunks;
 * :func:`pa_copy_blocks` / :func:`pa_swap_blocks` -- copy-on-write copies
-  inside a pool, swap-out / swap-in between the device and a host pool.
+  inside a pool, swap-out / swap-in between the device and a host pool;
+* :func:`pa_reshape_and_cache_fp8`, :func:`pa_decode_fp8`,
+  :func:`pa_varlen_fp8` -- the same path over an FP8 (e4m3) cache with
+  per-KV-head scales.
 
 PyTorch provides device memory and streams only.  The seeded workload
 generator lives in :mod:`.workload`; byte/flop accounting in :mod:`.accounting`.
@@ -25,14 +28,17 @@ from ._binding import (  # noqa: F401
     STATIC_WORKSPACE_BYTES,
     pa_copy_blocks,
     pa_decode,
+    pa_decode_fp8,
     pa_decode_static,
     pa_decode_workspace_size,
     pa_get_device_error,
     pa_reshape_and_cache,
+    pa_reshape_and_cache_fp8,
     pa_set_path,
     pa_status_string,
     pa_swap_blocks,
     pa_varlen,
+    pa_varlen_fp8,
     pa_varlen_workspace_size,
     pa_version,
 )

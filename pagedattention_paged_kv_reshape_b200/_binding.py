@@ -40,11 +40,21 @@ class Path(enum.IntEnum):
 
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+E4M3 = 3  # FP8 cache codes (torch.uint8 or torch.float8_e4m3fn pools)
+FP8_CACHE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
 
 # name -> (restype, argtypes); mirrors include/pa.h
 _SIGNATURES = {
     "pa_reshape_and_cache": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                                       _c_int, _c_int, _vp]),
+    "pa_reshape_and_cache_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int,
+                                          _c_int, _c_int, _c_int, _c_int, _vp]),
+    "pa_decode_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
+                               _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _vp, _c_size,
+                               _c_int, _vp]),
+    "pa_varlen_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int,
+                               _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                               _c_float, _vp, _c_size, _c_int, _vp]),
     "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _vp]),
     "pa_swap_blocks": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -142,6 +152,10 @@ def pa_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None) -> N
         _stream(stream)))
 
 
+def _pool_code(t) -> int:
+    return E4M3 if t.dtype in FP8_CACHE_DTYPES else _dtype_code(t)
+
+
 def _pool_pair(k_pool, v_pool, what: str):
     _require(k_pool.shape == v_pool.shape and k_pool.dim() == 4, f"{what} pools must be 4-D")
     _require(k_pool.dtype == v_pool.dtype, f"{what} dtypes must match")
@@ -163,7 +177,7 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
     n = _block_mapping(block_mapping)
     nb, hkv, bs, d = k_cache.shape
     _check(lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), n, hkv, d, bs,
-                                nb, _dtype_code(k_cache), _stream(stream)))
+                                nb, _pool_code(k_cache), _stream(stream)))
 
 
 def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, stream=None) -> None:
@@ -181,7 +195,7 @@ def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, stream=None) -> No
     _, hkv, bs, d = src_k.shape
     _check(lib().pa_swap_blocks(_ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v),
                                 _ptr(block_mapping), n, hkv, d, bs, src_k.shape[0],
-                                dst_k.shape[0], _dtype_code(src_k), _stream(stream)))
+                                dst_k.shape[0], _pool_code(src_k), _stream(stream)))
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
@@ -256,6 +270,71 @@ def pa_varlen(out, q, k_cache, v_cache, block_tables, query_start_loc, seq_lens,
     _check(lib().pa_varlen(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         block_tables.shape[1], _ptr(query_start_loc), _ptr(seq_lens), seq_lens.numel(), total_q,
+        int(max_query_len), int(max_seq_len), hq, k_cache.shape[1], d, k_cache.shape[2],
+        k_cache.shape[0], float(scale), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream)))
+    return out
+
+
+def _fp8_pools(k_cache, v_cache, k_scale, v_scale):
+    _require(k_cache.dtype in FP8_CACHE_DTYPES and v_cache.dtype == k_cache.dtype,
+             "FP8 caches must be uint8 or float8_e4m3fn")
+    _require(k_scale.dtype == torch.float32 and v_scale.dtype == torch.float32
+             and k_scale.numel() == k_cache.shape[1] == v_scale.numel(),
+             "k_scale / v_scale must be float32 [num_kv_heads]")
+    _dense(k_cache, v_cache, k_scale, v_scale)
+
+
+def pa_reshape_and_cache_fp8(k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                             stream=None) -> None:
+    """Quantising write of ``k``, ``v`` ``[T, Hkv, D]`` into the FP8 (e4m3) caches
+    at ``slot_mapping``: code = e4m3(float(x) / scale[head])."""
+    _dense(k, v, slot_mapping)
+    _fp8_pools(k_cache, v_cache, k_scale, v_scale)
+    _require(k.shape == v.shape and k.dim() == 3, "k, v must be [T, Hkv, D]")
+    _require(k_cache.shape[1] == k.shape[1] and k_cache.shape[3] == k.shape[2],
+             "cache heads/head_dim must match k")
+    _require(slot_mapping.dtype == torch.int32 and slot_mapping.numel() == k.shape[0],
+             "slot_mapping must be int32 [T]")
+    _check(lib().pa_reshape_and_cache_fp8(
+        _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), _ptr(k_scale),
+        _ptr(v_scale), k.shape[0], k.shape[1], k.shape[2], k_cache.shape[2], k_cache.shape[0],
+        _dtype_code(k), _stream(stream)))
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                  max_context_len: int, scale: float, workspace: torch.Tensor,
+                  stream=None) -> torch.Tensor:
+    """Decode attention over an FP8 cache (workspace: ``pa_decode_workspace_size``)."""
+    _dense(out, q, block_tables, context_lens, workspace)
+    _fp8_pools(k_cache, v_cache, k_scale, v_scale)
+    _require(q.shape == out.shape and q.dim() == 3 and q.dtype == out.dtype, "q/out shape")
+    _require(block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32,
+             "metadata must be int32")
+    S, hq, d = q.shape
+    _check(lib().pa_decode_fp8(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, hq, k_cache.shape[1],
+        d, k_cache.shape[2], k_cache.shape[0], int(max_context_len), float(scale),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _dtype_code(q),
+        _stream(stream)))
+    return out
+
+
+def pa_varlen_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, query_start_loc,
+                  seq_lens, max_query_len: int, max_seq_len: int, scale: float,
+                  workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """Mixed batch over an FP8 cache (workspace: ``pa_varlen_workspace_size``)."""
+    _dense(out, q, block_tables, query_start_loc, seq_lens, workspace)
+    _fp8_pools(k_cache, v_cache, k_scale, v_scale)
+    _require(q.shape == out.shape and q.dim() == 3 and q.dtype == out.dtype, "q/out shape")
+    _require(block_tables.dtype == torch.int32 and query_start_loc.dtype == torch.int32
+             and seq_lens.dtype == torch.int32, "metadata must be int32")
+    T, hq, d = q.shape
+    S = seq_lens.numel()
+    _check(lib().pa_varlen_fp8(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_tables), block_tables.shape[1], _ptr(query_start_loc), _ptr(seq_lens), S, T,
         int(max_query_len), int(max_seq_len), hq, k_cache.shape[1], d, k_cache.shape[2],
         k_cache.shape[0], float(scale), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream)))

@@ -40,10 +40,16 @@ def _logical_blocks(length: int, block_size: int) -> int:
     return -(-length // block_size)
 
 
+def kv_elem_bytes(b: PagedBatch) -> int:
+    """Bytes of one cached K or V element: 1 for an FP8 (e4m3) cache."""
+    return 1 if b.fp8 else ELEMENT_BYTES[b.dtype]
+
+
 def attention_bytes(b: PagedBatch) -> dict:
-    """Algorithmic bytes of one attention call over batch ``b``."""
+    """Algorithmic bytes of one attention call over batch ``b`` (an FP8 cache
+    adds its 2 x Hkv fp32 scales)."""
     elem = ELEMENT_BYTES[b.dtype]
-    per_tok = kv_bytes_per_token(b.num_kv_heads, b.head_dim, elem)
+    per_tok = kv_bytes_per_token(b.num_kv_heads, b.head_dim, kv_elem_bytes(b))
     lens = [int(x) for x in b.host_seq_lens]
     logical_kv = sum(lens) * per_tok
     sharers = sum(1 for r in b.requests if r.shares_prefix)
@@ -51,17 +57,19 @@ def attention_bytes(b: PagedBatch) -> dict:
     unique_kv = logical_kv - max(0, sharers - 1) * shared_tokens * per_tok
     qo = 2 * b.total_q * b.num_q_heads * b.head_dim * elem
     tables = 4 * sum(_logical_blocks(L, b.block_size) for L in lens)
-    meta = 4 * (2 * b.num_seqs + 1)
+    meta = 4 * (2 * b.num_seqs + 1) + (8 * b.num_kv_heads if b.fp8 else 0)
     return {"kv_logical": logical_kv, "kv_unique": unique_kv, "q_out": qo, "tables": tables,
             "meta": meta, "total": unique_kv + qo + tables + meta,
             "total_logical": logical_kv + qo + tables + meta}
 
 
 def reshape_bytes(b: PagedBatch) -> int:
-    """Algorithmic bytes of one reshape_and_cache call (read + write of the new rows)."""
+    """Algorithmic bytes of one reshape_and_cache call (read of the new rows,
+    write of their cached form) plus the slot mapping."""
     elem = ELEMENT_BYTES[b.dtype]
-    rows = b.total_q * kv_bytes_per_token(b.num_kv_heads, b.head_dim, elem)
-    return 2 * rows + 4 * b.total_q
+    read = b.total_q * kv_bytes_per_token(b.num_kv_heads, b.head_dim, elem)
+    write = b.total_q * kv_bytes_per_token(b.num_kv_heads, b.head_dim, kv_elem_bytes(b))
+    return read + write + 4 * b.total_q
 
 
 def chunk_flops(b: PagedBatch) -> int:

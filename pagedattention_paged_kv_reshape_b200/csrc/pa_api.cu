@@ -45,7 +45,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-int elem_bytes(pa_dtype dt) { return dt == PA_F32 ? 4 : 2; }
+int elem_bytes(pa_dtype dt) { return dt == PA_F32 ? 4 : dt == PA_E4M3 ? 1 : 2; }
 
 bool valid_dtype(int dt) { return dt == PA_F32 || dt == PA_BF16 || dt == PA_F16; }
 
@@ -127,6 +127,26 @@ pa_status make_map_2d(CUtensorMap* map, const void* base, pa_dtype dt, uint64_t 
   return PA_OK;
 }
 
+// 2-D view [rows][inner] of a 1-byte tensor (FP8 codes), box {inner, box_rows};
+// 128-byte rows are 128 B-swizzled (the consumers read them with swizzled
+// 16-byte loads), 64-byte rows are not.
+pa_status make_map_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                         uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(inner), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed: %d", r);
+  return PA_OK;
+}
+
 // 3-D view [d2][d1][inner] of a 16-bit tensor, box {64, b1, b2}, 128 B swizzle.
 pa_status make_map_3d(CUtensorMap* map, const void* base, pa_dtype dt, uint64_t inner,
                       uint64_t d1, uint64_t d2, uint32_t b1, uint32_t b2) {
@@ -164,6 +184,10 @@ struct AttnArgs {
   size_t workspace_bytes;
   pa_dtype dtype;
   cudaStream_t stream;
+  // FP8 (e4m3) cache: per-KV-head scales of K and V; null for a 16/32-bit cache
+  const float* k_scale = nullptr;
+  const float* v_scale = nullptr;
+  bool kv8() const { return k_scale != nullptr; }
 };
 
 #ifndef PA_STAGES
@@ -297,9 +321,10 @@ pa_status check_common(const AttnArgs& a) {
   return PA_OK;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool KV8>
 pa_status launch_simt(const AttnArgs& a, const Plan& p, const pa::Work& w) {
-  auto kern = pa::attn_simt_kernel<T, D>;
+  using C = typename std::conditional<KV8, uint8_t, T>::type;  // cache element
+  auto kern = pa::attn_simt_kernel<T, D, KV8>;
   int occ = 0;
   cudaError_t e = prepare(kern, 128, 0, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "simt kernel set-up");
@@ -308,16 +333,20 @@ pa_status launch_simt(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   if (grid < 1) grid = 1;
   e = launch_pdl(kern, static_cast<unsigned>(grid), 128, 0, a.stream, p.s,
                  static_cast<T*>(a.out), static_cast<const T*>(a.q),
-                 static_cast<const T*>(a.k_cache), static_cast<const T*>(a.v_cache),
-                 a.block_tables, a.qsl, a.seq_lens, w, static_cast<float>(a.scale * M_LOG2E));
+                 static_cast<const C*>(a.k_cache), static_cast<const C*>(a.v_cache),
+                 a.block_tables, a.qsl, a.seq_lens, w, static_cast<float>(a.scale * M_LOG2E),
+                 a.k_scale, a.v_scale);
   if (e != cudaSuccess) return cuda_fail(e, "simt kernel launch");
   return PA_OK;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool KV8>
 pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
-  using L = pa::MmaLayout<D, kNcw, kStages>;
-  auto kern = pa::attn_mma_kernel<T, D, kNcw, kStages>;
+  // FP8 stages are half as large: at head_dim 128 twice as many keep the same
+  // bytes in flight; at 64 the per-warp f16 staging tiles take that room
+  constexpr int kS = KV8 && D == 128 ? 2 * kStages : kStages;
+  using L = pa::MmaLayout<D, kNcw, kS, KV8>;
+  auto kern = pa::attn_mma_kernel<T, D, kNcw, kS, KV8>;
   int occ = 0;
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "mma kernel set-up");
@@ -325,9 +354,11 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   // one box = 16 cache rows, or one whole 8-token block
   const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
   const int box_rows = a.block_size < pa::kBlock ? a.block_size : pa::kBlock;
-  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, box_rows);
+  pa_status st = KV8 ? make_map_2d_u8(&tk, a.k_cache, D, rows, box_rows)
+                     : make_map_2d(&tk, a.k_cache, a.dtype, D, rows, box_rows);
   if (st != PA_OK) return st;
-  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, box_rows);
+  st = KV8 ? make_map_2d_u8(&tv, a.v_cache, D, rows, box_rows)
+           : make_map_2d(&tv, a.v_cache, a.dtype, D, rows, box_rows);
   if (st != PA_OK) return st;
   st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.qpt);
   if (st != PA_OK) return st;
@@ -336,7 +367,7 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   if (grid < 1) grid = 1;
   e = launch_pdl(kern, static_cast<unsigned>(grid), L::kThreads, L::kSmem, a.stream, tk, tv, tq,
                  p.s, static_cast<T*>(a.out), a.block_tables, a.qsl, a.seq_lens, w,
-                 static_cast<float>(a.scale * M_LOG2E));
+                 static_cast<float>(a.scale * M_LOG2E), a.k_scale, a.v_scale);
   if (e != cudaSuccess) return cuda_fail(e, "mma kernel launch");
   return PA_OK;
 }
@@ -377,13 +408,21 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
   pa_status st;
+  const bool d128 = a.head_dim == 128;
   if constexpr (sizeof(T) == 2) {
     if (use_mma)
-      st = a.head_dim == 128 ? launch_mma<T, 128>(a, p, w) : launch_mma<T, 64>(a, p, w);
+      st = a.kv8() ? (d128 ? launch_mma<T, 128, true>(a, p, w) : launch_mma<T, 64, true>(a, p, w))
+                   : (d128 ? launch_mma<T, 128, false>(a, p, w)
+                           : launch_mma<T, 64, false>(a, p, w));
     else
-      st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, w) : launch_simt<T, 64>(a, p, w);
+      st = a.kv8() ? (d128 ? launch_simt<T, 128, true>(a, p, w)
+                           : launch_simt<T, 64, true>(a, p, w))
+                   : (d128 ? launch_simt<T, 128, false>(a, p, w)
+                           : launch_simt<T, 64, false>(a, p, w));
   } else {
-    st = a.head_dim == 128 ? launch_simt<T, 128>(a, p, w) : launch_simt<T, 64>(a, p, w);
+    st = a.kv8() ? (d128 ? launch_simt<T, 128, true>(a, p, w) : launch_simt<T, 64, true>(a, p, w))
+                 : (d128 ? launch_simt<T, 128, false>(a, p, w)
+                         : launch_simt<T, 64, false>(a, p, w));
   }
   if (st != PA_OK) return st;
   if constexpr (sizeof(T) == 2) {
@@ -438,6 +477,8 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
   if (varlen) {
     if (!a.qsl || !aligned(a.qsl, 4)) return fail(PA_ERR_INVALID_ARG, "bad query_start_loc");
   }
+  if (a.kv8() && (!a.v_scale || !aligned(a.k_scale, 4) || !aligned(a.v_scale, 4)))
+    return fail(PA_ERR_INVALID_ARG, "bad k_scale / v_scale pointer");
   const int path = g_path.load();
   const bool sixteen = a.dtype != PA_F32;
   if (path == PA_PATH_MMA || path == PA_PATH_TCGEN05) {
@@ -447,7 +488,7 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
   const bool use_mma = sixteen && path != PA_PATH_SIMT;
   // Prefill-chunk rows (q_len >= one 128-row tile) go to the tcgen05 kernel
   // unless a family without it was forced.
-  p.s.chunk_qt = (use_mma && path != PA_PATH_MMA && p.chunk_qt > 0 &&
+  p.s.chunk_qt = (use_mma && !a.kv8() && path != PA_PATH_MMA && p.chunk_qt > 0 &&
                   a.max_query_len >= p.chunk_qt)
                      ? p.chunk_qt
                      : 0;
@@ -520,6 +561,57 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
   return PA_OK;
 }
 
+pa_status pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                                   const int32_t* slot_mapping, const float* k_scale,
+                                   const float* v_scale, int num_tokens, int num_kv_heads,
+                                   int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                                   void* stream) {
+  if (!valid_dtype(dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks < 0)
+    return fail(PA_ERR_INVALID_ARG, "bad sizes");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
+  if (!supported_block_size(block_size))
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", block_size);
+  if (num_tokens == 0) return PA_OK;
+  const void* ptrs[] = {k, v, k_cache, v_cache};
+  for (const void* p : ptrs) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(p, 16)) return fail(PA_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  }
+  if (!slot_mapping || !aligned(slot_mapping, 4))
+    return fail(PA_ERR_INVALID_ARG, "bad slot_mapping pointer");
+  if (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4))
+    return fail(PA_ERR_INVALID_ARG, "bad k_scale / v_scale pointer");
+  const long long warps = static_cast<long long>(num_tokens) * num_kv_heads;
+  const long long blocks = (warps * 32 + 255) / 256;
+  if (blocks > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many tokens");
+  const auto st = static_cast<cudaStream_t>(stream);
+  const long long slots = static_cast<long long>(num_blocks) * block_size;
+  const unsigned g = static_cast<unsigned>(blocks);
+  auto* kc = static_cast<uint8_t*>(k_cache);
+  auto* vc = static_cast<uint8_t*>(v_cache);
+  switch (dtype) {
+    case PA_BF16:
+      pa::reshape_and_cache_fp8_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), kc, vc,
+          slot_mapping, k_scale, v_scale, num_tokens, num_kv_heads, head_dim, block_size, slots);
+      break;
+    case PA_F16:
+      pa::reshape_and_cache_fp8_kernel<__half><<<g, 256, 0, st>>>(
+          static_cast<const __half*>(k), static_cast<const __half*>(v), kc, vc, slot_mapping,
+          k_scale, v_scale, num_tokens, num_kv_heads, head_dim, block_size, slots);
+      break;
+    default:
+      pa::reshape_and_cache_fp8_kernel<float><<<g, 256, 0, st>>>(
+          static_cast<const float*>(k), static_cast<const float*>(v), kc, vc, slot_mapping,
+          k_scale, v_scale, num_tokens, num_kv_heads, head_dim, block_size, slots);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache_fp8 launch");
+  return PA_OK;
+}
+
 // Device-visible address of a pointer the kernels may dereference: device
 // memory as is, page-locked host memory through its mapped address.  Pageable
 // host memory is refused.
@@ -547,7 +639,8 @@ static pa_status launch_block_copy(const void* src_k, const void* src_v, void* d
                                    int head_dim, int block_size, int src_num_blocks,
                                    int dst_num_blocks, pa_dtype dtype, void* stream,
                                    bool allow_host) {
-  if (!valid_dtype(dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (!valid_dtype(dtype) && dtype != PA_E4M3)
+    return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || src_num_blocks < 0 ||
       dst_num_blocks < 0)
     return fail(PA_ERR_INVALID_ARG, "bad sizes");
@@ -667,6 +760,37 @@ pa_status pa_varlen(void* out, const void* q, const void* k_cache, const void* v
              seq_lens, num_seqs, total_q, max_query_len, max_seq_len, num_q_heads,
              num_kv_heads, head_dim, block_size, num_blocks, scale, workspace, workspace_bytes,
              dtype, static_cast<cudaStream_t>(stream)};
+  return run_attention(a, true);
+}
+
+pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale,
+                        const int32_t* block_tables, int block_table_stride,
+                        const int32_t* context_lens, int num_seqs, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        int max_context_len, float scale, void* workspace,
+                        size_t workspace_bytes, pa_dtype dtype, void* stream) {
+  if (!k_scale) return fail(PA_ERR_INVALID_ARG, "null k_scale");
+  AttnArgs a{out, q, k_cache, v_cache, block_tables, block_table_stride, nullptr, context_lens,
+             num_seqs, num_seqs, 1, max_context_len, num_q_heads, num_kv_heads, head_dim,
+             block_size, num_blocks, scale, workspace, workspace_bytes, dtype,
+             static_cast<cudaStream_t>(stream), k_scale, v_scale};
+  return run_attention(a, false);
+}
+
+pa_status pa_varlen_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale,
+                        const int32_t* block_tables, int block_table_stride,
+                        const int32_t* query_start_loc, const int32_t* seq_lens, int num_seqs,
+                        int total_q, int max_query_len, int max_seq_len, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        float scale, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                        void* stream) {
+  if (!k_scale) return fail(PA_ERR_INVALID_ARG, "null k_scale");
+  AttnArgs a{out, q, k_cache, v_cache, block_tables, block_table_stride, query_start_loc,
+             seq_lens, num_seqs, total_q, max_query_len, max_seq_len, num_q_heads,
+             num_kv_heads, head_dim, block_size, num_blocks, scale, workspace, workspace_bytes,
+             dtype, static_cast<cudaStream_t>(stream), k_scale, v_scale};
   return run_attention(a, true);
 }
 

@@ -39,12 +39,19 @@ struct MetaSlot {
   int y1[kPart / kBlock];
 };
 
-template <int D, int NCW, int STAGES>
+// KV8: the cache holds FP8 e4m3 codes and a stage holds the 1-byte K and V
+// tiles (16 rows x D bytes).  At head_dim 128 they are 128 B-swizzled and the
+// consumers build their MMA operands straight from them (see fp8_direct
+// below); at head_dim 64 they are unswizzled and each consumer warp first
+// converts its tile into a 16-bit staging tile laid out like a 16-bit stage.
+template <int D, int NCW, int STAGES, bool KV8 = false>
 struct MmaLayout {
+  static constexpr bool kStaging = KV8 && D != 128;
   static constexpr int kHalves = D / 64;             // 64 16-bit elements = one 128 B swizzle row
   static constexpr int kHalfBytes = kBlock * 128;    // 16 rows x 128 B
-  static constexpr int kTileBytes = kHalves * kHalfBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;  // K tile then V tile
+  static constexpr int kTileBytes = kHalves * kHalfBytes;          // a 16-bit K or V tile
+  static constexpr int kKVTileBytes = KV8 ? kBlock * D : kTileBytes;  // ... as loaded
+  static constexpr int kStageBytes = 2 * kKVTileBytes;  // K tile then V tile
   static constexpr int kQSlotBytes = kHalves * kRows * 128;
   static constexpr int kQSlots = 2;
   static constexpr int kOffQ = STAGES * kStageBytes;
@@ -58,10 +65,13 @@ struct MmaLayout {
   static constexpr int kOffDesc = kOffBar + kNumBars * 8;
   static constexpr int kOffMeta = kOffDesc + kQSlots * static_cast<int>(sizeof(Unit));
   static constexpr int kOffFlags = kOffMeta + kMetaSlots * static_cast<int>(sizeof(MetaSlot));
-  static constexpr int kBytes = kOffFlags + 16;
+  // KV8: per consumer warp a 16-bit K and V staging tile
+  static constexpr int kOffStg = (kOffFlags + 16 + 1023) / 1024 * 1024;
+  static constexpr int kBytes = kStaging ? kOffStg + NCW * 2 * kTileBytes : kOffFlags + 16;
   static constexpr int kSmem = kBytes + 1024;  // slack to align the base to 1024 B
   static constexpr int kThreads = (NCW + 2) * 32;
   static_assert(kOffQ % 1024 == 0 && kQSlotBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kSmem <= 116 * 1024, "two CTAs per SM");
 };
 
 // Byte offset, inside one 128 B-swizzled tile half, of the 16-byte chunk `ch`
@@ -71,14 +81,82 @@ __device__ __forceinline__ uint32_t swz(int r, int ch) {
   return static_cast<uint32_t>(r * 128 + ((ch ^ (r & 7)) << 4));
 }
 
-template <typename T, int D, int NCW, int STAGES>
+// Two e4m3 codes (low byte first) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two) {
+  const __half2_raw h =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ void lds128(uint32_t addr, uint32_t (&w)[4]) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// One FP8 tile (16 rows x D codes, row-major, as TMA lands it) -> the 16-bit
+// (f16) tile layout of a 128 B-swizzled stage.  Lane l converts 16-byte
+// groups l, l + 32, ...; every e4m3 value is exact in f16.
+template <int D>
+__device__ __forceinline__ void convert_fp8_tile(uint32_t src, uint32_t dst, int lane) {
+  constexpr int kGroups = D / 16;  // 16-code groups per row
+#pragma unroll
+  for (int c = lane; c < kBlock * kGroups; c += 32) {
+    const int r = c / kGroups, g = c % kGroups;
+    uint32_t w[4];
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "r"(src + c * 16));
+    uint32_t hv[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>(w[i] & 0xffffu), __NV_E4M3);
+      const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
+      hv[2 * i] = static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16);
+      hv[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
+    }
+    // codes 16g .. 16g+15 = dims of half g/4, 16-byte chunks 2(g%4) and 2(g%4)+1
+    const uint32_t base = dst + (g >> 2) * (kBlock * 128);
+    const int ch = (g & 3) * 2;
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + swz(r, ch)), "r"(hv[0]),
+                 "r"(hv[1]), "r"(hv[2]), "r"(hv[3])
+                 : "memory");
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + swz(r, ch + 1)),
+                 "r"(hv[4]), "r"(hv[5]), "r"(hv[6]), "r"(hv[7])
+                 : "memory");
+  }
+}
+
+template <typename T, int D, int NCW, int STAGES, bool KV8 = false>
 __global__ void __launch_bounds__((NCW + 2) * 32, 2)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, Shape s, T* __restrict__ out,
                     const int* __restrict__ block_tables, const int* __restrict__ qsl,
-                    const int* __restrict__ seq_lens, Work w, float scale_log2) {
-  using L = MmaLayout<D, NCW, STAGES>;
+                    const int* __restrict__ seq_lens, Work w, float scale_log2,
+                    const float* __restrict__ k_scale, const float* __restrict__ v_scale) {
+  using L = MmaLayout<D, NCW, STAGES, KV8>;
+  // operand type of the MMAs: the input type, or f16 for an FP8 cache (every
+  // e4m3 value is exact in f16; q and P are converted to it)
+  using MT = typename std::conditional<KV8, __half, T>::type;
+  // fp8_direct (FP8, head_dim 128): the contraction dims of QK^T are visited in
+  // a permuted order that gives each lane one contiguous 16-byte run of a key
+  // row per four k-steps -- lane quad q4 of k-step 4G + s takes dims
+  // 64G + 16 q4 + 4s + {0,1} (fragment k 2q4, 2q4+1) and + {2,3} (k 2q4+8,
+  // 2q4+9), for K and, loaded the same way, for Q.  The output dims of P.V
+  // are permuted too: n-tile j, column n is head dim 16 n + j, so lane group g
+  // reads the 16 bytes of dims 16g .. 16g+15 of each of its four keys.  The
+  // epilogue writes every accumulator to its own head dim.
+  constexpr bool fp8_direct = KV8 && !L::kStaging;
   constexpr int KSTEPS = D / 16;  // k-steps of QK^T, also n-tile pairs of PV
   constexpr int NT = D / 8;       // PV n-tiles of 8 dims
   extern __shared__ uint8_t smem_raw[];
@@ -215,24 +293,28 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
           break;
         ++issued;
         const uint32_t kdst = sbase + st * L::kStageBytes;
-        if (s.block_size >= kBlock) {  // one 16-row box per half
+        // boxes per K or V tile: one per 64-dim half (16-bit), or one of D
+        // bytes (FP8); 16 rows, or 8 rows twice with 8-token blocks
+        constexpr int kBoxes = KV8 ? 1 : L::kHalves;
+        constexpr int kBoxBytes = L::kKVTileBytes / kBoxes;
+        if (s.block_size >= kBlock) {
           mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
 #pragma unroll
-          for (int h = 0; h < L::kHalves; ++h) {
-            tma_load_2d(kdst + h * L::kHalfBytes, &tm_k, full_bar(st), h * 64, y);
-            tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes, &tm_v, full_bar(st), h * 64, y);
+          for (int h = 0; h < kBoxes; ++h) {
+            tma_load_2d(kdst + h * kBoxBytes, &tm_k, full_bar(st), h * 64, y);
+            tma_load_2d(kdst + L::kKVTileBytes + h * kBoxBytes, &tm_v, full_bar(st), h * 64, y);
           }
         } else {  // 8-token blocks: rows 0-7 and, if the tile has them, rows 8-15
           const int y1 = meta[ms].y1[jj];
           mbar_arrive_expect_tx(full_bar(st), y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
 #pragma unroll
-          for (int h = 0; h < L::kHalves; ++h) {
-            tma_load_2d(kdst + h * L::kHalfBytes, &tm_k, full_bar(st), h * 64, y);
-            tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes, &tm_v, full_bar(st), h * 64, y);
+          for (int h = 0; h < kBoxes; ++h) {
+            tma_load_2d(kdst + h * kBoxBytes, &tm_k, full_bar(st), h * 64, y);
+            tma_load_2d(kdst + L::kKVTileBytes + h * kBoxBytes, &tm_v, full_bar(st), h * 64, y);
             if (y1 >= 0) {
-              tma_load_2d(kdst + h * L::kHalfBytes + 1024, &tm_k, full_bar(st), h * 64, y1);
-              tma_load_2d(kdst + L::kTileBytes + h * L::kHalfBytes + 1024, &tm_v, full_bar(st),
-                          h * 64, y1);
+              tma_load_2d(kdst + h * kBoxBytes + kBoxBytes / 2, &tm_k, full_bar(st), h * 64, y1);
+              tma_load_2d(kdst + L::kKVTileBytes + h * kBoxBytes + kBoxBytes / 2, &tm_v,
+                          full_bar(st), h * 64, y1);
             }
           }
         }
@@ -274,7 +356,31 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
       break;
     }
     uint32_t qa[KSTEPS][4];
-    {
+    if constexpr (fp8_direct) {
+      const uint32_t qb = sbase + L::kOffQ + qs * L::kQSlotBytes;
+      const int g = lane >> 2, q4 = lane & 3;
+#pragma unroll
+      for (int G = 0; G < D / 64; ++G) {
+        uint32_t a0[4], a1[4], b0[4], b1[4];  // rows g, g+8; dims 16q4 .. +7, +8 .. +15
+        lds128(qb + G * (kRows * 128) + swz(g, 2 * q4), a0);
+        lds128(qb + G * (kRows * 128) + swz(g, 2 * q4 + 1), a1);
+        lds128(qb + G * (kRows * 128) + swz(g + 8, 2 * q4), b0);
+        lds128(qb + G * (kRows * 128) + swz(g + 8, 2 * q4 + 1), b1);
+#pragma unroll
+        for (int st2 = 0; st2 < 2; ++st2) {
+          const uint32_t* ra = st2 ? a1 : a0;
+          const uint32_t* rb = st2 ? b1 : b0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t* f = qa[4 * G + 2 * st2 + h];
+            f[0] = ra[2 * h];
+            f[1] = rb[2 * h];
+            f[2] = ra[2 * h + 1];
+            f[3] = rb[2 * h + 1];
+          }
+        }
+      }
+    } else {
       const uint32_t qb = sbase + L::kOffQ + qs * L::kQSlotBytes;
       const int mi = lane >> 3;
       const int r = (lane & 7) + ((mi & 1) << 3);
@@ -285,6 +391,15 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
                 qa[kk][3]);
       }
     }
+    if constexpr (KV8 && !std::is_same<T, __half>::value) {  // q to the f16 operand type
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack2<T>(qa[kk][e]);
+          qa[kk][e] = pack2<__half>(f.x, f.y);
+        }
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(qempty_bar(qs));
     ++k;
@@ -293,6 +408,8 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
     float o[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    // FP8: the K scale of this KV head folds into the softmax scale
+    const float sl = KV8 ? scale_log2 * __ldg(k_scale + u.kvh) : scale_log2;
     const int lim0 = u.lim0 + r0 / s.gs;
     const int lim1 = u.lim0 + r1 / s.gs;
     const int nblk = ceil_div(u.kv_end - u.kv_begin, kBlock);
@@ -301,15 +418,52 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
       const int nn = n + j;
       const int st = nn % STAGES;
       if (!mbar_wait(full_bar(st), (nn / STAGES) & 1, kWhereWaitFull, abort_flag)) return;
-      const uint32_t kb = sbase + st * L::kStageBytes;
-      const uint32_t vb = kb + L::kTileBytes;
+      uint32_t kb = sbase + st * L::kStageBytes;
+      uint32_t vb = kb + L::kKVTileBytes;
+      if constexpr (L::kStaging) {
+        // FP8 codes -> f16 staging tiles of this warp, then the stage is free
+        const uint32_t stg = sbase + L::kOffStg + warp * 2 * L::kTileBytes;
+        convert_fp8_tile<D>(kb, stg, lane);
+        convert_fp8_tile<D>(kb + L::kKVTileBytes, stg + L::kTileBytes, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(st));
+        kb = stg;
+        vb = stg + L::kTileBytes;
+      }
+      // FP8 direct: this lane's V bytes come into registers as soon as the
+      // stage lands (keys 2q4, 2q4+1, 2q4+8, 2q4+9; head dims 16g .. 16g+15).
+      // (Reading them late, after the softmax, gave sporadically wrong units,
+      // and so did releasing the stage right after Q K^T; the stage is
+      // released at the end of the tile, as on the 16-bit path.)
+      uint32_t va[4], vb1[4], vc[4], vd[4];
+      if constexpr (fp8_direct) {
+        const int g = lane >> 2, q4 = lane & 3;
+        lds128(vb + swz(2 * q4, g), va);
+        lds128(vb + swz(2 * q4 + 1, g), vb1);
+        lds128(vb + swz(2 * q4 + 8, g), vc);
+        lds128(vb + swz(2 * q4 + 9, g), vd);
+      }
       const int blk_start = u.kv_begin + j * kBlock;
 
       // ---- S = Q K^T over this block's 16 tokens
       float sacc[2][4];
 #pragma unroll
       for (int t = 0; t < 2; ++t) sacc[t][0] = sacc[t][1] = sacc[t][2] = sacc[t][3] = 0.f;
-      {
+      if constexpr (fp8_direct) {
+        const int g = lane >> 2, q4 = lane & 3;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+          for (int G = 0; G < D / 64; ++G) {
+            uint32_t w[4];  // key nt*8+g, dims 64G + 16 q4 .. +15
+            lds128(kb + swz(nt * 8 + g, 4 * G + q4), w);
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4)
+              mma_16816<MT>(sacc[nt], qa[4 * G + s4], fp8x2_to_f16x2(w[s4]),
+                            fp8x2_to_f16x2(w[s4] >> 16));
+          }
+        }
+      } else {
         const int mi = lane >> 3;
         const int tk = (lane & 7) + ((mi >> 1) << 3);
 #pragma unroll
@@ -317,15 +471,15 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
           uint32_t b0, b1, b2, b3;
           const int ch = (kk & 3) * 2 + (mi & 1);
           ldsm_x4(kb + (kk >> 2) * L::kHalfBytes + swz(tk, ch), b0, b1, b2, b3);
-          mma_16816<T>(sacc[0], qa[kk], b0, b1);
-          mma_16816<T>(sacc[1], qa[kk], b2, b3);
+          mma_16816<MT>(sacc[0], qa[kk], b0, b1);
+          mma_16816<MT>(sacc[1], qa[kk], b2, b3);
         }
       }
       float x[2][4];
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[t][e] = sacc[t][e] * scale_log2;
+        for (int e = 0; e < 4; ++e) x[t][e] = sacc[t][e] * sl;
       if (blk_start + kBlock > u.lim0) {  // some key of this block is past some row's limit
 #pragma unroll
         for (int t = 0; t < 2; ++t)
@@ -347,13 +501,13 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
       const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
       const float a0 = exp2f(m0 - mu0), a1 = exp2f(m1 - mu1);
       uint32_t pa[4];
-      pa[0] = pack2<T>(exp2f(x[0][0] - mu0), exp2f(x[0][1] - mu0));
-      pa[1] = pack2<T>(exp2f(x[0][2] - mu1), exp2f(x[0][3] - mu1));
-      pa[2] = pack2<T>(exp2f(x[1][0] - mu0), exp2f(x[1][1] - mu0));
-      pa[3] = pack2<T>(exp2f(x[1][2] - mu1), exp2f(x[1][3] - mu1));
+      pa[0] = pack2<MT>(exp2f(x[0][0] - mu0), exp2f(x[0][1] - mu0));
+      pa[1] = pack2<MT>(exp2f(x[0][2] - mu1), exp2f(x[0][3] - mu1));
+      pa[2] = pack2<MT>(exp2f(x[1][0] - mu0), exp2f(x[1][1] - mu0));
+      pa[3] = pack2<MT>(exp2f(x[1][2] - mu1), exp2f(x[1][3] - mu1));
       // the normaliser sums the same rounded weights the P.V product uses
-      const float2 p00 = unpack2<T>(pa[0]), p01 = unpack2<T>(pa[1]);
-      const float2 p10 = unpack2<T>(pa[2]), p11 = unpack2<T>(pa[3]);
+      const float2 p00 = unpack2<MT>(pa[0]), p01 = unpack2<MT>(pa[1]);
+      const float2 p10 = unpack2<MT>(pa[2]), p11 = unpack2<MT>(pa[3]);
       l0 = l0 * a0 + ((p00.x + p00.y) + (p10.x + p10.y));
       l1 = l1 * a1 + ((p01.x + p01.y) + (p11.x + p11.y));
       m0 = mn0;
@@ -373,7 +527,21 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
         vm0 = (t0 < nv ? 0x0000ffffu : 0u) | (t0 + 1 < nv ? 0xffff0000u : 0u);
         vm1 = (t0 + 8 < nv ? 0x0000ffffu : 0u) | (t0 + 9 < nv ? 0xffff0000u : 0u);
       }
-      {
+      if constexpr (fp8_direct) {  // V from the bytes loaded above
+#pragma unroll
+        for (int jw = 0; jw < 4; ++jw) {
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {  // bytes 2hb, 2hb+1 of word jw: n-tiles 4jw+2hb, +1
+            const uint32_t sel = hb ? 0x7362u : 0x5140u;
+            const uint32_t lo = prmt(va[jw], vb1[jw], sel);  // (key 2q4, 2q4+1) x two dims
+            const uint32_t hi = prmt(vc[jw], vd[jw], sel);   // (key 2q4+8, 2q4+9)
+            const int j = 4 * jw + 2 * hb;
+            mma_16816<MT>(o[j], pa, fp8x2_to_f16x2(lo) & vm0, fp8x2_to_f16x2(hi) & vm1);
+            mma_16816<MT>(o[j + 1], pa, fp8x2_to_f16x2(lo >> 16) & vm0,
+                          fp8x2_to_f16x2(hi >> 16) & vm1);
+          }
+        }
+      } else {
         const int mi = lane >> 3;
         const int tk = (lane & 7) + ((mi & 1) << 3);
 #pragma unroll
@@ -381,15 +549,22 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
           uint32_t b0, b1, b2, b3;
           const int ch = (jj & 3) * 2 + (mi >> 1);
           ldsm_x4_t(vb + (jj >> 2) * L::kHalfBytes + swz(tk, ch), b0, b1, b2, b3);
-          mma_16816<T>(o[2 * jj], pa, b0 & vm0, b1 & vm1);
-          mma_16816<T>(o[2 * jj + 1], pa, b2 & vm0, b3 & vm1);
+          mma_16816<MT>(o[2 * jj], pa, b0 & vm0, b1 & vm1);
+          mma_16816<MT>(o[2 * jj + 1], pa, b2 & vm0, b3 & vm1);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar(st));
+      __syncwarp();  // (FP8 through staging: every lane is done with the staging tiles)
+      if (!L::kStaging && lane == 0) mbar_arrive(empty_bar(st));
     }
     n += nblk;
 
+    if constexpr (KV8) {  // the V scale of this KV head
+      const float vsc = __ldg(v_scale + u.kvh);
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[t][e] *= vsc;
+    }
     // ---- merge the warps' states
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -403,8 +578,17 @@ __global__ void __launch_bounds__((NCW + 2) * 32, 2)
     }
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-      *reinterpret_cast<float2*>(&co[warp][r0][t * 8 + 2 * quad]) = make_float2(o[t][0], o[t][1]);
-      *reinterpret_cast<float2*>(&co[warp][r1][t * 8 + 2 * quad]) = make_float2(o[t][2], o[t][3]);
+      if constexpr (fp8_direct) {  // n-tile t, columns 2q, 2q+1: head dims 32q + t, 32q + 16 + t
+        co[warp][r0][32 * quad + t] = o[t][0];
+        co[warp][r0][32 * quad + 16 + t] = o[t][1];
+        co[warp][r1][32 * quad + t] = o[t][2];
+        co[warp][r1][32 * quad + 16 + t] = o[t][3];
+      } else {
+        *reinterpret_cast<float2*>(&co[warp][r0][t * 8 + 2 * quad]) =
+            make_float2(o[t][0], o[t][1]);
+        *reinterpret_cast<float2*>(&co[warp][r1][t * 8 + 2 * quad]) =
+            make_float2(o[t][2], o[t][3]);
+      }
     }
     if (!consumers_sync()) return;
     epilogue<T, D, NCW>(s, u, cm, cl, co, out, w, tid, NCW * 32);

@@ -11,6 +11,10 @@
 // Lane layout for one block: for scores, lane = 2 * token + half, each lane
 // dots half of head_dim and a shuffle joins the halves; for P.V, lane owns
 // head dims lane, lane + 32, ...
+//
+// KV8: the cache holds FP8 e4m3 codes with one fp32 scale per KV head for K
+// and for V; codes are decoded to fp32 as they are loaded, the K scale folds
+// into the softmax scale and the V scale multiplies the accumulator.
 #pragma once
 
 #include "pa_sched.cuh"
@@ -40,12 +44,39 @@ __device__ __forceinline__ void load_half_row(const T* __restrict__ src, float (
   }
 }
 
-template <typename T, int D>
+template <int D>
+__device__ __forceinline__ void load_half_row(const uint8_t* __restrict__ src,
+                                              float (&dst)[D / 2]) {
+  static_assert(D / 2 % 16 == 0, "row half must be 16-byte vectors");
+  const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int c = 0; c < D / 2 / 16; ++c) {
+    const uint4 w = __ldg(p + c);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((wv[e >> 1] >> (16 * (e & 1))) & 0xffffu), __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+      dst[c * 16 + 2 * e] = f.x;
+      dst[c * 16 + 2 * e + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ float fp8_to_f32(uint8_t code) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
+  return __half2float(*reinterpret_cast<const __half*>(&h));
+}
+
+template <typename T, int D, bool KV8 = false>
 __global__ void __launch_bounds__(128, 1)
     attn_simt_kernel(Shape s, T* __restrict__ out, const T* __restrict__ q,
-                     const T* __restrict__ k_cache, const T* __restrict__ v_cache,
+                     const typename std::conditional<KV8, uint8_t, T>::type* __restrict__ k_cache,
+                     const typename std::conditional<KV8, uint8_t, T>::type* __restrict__ v_cache,
                      const int* __restrict__ block_tables, const int* __restrict__ qsl,
-                     const int* __restrict__ seq_lens, Work w, float scale_log2) {
+                     const int* __restrict__ seq_lens, Work w, float scale_log2,
+                     const float* __restrict__ k_scale, const float* __restrict__ v_scale) {
   constexpr int NW = 4;
   constexpr int HALF = D / 2;
   constexpr int PER = D / 32;
@@ -100,6 +131,7 @@ __global__ void __launch_bounds__(128, 1)
 
     const int nblk = ceil_div(u.kv_end - u.kv_begin, kBlock);
     const int* table = block_tables + static_cast<size_t>(u.row) * s.table_stride;
+    const float sl = KV8 ? scale_log2 * __ldg(k_scale + u.kvh) : scale_log2;
     for (int j = warp; j < nblk; j += NW) {
       const int blk_start = u.kv_begin + j * kBlock;
       // cache rows of keys 0-7 and 8-15 of this tile (two 8-token blocks, or
@@ -113,7 +145,10 @@ __global__ void __launch_bounds__(128, 1)
                          : y0;
       auto row_of = [&](int t) { return static_cast<size_t>(t < 8 ? y0 + t : y1 + t - 8); };
       float kr[HALF];
-      load_half_row<T, D>(k_cache + row_of(tok) * D + half * HALF, kr);
+      if constexpr (KV8)
+        load_half_row<D>(k_cache + row_of(tok) * D + half * HALF, kr);
+      else
+        load_half_row<T, D>(k_cache + row_of(tok) * D + half * HALF, kr);
       const int kidx = blk_start + tok;
 #pragma unroll
       for (int r = 0; r < kRows; ++r) {
@@ -123,7 +158,7 @@ __global__ void __launch_bounds__(128, 1)
           for (int e = 0; e < HALF; ++e) sc = fmaf(q_s[r][half * HALF + e], kr[e], sc);
           sc += __shfl_xor_sync(0xffffffffu, sc, 1);
           const int lim = u.lim0 + r / s.gs;
-          const float x = kidx < lim ? sc * scale_log2 : -INFINITY;
+          const float x = kidx < lim ? sc * sl : -INFINITY;
           float bm = x;
 #pragma unroll
           for (int off = 2; off < 32; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
@@ -144,11 +179,15 @@ __global__ void __launch_bounds__(128, 1)
       const int nvalid = u.kv_end - blk_start;  // V rows at or past this are padding
 #pragma unroll 4
       for (int t2 = 0; t2 < kBlock; ++t2) {
-        const T* vt = v_cache + row_of(t2) * D;
+        const auto* vt = v_cache + row_of(t2) * D;
         float vv[PER];
 #pragma unroll
-        for (int e = 0; e < PER; ++e)
-          vv[e] = t2 < nvalid ? to_f32<T>(vt[lane + 32 * e]) : 0.f;
+        for (int e = 0; e < PER; ++e) {
+          if constexpr (KV8)
+            vv[e] = t2 < nvalid ? fp8_to_f32(vt[lane + 32 * e]) : 0.f;
+          else
+            vv[e] = t2 < nvalid ? to_f32<T>(vt[lane + 32 * e]) : 0.f;
+        }
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
           if (r < nrows) {
@@ -160,6 +199,13 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
 
+    if constexpr (KV8) {  // the V scale of this KV head
+      const float vsc = __ldg(v_scale + u.kvh);
+#pragma unroll
+      for (int r = 0; r < kRows; ++r)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[r][e] *= vsc;
+    }
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
       if (lane == 0) {

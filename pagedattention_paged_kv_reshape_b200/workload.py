@@ -78,6 +78,14 @@ class PagedBatch:
     host_seq_lens: np.ndarray | None = None
     host_qsl: np.ndarray | None = None
     host_slots: np.ndarray | None = None
+    # FP8 (e4m3) cache: k_cache / v_cache hold uint8 codes; per-KV-head fp32 scales
+    kv_dtype: str = "same"
+    k_scale: torch.Tensor | None = None
+    v_scale: torch.Tensor | None = None
+
+    @property
+    def fp8(self) -> bool:
+        return self.kv_dtype == "fp8"
 
     @property
     def num_seqs(self) -> int:
@@ -118,14 +126,19 @@ def build_batch(requests, *, num_q_heads: int, num_kv_heads: int, head_dim: int,
                 seed: int, device="cpu", name: str = "custom", pool_factor: float = 1.0,
                 pool_blocks: int | None = None, shared_prefix_len: int = 0,
                 extra_table_cols: int = 1, poison: bool = True,
-                block_size: int = BLOCK_SIZE) -> PagedBatch:
+                block_size: int = BLOCK_SIZE, kv_dtype: str = "same") -> PagedBatch:
     """Lay out ``requests`` in a shuffled block pool and draw all values.
 
     ``pool_factor`` sizes the pool to that multiple of the blocks the batch
     needs (plus the poison block); ``pool_blocks`` fixes it instead.
     ``shared_prefix_len`` (a multiple of ``block_size``) is the length of the
     common prefix run used by requests with ``shares_prefix``.
+    ``kv_dtype="fp8"`` makes an FP8 (e4m3) cache: uint8 codes drawn as the e4m3
+    rounding of N(0,1) * 48 (torch's float8 conversion), per-KV-head scales
+    drawn from U[0.012, 0.024], and the NaN code 0x7F in unowned slots.
     """
+    if kv_dtype not in ("same", "fp8"):
+        raise ValueError(f"unknown kv_dtype {kv_dtype!r}")
     if dtype not in TORCH_DTYPES:
         raise ValueError(f"unknown dtype {dtype!r}")
     if shared_prefix_len % block_size:
@@ -183,12 +196,21 @@ def build_batch(requests, *, num_q_heads: int, num_kv_heads: int, head_dim: int,
     q = torch.empty((total_q, num_q_heads, head_dim), dtype=tdt, device=device)
     k_new = torch.empty((total_q, num_kv_heads, head_dim), dtype=tdt, device=device)
     v_new = torch.empty_like(k_new)
-    k_cache = torch.empty((pool_blocks, num_kv_heads, block_size, head_dim), dtype=tdt,
+    fp8 = kv_dtype == "fp8"
+    cdt = torch.float32 if fp8 else tdt
+    k_cache = torch.empty((pool_blocks, num_kv_heads, block_size, head_dim), dtype=cdt,
                           device=device)
     v_cache = torch.empty_like(k_cache)
     for t in (q, k_new, v_new, k_cache, v_cache):
         if t.numel():
             _randn_into(t, gen)
+    k_scale = v_scale = None
+    if fp8:
+        k_cache = (k_cache * 48.0).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        v_cache = (v_cache * 48.0).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        k_scale = torch.from_numpy(rng.uniform(0.012, 0.024, num_kv_heads).astype(np.float32))
+        v_scale = torch.from_numpy(rng.uniform(0.012, 0.024, num_kv_heads).astype(np.float32))
+        k_scale, v_scale = k_scale.to(device), v_scale.to(device)
 
     if poison and pool_blocks:
         live = np.zeros((pool_blocks, block_size), dtype=bool)
@@ -198,7 +220,7 @@ def build_batch(requests, *, num_q_heads: int, num_kv_heads: int, head_dim: int,
                 n = min(block_size, cached - pos)
                 live[tables[i, pos // block_size], :n] = True
         dead = torch.from_numpy(~live).to(device)
-        nan = float("nan")
+        nan = 0x7F if fp8 else float("nan")   # the e4m3 NaN code for an FP8 cache
         k_cache.masked_fill_(dead[:, None, :, None], nan)
         v_cache.masked_fill_(dead[:, None, :, None], nan)
 
@@ -214,6 +236,7 @@ def build_batch(requests, *, num_q_heads: int, num_kv_heads: int, head_dim: int,
         scale=1.0 / math.sqrt(head_dim), poison_block=poison_block,
         shared_blocks=[int(b) for b in shared],
         host_tables=tables, host_seq_lens=seq_lens, host_qsl=qsl, host_slots=slots,
+        kv_dtype=kv_dtype, k_scale=k_scale, v_scale=v_scale,
     )
 
 
@@ -298,6 +321,10 @@ CONFIGS = {
     "gqa_bs256_b32": dict(requests=gqa_requests, num_q_heads=32, num_kv_heads=8, head_dim=128,
                           dtype="bf16", pool_factor=1.25, kind="decode", block_size=32,
                           about="gqa_bs256 with 32-token blocks (\"vLLM 架构源码解析\" §5.1)"),
+    "gqa_bs256_fp8": dict(requests=gqa_requests, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                          dtype="bf16", pool_factor=1.25, kind="decode", kv_dtype="fp8",
+                          about="gqa_bs256 over an FP8 (e4m3) cache with per-KV-head scales "
+                                "(\"vLLM 深度拆解\" §10.1)"),
     "prefill_16x512": dict(requests=prefill_requests, num_q_heads=32, num_kv_heads=8,
                            head_dim=128, dtype="bf16", pool_factor=1.0, kind="varlen",
                            about="16 causal prefill chunks of 512 tokens on 1536 cached tokens, "

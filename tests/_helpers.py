@@ -37,7 +37,11 @@ def f64(t: torch.Tensor) -> np.ndarray:
 
 def gpu_cache_write(b: PagedBatch):
     kc, vc = b.k_cache.clone(), b.v_cache.clone()
-    pa.pa_reshape_and_cache(b.k_new, b.v_new, kc, vc, b.slot_mapping)
+    if b.fp8:
+        pa.pa_reshape_and_cache_fp8(b.k_new, b.v_new, kc, vc, b.slot_mapping, b.k_scale,
+                                    b.v_scale)
+    else:
+        pa.pa_reshape_and_cache(b.k_new, b.v_new, kc, vc, b.slot_mapping)
     return kc, vc
 
 
@@ -57,12 +61,21 @@ def gpu_attention(b: PagedBatch, kc, vc, varlen: bool | None = None, out=None):
         ws = poisoned_workspace(pa.pa_varlen_workspace_size(
             b.num_seqs, b.total_q, b.num_q_heads, b.num_kv_heads, b.head_dim, b.max_query_len,
             b.max_seq_len), b.q.device)
-        pa.pa_varlen(out, b.q, kc, vc, b.block_tables, b.query_start_loc, b.seq_lens,
-                     b.max_query_len, b.max_seq_len, b.scale, ws)
+        if b.fp8:
+            pa.pa_varlen_fp8(out, b.q, kc, vc, b.k_scale, b.v_scale, b.block_tables,
+                             b.query_start_loc, b.seq_lens, b.max_query_len, b.max_seq_len,
+                             b.scale, ws)
+        else:
+            pa.pa_varlen(out, b.q, kc, vc, b.block_tables, b.query_start_loc, b.seq_lens,
+                         b.max_query_len, b.max_seq_len, b.scale, ws)
     else:
         ws = poisoned_workspace(pa.pa_decode_workspace_size(
             b.num_seqs, b.num_q_heads, b.num_kv_heads, b.head_dim, b.max_seq_len), b.q.device)
-        pa.pa_decode(out, b.q, kc, vc, b.block_tables, b.seq_lens, b.max_seq_len, b.scale, ws)
+        if b.fp8:
+            pa.pa_decode_fp8(out, b.q, kc, vc, b.k_scale, b.v_scale, b.block_tables, b.seq_lens,
+                             b.max_seq_len, b.scale, ws)
+        else:
+            pa.pa_decode(out, b.q, kc, vc, b.block_tables, b.seq_lens, b.max_seq_len, b.scale, ws)
     pa.pa_get_device_error()
     return out
 
@@ -80,9 +93,21 @@ def oracle_step(b: PagedBatch, varlen: bool | None = None, seqs=None):
     """Oracle cache write then attention, on host copies of the batch."""
     varlen = (not b.is_decode) if varlen is None else varlen
     bs = b.block_size
+    q = host(b.q)
+    if b.fp8:
+        ks, vs = host(b.k_scale), host(b.v_scale)
+        kc, vc = O.reshape_and_cache_fp8(host(b.k_cache), host(b.v_cache), host(b.k_new),
+                                         host(b.v_new), b.host_slots, ks, vs, b.dtype,
+                                         block_size=bs)
+        if varlen:
+            out = O.paged_varlen_fp8(q, kc, vc, ks, vs, b.host_tables, b.host_qsl,
+                                     b.host_seq_lens, b.scale, b.dtype, block_size=bs, seqs=seqs)
+        else:
+            out = O.paged_decode_fp8(q, kc, vc, ks, vs, b.host_tables, b.host_seq_lens, b.scale,
+                                     b.dtype, block_size=bs, seqs=seqs)
+        return out, kc, vc
     kc, vc = O.reshape_and_cache(host(b.k_cache), host(b.v_cache), host(b.k_new),
                                  host(b.v_new), b.host_slots, block_size=bs)
-    q = host(b.q)
     if varlen:
         out = O.paged_varlen(q, kc, vc, b.host_tables, b.host_qsl, b.host_seq_lens, b.scale,
                              b.dtype, block_size=bs, seqs=seqs)
@@ -125,6 +150,17 @@ def oracle_rows(b: PagedBatch, rows, varlen: bool | None = None):
     varlen = (not b.is_decode) if varlen is None else varlen
     c = compact(b, rows)
     bs = b.block_size
+    if b.fp8:
+        ks, vs = host(b.k_scale), host(b.v_scale)
+        kc, vc = O.reshape_and_cache_fp8(c["kc"], c["vc"], c["k_new"], c["v_new"], c["slots"],
+                                         ks, vs, b.dtype, block_size=bs)
+        if varlen:
+            out = O.paged_varlen_fp8(c["q"], kc, vc, ks, vs, c["tables"], c["qsl"], c["lens"],
+                                     b.scale, b.dtype, block_size=bs)
+        else:
+            out = O.paged_decode_fp8(c["q"], kc, vc, ks, vs, c["tables"], c["lens"], b.scale,
+                                     b.dtype, block_size=bs)
+        return c["tokens"], out
     kc, vc = O.reshape_and_cache(c["kc"], c["vc"], c["k_new"], c["v_new"], c["slots"],
                                  block_size=bs)
     if varlen:
