@@ -40,3 +40,4 @@ from .fp8 import (  # noqa: F401,E402
     E4M3_MAX, e4m3_decode, e4m3_encode, dequantize, reshape_and_cache_fp8, paged_decode_fp8,
     paged_varlen_fp8,
 )
+from .rope import rope_table, rotate, rope_reshape_and_cache  # noqa: F401,E402
