@@ -419,6 +419,44 @@ def measure_block_ops(torch, pa, dev, peak) -> dict:
             "blocks": "8 KV heads x 16 tokens x 128 dims, bf16, K and V"}
 
 
+def measure_rope_write(torch, pa, dev, peak) -> dict:
+    """pa_rope_reshape_and_cache on 16384 new tokens (32 query / 8 KV heads,
+    head_dim 128, bf16, full rotation, NeoX pairs): q is read and written, k and
+    v read, both cache rows written, plus one table row, position and slot per
+    token -- about 410 MB per call, more than the L2."""
+    T, hq, hkv, d, bs = 16384, 32, 8, 128, 16
+    g = torch.Generator(device=dev).manual_seed(77)
+    q = torch.randn(T, hq, d, generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn(T, hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn(T, hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    nb = T // bs + 64
+    kc = torch.zeros(nb, hkv, bs, d, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(77))[:T // bs]
+    slots = (perm.repeat_interleave(bs) * bs + torch.arange(T) % bs).int().to(dev)
+    positions = (torch.arange(T) % 8192).int().to(dev)
+    inv = 10000.0 ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
+    ang = torch.arange(8192, dtype=torch.float64)[:, None] * inv[None, :]
+    table = torch.cat([ang.cos(), ang.sin()], 1).float().to(dev)
+    for _ in range(3):
+        pa.pa_rope_reshape_and_cache(q, k, v, kc, vc, slots, positions, table)
+    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s_ev.record()
+    iters = 20
+    for _ in range(iters):
+        pa.pa_rope_reshape_and_cache(q, k, v, kc, vc, slots, positions, table)
+    e_ev.record()
+    torch.cuda.synchronize()
+    pa.pa_get_device_error()
+    ms = s_ev.elapsed_time(e_ev) / iters
+    nbytes = (2 * T * hq * d * 2 + 2 * T * hkv * d * 2 + 2 * T * hkv * d * 2 + T * d * 4
+              + 8 * T)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"tokens": T, "ms": round(ms, 4), "algorithmic_bytes": nbytes, "gbs": round(gbs, 1),
+            "pct_of_hbm_peak": round(100 * gbs / peak, 1)}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -508,7 +546,7 @@ def run_ours(args):
         tensor_peak = measured_tensor_peak()
         per = {}
         for name in ("gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512", "gqa_bs256_b8",
-                     "gqa_bs256_b32", "gqa_bs256_fp8"):
+                     "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256"):
             if name == args.workload:
                 continue
             del b
@@ -536,6 +574,7 @@ def run_ours(args):
             per[name] = ent
         result["per_config"] = per
         result["block_ops"] = measure_block_ops(torch, pa, dev, peak)
+        result["rope_cache_write"] = measure_rope_write(torch, pa, dev, peak)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         del b

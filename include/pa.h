@@ -52,8 +52,9 @@
  *   block_idx]).  Entries past ceil(len/block_size) are never read.
  * - Grouped-query attention: query head h reads KV head
  *   h / (num_q_heads / num_kv_heads).  num_q_heads % num_kv_heads == 0.
- * - head_dim is 64 or 128.  dtype: PA_F32, PA_BF16 or PA_F16; q, k, v, the
- *   caches and out all have that dtype.  Arithmetic is fp32 with one
+ * - head_dim is 64 or 128, or 256 for bf16/f16 attention over a 16-bit cache
+ *   (the tensor-core decode kernel; no FP8 cache, no PA_PATH_SIMT).  dtype:
+ *   PA_F32, PA_BF16 or PA_F16; q, k, v, the caches and out all have that dtype.  Arithmetic is fp32 with one
  *   round-to-nearest-even conversion of the output.
  * - Errors: a status other than PA_OK returned by a call means nothing was
  *   launched (argument checks are done on the host before any launch) or a
@@ -130,6 +131,37 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
                                const int32_t* slot_mapping, int num_tokens, int num_kv_heads,
                                int head_dim, int block_size, int num_blocks, pa_dtype dtype,
                                void* stream);
+
+/*
+ * pa_rope_reshape_and_cache -- pa_reshape_and_cache with the rotary position
+ * embedding fused in (the kernel-fusion theme of "vLLM 深度拆解" §6.1: the
+ * elementwise work rides along with the neighbouring kernel, so q and k make
+ * one trip through HBM).  The pages do not define a position encoding; the
+ * rotation is RoFormer's: the first rot_dim dims of each head form rot_dim/2
+ * pairs -- (2i, 2i+1) when neox == 0, (i, i + rot_dim/2) when neox != 0 --
+ * and the pair (x1, x2) of token t becomes (x1 c - x2 s, x2 c + x1 s) with
+ * c = cos_sin[positions[t]][i] and s = cos_sin[positions[t]][rot_dim/2 + i].
+ * Dims from rot_dim on pass through.
+ *
+ *   q             [num_tokens, num_q_heads, head_dim], rotated IN PLACE
+ *   k, v          [num_tokens, num_kv_heads, head_dim], read only
+ *   k_cache,      as for pa_reshape_and_cache: token t's rotated k row and
+ *   v_cache         its v row go to slot slot_mapping[t] (slot < 0: padding,
+ *                   skipped; q is rotated all the same)
+ *   positions     int32 [num_tokens], each in [0, max_position)
+ *   cos_sin       fp32 [max_position, rot_dim]: cosines then sines
+ *
+ * Each result is computed in fp32 and rounded once to `dtype`.  A position
+ * outside [0, max_position) leaves that token's q and cache rows untouched
+ * and is recorded as PA_ERR_DEVICE_BOUNDS; slots as for pa_reshape_and_cache.
+ */
+pa_status pa_rope_reshape_and_cache(void* q, const void* k, const void* v, void* k_cache,
+                                    void* v_cache, const int32_t* slot_mapping,
+                                    const int32_t* positions, const float* cos_sin,
+                                    int max_position, int rot_dim, int neox, int num_tokens,
+                                    int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int num_blocks, pa_dtype dtype,
+                                    void* stream);
 
 /*
  * FP8 KV cache ("vLLM 深度拆解" §10.1: native FP8 with calibrated scales is

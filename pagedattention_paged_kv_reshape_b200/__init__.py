@@ -12,7 +12,9 @@ kernels, and this thin Python binding of it:
   inside a pool, swap-out / swap-in between the device and a host pool;
 * :func:`pa_reshape_and_cache_fp8`, :func:`pa_decode_fp8`,
   :func:`pa_varlen_fp8` -- the same path over an FP8 (e4m3) cache with
-  per-KV-head scales.
+  per-KV-head scales;
+* :func:`pa_rope_reshape_and_cache` -- the cache write with the rotary
+  position embedding of q and k fused in.
 
 PyTorch provides device memory and streams only.  The seeded workload
 generator lives in :mod:`.workload`; byte/flop accounting in :mod:`.accounting`.
@@ -34,6 +36,7 @@ from ._binding import (  # noqa: F401
     pa_get_device_error,
     pa_reshape_and_cache,
     pa_reshape_and_cache_fp8,
+    pa_rope_reshape_and_cache,
     pa_set_path,
     pa_status_string,
     pa_swap_blocks,

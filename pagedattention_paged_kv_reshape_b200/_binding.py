@@ -55,6 +55,9 @@ _SIGNATURES = {
     "pa_varlen_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _c_int,
                                _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                _c_float, _vp, _c_size, _c_int, _vp]),
+    "pa_rope_reshape_and_cache": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
+                                           _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                           _c_int, _c_int, _c_int, _vp]),
     "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _vp]),
     "pa_swap_blocks": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -150,6 +153,29 @@ def pa_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None) -> N
         _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), k.shape[0],
         k.shape[1], k.shape[2], k_cache.shape[2], k_cache.shape[0], _dtype_code(k),
         _stream(stream)))
+
+
+def pa_rope_reshape_and_cache(q, k, v, k_cache, v_cache, slot_mapping, positions, cos_sin,
+                              neox: bool = True, stream=None) -> None:
+    """Rotate ``q`` ``[T, Hq, D]`` in place and write the rotated ``k`` and the
+    ``v`` rows ``[T, Hkv, D]`` into the caches at ``slot_mapping``; angles from
+    ``cos_sin`` fp32 ``[max_position, rot_dim]`` at int32 ``positions``."""
+    _dense(q, k, v, k_cache, v_cache, slot_mapping, positions, cos_sin)
+    _require(q.dim() == 3 and k.shape == v.shape and k.dim() == 3 and q.shape[0] == k.shape[0]
+             and q.shape[2] == k.shape[2], "q [T, Hq, D], k/v [T, Hkv, D]")
+    _require(k_cache.shape == v_cache.shape and k_cache.dim() == 4
+             and k_cache.shape[1] == k.shape[1] and k_cache.shape[3] == k.shape[2],
+             "caches [num_blocks, Hkv, block_size, D]")
+    _require(q.dtype == k.dtype == v.dtype == k_cache.dtype == v_cache.dtype, "dtypes must match")
+    _require(slot_mapping.dtype == torch.int32 and positions.dtype == torch.int32
+             and slot_mapping.numel() == positions.numel() == q.shape[0],
+             "slot_mapping and positions must be int32 [T]")
+    _require(cos_sin.dtype == torch.float32 and cos_sin.dim() == 2, "cos_sin fp32 [P, rot_dim]")
+    _check(lib().pa_rope_reshape_and_cache(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+        _ptr(positions), _ptr(cos_sin), cos_sin.shape[0], cos_sin.shape[1], int(bool(neox)),
+        q.shape[0], q.shape[1], k.shape[1], q.shape[2], k_cache.shape[2], k_cache.shape[0],
+        _dtype_code(q), _stream(stream)))
 
 
 def _pool_code(t) -> int:

@@ -297,8 +297,10 @@ pa_status check_common(const AttnArgs& a) {
   if (a.num_q_heads <= 0 || a.num_kv_heads <= 0 || a.num_q_heads % a.num_kv_heads != 0)
     return fail(PA_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
                 a.num_q_heads, a.num_kv_heads);
-  if (a.head_dim != 64 && a.head_dim != 128)
-    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", a.head_dim);
+  if (a.head_dim != 64 && a.head_dim != 128 && a.head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128, 256)", a.head_dim);
+  if (a.head_dim == 256 && (a.dtype == PA_F32 || a.kv8()))
+    return fail(PA_ERR_UNSUPPORTED, "head_dim 256 runs on the bf16/f16 tensor-core path only");
   if (!supported_block_size(a.block_size))
     return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", a.block_size);
   if (!(std::isfinite(a.scale))) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
@@ -410,7 +412,9 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   pa_status st;
   const bool d128 = a.head_dim == 128;
   if constexpr (sizeof(T) == 2) {
-    if (use_mma)
+    if (a.head_dim == 256)
+      st = launch_mma<T, 256, false>(a, p, w);
+    else if (use_mma)
       st = a.kv8() ? (d128 ? launch_mma<T, 128, true>(a, p, w) : launch_mma<T, 64, true>(a, p, w))
                    : (d128 ? launch_mma<T, 128, false>(a, p, w)
                            : launch_mma<T, 64, false>(a, p, w));
@@ -449,7 +453,10 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = a.head_dim == 128
+  e = a.head_dim == 256
+          ? cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 256>, p.s, a.qsl, a.seq_lens, w,
+                               static_cast<T*>(a.out))
+      : a.head_dim == 128
           ? cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 128>, p.s, a.qsl, a.seq_lens, w,
                                static_cast<T*>(a.out))
           : cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 64>, p.s, a.qsl, a.seq_lens, w,
@@ -486,9 +493,12 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
       return fail(PA_ERR_UNSUPPORTED, "tensor-core path needs bf16 or f16 (got fp32)");
   }
   const bool use_mma = sixteen && path != PA_PATH_SIMT;
+  if (a.head_dim == 256 && !use_mma)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim 256 has no CUDA-core path");
   // Prefill-chunk rows (q_len >= one 128-row tile) go to the tcgen05 kernel
   // unless a family without it was forced.
-  p.s.chunk_qt = (use_mma && !a.kv8() && path != PA_PATH_MMA && p.chunk_qt > 0 &&
+  p.s.chunk_qt = (use_mma && !a.kv8() && a.head_dim != 256 && path != PA_PATH_MMA &&
+                  p.chunk_qt > 0 &&
                   a.max_query_len >= p.chunk_qt)
                      ? p.chunk_qt
                      : 0;
@@ -535,8 +545,8 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
   if (!valid_dtype(dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks < 0)
     return fail(PA_ERR_INVALID_ARG, "bad sizes");
-  if (head_dim != 64 && head_dim != 128)
-    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128, 256)", head_dim);
   if (!supported_block_size(block_size))
     return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", block_size);
   if (num_tokens == 0) return PA_OK;
@@ -612,6 +622,65 @@ pa_status pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, 
   return PA_OK;
 }
 
+pa_status pa_rope_reshape_and_cache(void* q, const void* k, const void* v, void* k_cache,
+                                    void* v_cache, const int32_t* slot_mapping,
+                                    const int32_t* positions, const float* cos_sin,
+                                    int max_position, int rot_dim, int neox, int num_tokens,
+                                    int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int num_blocks, pa_dtype dtype,
+                                    void* stream) {
+  if (!valid_dtype(dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks < 0 ||
+      max_position <= 0)
+    return fail(PA_ERR_INVALID_ARG, "bad sizes");
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128, 256)", head_dim);
+  if (!supported_block_size(block_size))
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", block_size);
+  if (rot_dim < 2 || rot_dim > head_dim || rot_dim % 2 != 0)
+    return fail(PA_ERR_INVALID_ARG, "rot_dim %d must be even and in [2, head_dim]", rot_dim);
+  if (num_tokens == 0) return PA_OK;
+  const void* ptrs[] = {q, k, v, k_cache, v_cache};
+  for (const void* p : ptrs) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned(p, 16)) return fail(PA_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  }
+  if (!slot_mapping || !positions || !cos_sin || !aligned(slot_mapping, 4) ||
+      !aligned(positions, 4) || !aligned(cos_sin, 4))
+    return fail(PA_ERR_INVALID_ARG, "bad slot_mapping / positions / cos_sin pointer");
+  const long long warps = static_cast<long long>(num_tokens) * (num_q_heads + num_kv_heads);
+  const long long blocks = (warps * 32 + 255) / 256;
+  if (blocks > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many tokens");
+  const auto st = static_cast<cudaStream_t>(stream);
+  const unsigned g = static_cast<unsigned>(blocks);
+  const long long slots = static_cast<long long>(num_blocks) * block_size;
+  switch (dtype) {
+    case PA_BF16:
+      pa::rope_reshape_and_cache_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+          static_cast<__nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+          static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(k_cache),
+          static_cast<__nv_bfloat16*>(v_cache), slot_mapping, positions, cos_sin, max_position,
+          rot_dim, neox != 0, num_tokens, num_q_heads, num_kv_heads, head_dim, block_size, slots);
+      break;
+    case PA_F16:
+      pa::rope_reshape_and_cache_kernel<__half><<<g, 256, 0, st>>>(
+          static_cast<__half*>(q), static_cast<const __half*>(k), static_cast<const __half*>(v),
+          static_cast<__half*>(k_cache), static_cast<__half*>(v_cache), slot_mapping, positions,
+          cos_sin, max_position, rot_dim, neox != 0, num_tokens, num_q_heads, num_kv_heads,
+          head_dim, block_size, slots);
+      break;
+    default:
+      pa::rope_reshape_and_cache_kernel<float><<<g, 256, 0, st>>>(
+          static_cast<float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+          static_cast<float*>(k_cache), static_cast<float*>(v_cache), slot_mapping, positions,
+          cos_sin, max_position, rot_dim, neox != 0, num_tokens, num_q_heads, num_kv_heads,
+          head_dim, block_size, slots);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rope_reshape_and_cache launch");
+  return PA_OK;
+}
+
 // Device-visible address of a pointer the kernels may dereference: device
 // memory as is, page-locked host memory through its mapped address.  Pageable
 // host memory is refused.
@@ -644,8 +713,8 @@ static pa_status launch_block_copy(const void* src_k, const void* src_v, void* d
   if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || src_num_blocks < 0 ||
       dst_num_blocks < 0)
     return fail(PA_ERR_INVALID_ARG, "bad sizes");
-  if (head_dim != 64 && head_dim != 128)
-    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128, 256)", head_dim);
   if (!supported_block_size(block_size))
     return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", block_size);
   if (num_pairs == 0) return PA_OK;
@@ -807,8 +876,8 @@ pa_status pa_get_device_error(void* stream) {
   static const char* where[] = {"?", "reshape_and_cache slot", "block-table entry",
                                 "row metadata", "wait for K/V tile", "wait for free stage",
                                 "wait for query tile", "tensor memory", "wait for MMA/barrier",
-                                "block copy pair"};
-  const int w = rec.where >= 0 && rec.where <= 9 ? rec.where : 0;
+                                "block copy pair", "rope position"};
+  const int w = rec.where >= 0 && rec.where <= 10 ? rec.where : 0;
   return fail(static_cast<pa_status>(rec.code), "device: %s (%s; a=%lld b=%lld)",
               pa_status_string(static_cast<pa_status>(rec.code)), where[w], rec.a, rec.b);
 }

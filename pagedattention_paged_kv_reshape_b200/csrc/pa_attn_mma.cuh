@@ -71,7 +71,9 @@ struct MmaLayout {
   static constexpr int kSmem = kBytes + 1024;  // slack to align the base to 1024 B
   static constexpr int kThreads = (NCW + 2) * 32;
   static_assert(kOffQ % 1024 == 0 && kQSlotBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
-  static_assert(kSmem <= 116 * 1024, "two CTAs per SM");
+  // two CTAs per SM up to head_dim 128; one at 256
+  static_assert(D > 128 || kSmem <= 116 * 1024, "two CTAs per SM");
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
 
 // Byte offset, inside one 128 B-swizzled tile half, of the 16-byte chunk `ch`
@@ -137,7 +139,7 @@ __device__ __forceinline__ void convert_fp8_tile(uint32_t src, uint32_t dst, int
 }
 
 template <typename T, int D, int NCW, int STAGES, bool KV8 = false>
-__global__ void __launch_bounds__((NCW + 2) * 32, 2)
+__global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, Shape s, T* __restrict__ out,

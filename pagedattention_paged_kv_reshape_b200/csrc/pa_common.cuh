@@ -54,6 +54,7 @@ enum ErrWhere : int {
   kWhereTmem = 7,
   kWhereWaitMma = 8,
   kWhereCopyPair = 9,
+  kWhereRopePos = 10,
 };
 
 __device__ __forceinline__ void report_error(unsigned code, int where, long long a, long long b) {

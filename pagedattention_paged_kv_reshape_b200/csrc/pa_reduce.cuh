@@ -61,7 +61,12 @@ __global__ void __launch_bounds__(256) reduce_kernel(Shape s, const int* __restr
           for (int j = 0; j < kUnroll; ++j) {  // issue every load first
             const int jj = min(j0 + j, n - 1);
             const float* src = po + static_cast<size_t>(p0 + jj) * D;
-            if constexpr (kPer == 4) {
+            if constexpr (kPer == 8) {
+              const float4 a = *reinterpret_cast<const float4*>(src);
+              const float4 b = *reinterpret_cast<const float4*>(src + 4);
+              v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
+              v[j][4] = b.x; v[j][5] = b.y; v[j][6] = b.z; v[j][7] = b.w;
+            } else if constexpr (kPer == 4) {
               const float4 a = *reinterpret_cast<const float4*>(src);
               v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
             } else {

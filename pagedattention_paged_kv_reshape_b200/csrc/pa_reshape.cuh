@@ -85,4 +85,74 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Rotary position embedding fused with the cache write ("vLLM 深度拆解" §6.1:
+// fold elementwise work into the neighbouring kernel so activations cross
+// HBM once).  The rotation is RoFormer's: the first rot_dim dims of a head
+// form rot_dim/2 pairs -- (2i, 2i+1), or (i, i + rot_dim/2) with `neox` --
+// and the pair (x1, x2) of a token at position p becomes
+// (x1 c - x2 s, x2 c + x1 s) with c, s = cos_sin[p][i], cos_sin[p][R/2 + i].
+// One warp per (token, head): a query head is rotated in place; a KV head
+// writes its rotated k row and its v row into the cache at the token's slot
+// (padding tokens, slot < 0, rotate q only).  Each result is computed in fp32
+// and rounded once to the storage type.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    rope_reshape_and_cache_kernel(T* __restrict__ q, const T* __restrict__ k,
+                                  const T* __restrict__ v, T* __restrict__ k_cache,
+                                  T* __restrict__ v_cache, const int* __restrict__ slot_mapping,
+                                  const int* __restrict__ positions,
+                                  const float* __restrict__ cos_sin, int max_position,
+                                  int rot_dim, bool neox, int num_tokens, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  long long num_slots) {
+  const int heads = num_q_heads + num_kv_heads;
+  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= static_cast<long long>(num_tokens) * heads) return;
+  const int t = static_cast<int>(gw / heads), h = static_cast<int>(gw % heads);
+  const int pos = __ldg(positions + t);
+  if (pos < 0 || pos >= max_position) {
+    if (lane == 0 && h == 0) report_error(PA_ERR_DEVICE_BOUNDS, kWhereRopePos, t, pos);
+    return;
+  }
+  const float* cs = cos_sin + static_cast<size_t>(pos) * rot_dim;
+  const int half = rot_dim / 2;
+  auto pair = [&](int i, int& i1, int& i2) {
+    i1 = neox ? i : 2 * i;
+    i2 = neox ? i + half : 2 * i + 1;
+  };
+  if (h < num_q_heads) {
+    T* x = q + (static_cast<size_t>(t) * num_q_heads + h) * head_dim;
+    for (int i = lane; i < half; i += 32) {
+      int i1, i2;
+      pair(i, i1, i2);
+      const float c = __ldg(cs + i), sn = __ldg(cs + half + i);
+      const float x1 = to_f32<T>(x[i1]), x2 = to_f32<T>(x[i2]);
+      x[i1] = from_f32<T>(fmaf(x1, c, -x2 * sn));
+      x[i2] = from_f32<T>(fmaf(x2, c, x1 * sn));
+    }
+    return;
+  }
+  const int kh = h - num_q_heads;
+  const int slot = __ldg(slot_mapping + t);
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (lane == 0) report_error(PA_ERR_DEVICE_BOUNDS, kWhereReshapeSlot, t, slot);
+    return;
+  }
+  const long long blk = slot / block_size, off = slot % block_size;
+  const size_t src = (static_cast<size_t>(t) * num_kv_heads + kh) * head_dim;
+  const size_t dst = ((blk * num_kv_heads + kh) * block_size + off) * head_dim;
+  for (int i = lane; i < half; i += 32) {
+    int i1, i2;
+    pair(i, i1, i2);
+    const float c = __ldg(cs + i), sn = __ldg(cs + half + i);
+    const float x1 = to_f32<T>(k[src + i1]), x2 = to_f32<T>(k[src + i2]);
+    k_cache[dst + i1] = from_f32<T>(fmaf(x1, c, -x2 * sn));
+    k_cache[dst + i2] = from_f32<T>(fmaf(x2, c, x1 * sn));
+  }
+  for (int e = rot_dim + lane; e < head_dim; e += 32) k_cache[dst + e] = k[src + e];
+  for (int e = lane; e < head_dim; e += 32) v_cache[dst + e] = v[src + e];
+}
+
 }  // namespace pa

@@ -325,6 +325,10 @@ CONFIGS = {
                           dtype="bf16", pool_factor=1.25, kind="decode", kv_dtype="fp8",
                           about="gqa_bs256 over an FP8 (e4m3) cache with per-KV-head scales "
                                 "(\"vLLM 深度拆解\" §10.1)"),
+    "gqa_bs256_d256": dict(requests=gqa_requests, num_q_heads=16, num_kv_heads=4,
+                           head_dim=256, dtype="bf16", pool_factor=1.25, kind="decode",
+                           about="gqa_bs256's lengths with head_dim 256, 16/4 heads (the same "
+                                 "KV bytes per token)"),
     "prefill_16x512": dict(requests=prefill_requests, num_q_heads=32, num_kv_heads=8,
                            head_dim=128, dtype="bf16", pool_factor=1.0, kind="varlen",
                            about="16 causal prefill chunks of 512 tokens on 1536 cached tokens, "

@@ -122,6 +122,8 @@ def _decode(lib, **kw):
     (dict(hq=6, hkv=4), pa.Status.INVALID_ARG),        # Hq % Hkv != 0
     (dict(hkv=0), pa.Status.INVALID_ARG),
     (dict(d=96), pa.Status.UNSUPPORTED),
+    (dict(d=512), pa.Status.UNSUPPORTED),
+    (dict(d=256, dt=0), pa.Status.UNSUPPORTED),        # 256: bf16/f16 tensor-core path only
     (dict(bs=24), pa.Status.UNSUPPORTED),
     (dict(bs=64), pa.Status.UNSUPPORTED),
     (dict(dt=7), pa.Status.INVALID_ARG),

@@ -40,7 +40,8 @@ def decode_batch(lengths, hq, hkv, d, dtype, seed=0, **kw):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dtype,d,bs", [("f32", 64, 16), ("bf16", 128, 16), ("f16", 64, 16),
-                                        ("bf16", 64, 16), ("bf16", 128, 8), ("f32", 64, 32)])
+                                        ("bf16", 64, 16), ("bf16", 128, 8), ("f32", 64, 32),
+                                        ("bf16", 256, 16), ("f32", 256, 8)])
 def test_reshape_and_cache_bit_exact(dtype, d, bs):
     b = W.build_batch([W.Request(L, q) for L, q in [(1, 1), (40, 7), (300, 300), (17, 1)]],
                       num_q_heads=4, num_kv_heads=4, head_dim=d, dtype=dtype, seed=3, device=DEV,
@@ -226,6 +227,37 @@ def test_block_sizes_match_oracle(case, path):
         out_d, _, _ = gpu_step(bd, varlen=False)
         ref_d, _, _ = oracle_step(bd, varlen=False)
         assert_close(out_d, ref_d, dtype, f"decode block_size {bs} case {case} ({path})")
+
+
+HEAD_DIM_256_CASES = [
+    # head_dim 256 runs on the bf16/f16 tensor-core decode kernel (chunk rows too)
+    ([(700, 37), (1, 1), (2000, 1), (600, 160), (9, 9)], 16, 2, "bf16"),    # group 8
+    ([(1300, 1), (33, 1), (4096, 1)], 8, 8, "f16"),                          # MHA, split-K
+    ([(520, 20), (17, 17), (1025, 1)], 32, 8, "bf16"),                      # group 4
+]
+
+
+@pytest.mark.parametrize("case", range(len(HEAD_DIM_256_CASES)))
+def test_head_dim_256_matches_oracle(case):
+    rows, hq, hkv, dtype = HEAD_DIM_256_CASES[case]
+    b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
+                      head_dim=256, dtype=dtype, seed=700 + case, device=DEV, pool_factor=1.2)
+    varlen = any(q_ != 1 for _, q_ in rows)
+    out, kc, vc = gpu_step(b, varlen=varlen)
+    ref, okc, _ = oracle_step(b, varlen=varlen)
+    assert np.array_equal(host(kc).view(np.uint8), okc.view(np.uint8))
+    assert_close(out, ref, dtype, f"head_dim 256 case {case}")
+
+
+def test_head_dim_256_refuses_cuda_core_paths():
+    b = decode_batch([100, 40], 8, 2, 256, "bf16", seed=71)
+    kc, vc = gpu_cache_write(b)
+    ws = pa.alloc_workspace(pa.pa_decode_workspace_size(2, 8, 2, 256, 100), DEV)
+    pa.pa_set_path(pa.Path.SIMT)
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode(torch.empty_like(b.q), b.q, kc, vc, b.block_tables, b.seq_lens, 100,
+                     b.scale, ws)
+    assert e.value.status == pa.Status.UNSUPPORTED
 
 
 def test_chunk_kernel_agrees_with_decode_kernel_tiles():
