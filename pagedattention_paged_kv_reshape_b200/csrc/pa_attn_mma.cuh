@@ -90,6 +90,16 @@ __device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two) {
   return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
+// Four e4m3 codes -> two f16x2: codes 0, 1 into `lo`, codes 2, 3 into `hi`.
+__device__ __forceinline__ void fp8x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 __device__ __forceinline__ void lds128(uint32_t addr, uint32_t (&w)[4]) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
@@ -460,9 +470,11 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
             uint32_t w[4];  // key nt*8+g, dims 64G + 16 q4 .. +15
             lds128(kb + swz(nt * 8 + g, 4 * G + q4), w);
 #pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4)
-              mma_16816<MT>(sacc[nt], qa[4 * G + s4], fp8x2_to_f16x2(w[s4]),
-                            fp8x2_to_f16x2(w[s4] >> 16));
+            for (int s4 = 0; s4 < 4; ++s4) {
+              uint32_t b0, b1;
+              fp8x4_to_f16x2x2(w[s4], b0, b1);
+              mma_16816<MT>(sacc[nt], qa[4 * G + s4], b0, b1);
+            }
           }
         }
       } else {
@@ -530,30 +542,54 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
         vm1 = (t0 + 8 < nv ? 0x0000ffffu : 0u) | (t0 + 9 < nv ? 0xffff0000u : 0u);
       }
       if constexpr (fp8_direct) {  // V from the bytes loaded above
+        auto pv8 = [&](bool masked) {
 #pragma unroll
-        for (int jw = 0; jw < 4; ++jw) {
+          for (int jw = 0; jw < 4; ++jw) {
 #pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {  // bytes 2hb, 2hb+1 of word jw: n-tiles 4jw+2hb, +1
-            const uint32_t sel = hb ? 0x7362u : 0x5140u;
-            const uint32_t lo = prmt(va[jw], vb1[jw], sel);  // (key 2q4, 2q4+1) x two dims
-            const uint32_t hi = prmt(vc[jw], vd[jw], sel);   // (key 2q4+8, 2q4+9)
-            const int j = 4 * jw + 2 * hb;
-            mma_16816<MT>(o[j], pa, fp8x2_to_f16x2(lo) & vm0, fp8x2_to_f16x2(hi) & vm1);
-            mma_16816<MT>(o[j + 1], pa, fp8x2_to_f16x2(lo >> 16) & vm0,
-                          fp8x2_to_f16x2(hi >> 16) & vm1);
+            for (int hb = 0; hb < 2; ++hb) {  // bytes 2hb, 2hb+1 of word jw: n-tiles 4jw+2hb, +1
+              const uint32_t sel = hb ? 0x7362u : 0x5140u;
+              uint32_t l0, l1, h0, h1;  // (key 2q4, 2q4+1) and (key 2q4+8, 2q4+9), two dims
+              fp8x4_to_f16x2x2(prmt(va[jw], vb1[jw], sel), l0, l1);
+              fp8x4_to_f16x2x2(prmt(vc[jw], vd[jw], sel), h0, h1);
+              if (masked) {
+                l0 &= vm0;
+                l1 &= vm0;
+                h0 &= vm1;
+                h1 &= vm1;
+              }
+              const int j = 4 * jw + 2 * hb;
+              mma_16816<MT>(o[j], pa, l0, h0);
+              mma_16816<MT>(o[j + 1], pa, l1, h1);
+            }
           }
-        }
+        };
+        if (blk_start + kBlock > u.kv_end)  // padding rows: only the last tile has them
+          pv8(true);
+        else
+          pv8(false);
       } else {
         const int mi = lane >> 3;
         const int tk = (lane & 7) + ((mi & 1) << 3);
+        auto pv16 = [&](bool masked) {
 #pragma unroll
-        for (int jj = 0; jj < KSTEPS; ++jj) {
-          uint32_t b0, b1, b2, b3;
-          const int ch = (jj & 3) * 2 + (mi >> 1);
-          ldsm_x4_t(vb + (jj >> 2) * L::kHalfBytes + swz(tk, ch), b0, b1, b2, b3);
-          mma_16816<MT>(o[2 * jj], pa, b0 & vm0, b1 & vm1);
-          mma_16816<MT>(o[2 * jj + 1], pa, b2 & vm0, b3 & vm1);
-        }
+          for (int jj = 0; jj < KSTEPS; ++jj) {
+            uint32_t b0, b1, b2, b3;
+            const int ch = (jj & 3) * 2 + (mi >> 1);
+            ldsm_x4_t(vb + (jj >> 2) * L::kHalfBytes + swz(tk, ch), b0, b1, b2, b3);
+            if (masked) {
+              b0 &= vm0;
+              b1 &= vm1;
+              b2 &= vm0;
+              b3 &= vm1;
+            }
+            mma_16816<MT>(o[2 * jj], pa, b0, b1);
+            mma_16816<MT>(o[2 * jj + 1], pa, b2, b3);
+          }
+        };
+        if (blk_start + kBlock > u.kv_end)  // padding rows: only the last tile has them
+          pv16(true);
+        else
+          pv16(false);
       }
       __syncwarp();  // (FP8 through staging: every lane is done with the staging tiles)
       if (!L::kStaging && lane == 0) mbar_arrive(empty_bar(st));
