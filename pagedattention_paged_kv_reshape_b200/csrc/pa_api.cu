@@ -648,33 +648,35 @@ pa_status pa_rope_reshape_and_cache(void* q, const void* k, const void* v, void*
   if (!slot_mapping || !positions || !cos_sin || !aligned(slot_mapping, 4) ||
       !aligned(positions, 4) || !aligned(cos_sin, 4))
     return fail(PA_ERR_INVALID_ARG, "bad slot_mapping / positions / cos_sin pointer");
-  const long long warps = static_cast<long long>(num_tokens) * (num_q_heads + num_kv_heads);
+  // quads of four elements line up with both pair layouts when rot_dim is a
+  // multiple of 8; the table rows then start 16-byte aligned if the base is
+  const bool vec = rot_dim % 8 == 0 && aligned(cos_sin, 16);
+  const long long parts = vec ? (num_q_heads + 7) / 8 + (num_kv_heads + 7) / 8
+                              : static_cast<long long>(num_q_heads) + num_kv_heads;
+  const long long warps = static_cast<long long>(num_tokens) * parts;
   const long long blocks = (warps * 32 + 255) / 256;
   if (blocks > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many tokens");
   const auto st = static_cast<cudaStream_t>(stream);
   const unsigned g = static_cast<unsigned>(blocks);
   const long long slots = static_cast<long long>(num_blocks) * block_size;
+  auto launch = [&](auto* tag) {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    auto kern = vec ? pa::rope_reshape_and_cache_vec_kernel<T> : pa::rope_reshape_and_cache_kernel<T>;
+    kern<<<g, 256, 0, st>>>(static_cast<T*>(q), static_cast<const T*>(k),
+                            static_cast<const T*>(v), static_cast<T*>(k_cache),
+                            static_cast<T*>(v_cache), slot_mapping, positions, cos_sin,
+                            max_position, rot_dim, neox != 0, num_tokens, num_q_heads,
+                            num_kv_heads, head_dim, block_size, slots);
+  };
   switch (dtype) {
     case PA_BF16:
-      pa::rope_reshape_and_cache_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
-          static_cast<__nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-          static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(k_cache),
-          static_cast<__nv_bfloat16*>(v_cache), slot_mapping, positions, cos_sin, max_position,
-          rot_dim, neox != 0, num_tokens, num_q_heads, num_kv_heads, head_dim, block_size, slots);
+      launch(static_cast<__nv_bfloat16*>(nullptr));
       break;
     case PA_F16:
-      pa::rope_reshape_and_cache_kernel<__half><<<g, 256, 0, st>>>(
-          static_cast<__half*>(q), static_cast<const __half*>(k), static_cast<const __half*>(v),
-          static_cast<__half*>(k_cache), static_cast<__half*>(v_cache), slot_mapping, positions,
-          cos_sin, max_position, rot_dim, neox != 0, num_tokens, num_q_heads, num_kv_heads,
-          head_dim, block_size, slots);
+      launch(static_cast<__half*>(nullptr));
       break;
     default:
-      pa::rope_reshape_and_cache_kernel<float><<<g, 256, 0, st>>>(
-          static_cast<float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-          static_cast<float*>(k_cache), static_cast<float*>(v_cache), slot_mapping, positions,
-          cos_sin, max_position, rot_dim, neox != 0, num_tokens, num_q_heads, num_kv_heads,
-          head_dim, block_size, slots);
+      launch(static_cast<float*>(nullptr));
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "rope_reshape_and_cache launch");

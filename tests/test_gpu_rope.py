@@ -30,16 +30,33 @@ def within_ulp(got: np.ndarray, ref: np.ndarray, dtype: str, what: str):
     assert not bad.any(), f"{what}: {bad.sum()} values off by more than one ulp"
 
 
-@pytest.mark.parametrize("dtype,d,rot,neox,bs", [("bf16", 128, 128, True, 16),
-                                                ("f16", 64, 32, False, 8),
-                                                ("f32", 128, 64, True, 32),
-                                                ("bf16", 64, 64, False, 16)])
-def test_rope_cache_write_matches_oracle(dtype, d, rot, neox, bs):
+# (q dtype, head_dim, rot_dim, NeoX pairs, block_size, q heads, KV heads, table
+# offset in floats).  rot_dim a multiple of 8 with an aligned table takes the
+# vector kernel (8-head parts: 24/12 heads make ragged parts); rot_dim 36 or 62,
+# or a table 4 bytes off alignment, take the per-element kernel.
+ROPE_CASES = [("bf16", 128, 128, True, 16, 8, 2, 0),
+              ("f16", 64, 32, False, 8, 8, 2, 0),
+              ("f32", 128, 64, True, 32, 8, 2, 0),
+              ("bf16", 64, 64, False, 16, 8, 2, 0),
+              ("bf16", 128, 128, False, 16, 24, 12, 0),
+              ("f16", 256, 192, True, 32, 24, 12, 0),
+              ("f32", 64, 56, False, 16, 4, 4, 0),
+              ("bf16", 128, 36, True, 16, 8, 2, 0),
+              ("f16", 64, 62, False, 8, 8, 4, 0),
+              ("bf16", 128, 128, True, 16, 8, 2, 1)]
+
+
+@pytest.mark.parametrize("dtype,d,rot,neox,bs,hq,hkv,offset", ROPE_CASES)
+def test_rope_cache_write_matches_oracle(dtype, d, rot, neox, bs, hq, hkv, offset):
     b = W.build_batch([W.Request(L, q) for L, q in [(1, 1), (40, 7), (300, 300), (17, 1)]],
-                      num_q_heads=8, num_kv_heads=2, head_dim=d, dtype=dtype, seed=9,
+                      num_q_heads=hq, num_kv_heads=hkv, head_dim=d, dtype=dtype, seed=9,
                       device=DEV, pool_factor=1.3, block_size=bs)
     maxp = 512
-    table = torch.from_numpy(O.rope_table(maxp, rot).astype(np.float32)).to(DEV)
+    host_table = O.rope_table(maxp, rot).astype(np.float32)
+    buf = torch.empty(maxp * rot + offset, dtype=torch.float32, device=DEV)
+    table = buf[offset:].view(maxp, rot)
+    table.copy_(torch.from_numpy(host_table))
+    assert (table.data_ptr() % 16 == 0) == (offset == 0)
     positions = torch.from_numpy(np.concatenate(
         [np.arange(r.seq_len - r.q_len, r.seq_len) for r in b.requests]).astype(np.int32)).to(DEV)
     slots = b.slot_mapping.clone()
@@ -70,10 +87,13 @@ def test_rope_cache_write_matches_oracle(dtype, d, rot, neox, bs):
     assert np.array_equal(k_now[written][..., rot:], ok.transpose(0, 2, 1, 3)[written][..., rot:])
 
 
-def test_rope_bad_position_is_reported():
+@pytest.mark.parametrize("offset", [0, 1])   # vector kernel, per-element kernel
+def test_rope_bad_position_is_reported(offset):
     b = W.build_batch([W.Request(20, 4)], num_q_heads=4, num_kv_heads=2, head_dim=64,
                       dtype="bf16", seed=2, device=DEV)
-    table = torch.from_numpy(O.rope_table(32, 64).astype(np.float32)).to(DEV)
+    buf = torch.empty(32 * 64 + offset, dtype=torch.float32, device=DEV)
+    table = buf[offset:].view(32, 64)
+    table.copy_(torch.from_numpy(O.rope_table(32, 64).astype(np.float32)))
     positions = torch.tensor([16, 17, 40, 19], dtype=torch.int32, device=DEV)   # 40 >= 32
     q = b.q.clone()
     pa.pa_rope_reshape_and_cache(q, b.k_new, b.v_new, b.k_cache, b.v_cache, b.slot_mapping,
