@@ -8,7 +8,9 @@ through the C ABI.  The KV cache is resident in HBM (it is the engine's state);
 ``value`` is the step's algorithmic bytes (every visible K/V row once, q, out,
 block-table entries, the cache write) over the device time of the step, in
 GB/s.  ``e2e`` repeats the measurement with each step's inputs copied from
-pinned host memory and its output copied back inside the timed region.
+pinned host memory and its output copied back inside the timed region (the
+copies on their own streams, double-buffered, overlapping the compute of the
+neighbouring steps).
 
 Usage:  python bench.py [--gpus N --steps K --warmup W] [--workload NAME]
         python bench.py --impl reference ...   (the fp64 oracle on host cores)
@@ -296,8 +298,11 @@ def launches_per_step(b) -> int:
     return 1 + 2 + (1 if split else 0)   # cache write + schedule + attention (+ reduce)
 
 
-def time_steps(torch, pa, b, steps, warmup):
-    """Device time of ``steps`` steps and the mean duration of the attention call."""
+def time_steps(torch, pa, b, steps, warmup, sample_every=10):
+    """Device time of ``steps`` steps and the mean duration of the attention
+    call, taken with events around the call of every ``sample_every``-th step
+    inside the same timed region (events around every call cost ~2% of the
+    step time on B200; one in ten costs nothing measurable)."""
     out = torch.empty_like(b.q)
     ws = workspace_for(pa, b)
     step, attend = make_step(pa, b, out, ws)
@@ -306,52 +311,84 @@ def time_steps(torch, pa, b, steps, warmup):
     pa.pa_get_device_error()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    every = sample_every if steps >= sample_every else 1
+    ev = []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(steps):
+        if i % every:
+            step()
+            continue
         cache_write(pa, b, b.k_new, b.v_new, b.slot_mapping)
-        ev[i][0].record(stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
         attend()
-        ev[i][1].record(stream)
+        e1.record(stream)
+        ev.append((e0, e1))
     end.record(stream)
     torch.cuda.synchronize()
     pa.pa_get_device_error()
     total_ms = start.elapsed_time(end)
-    attn_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
+    attn_ms = statistics.fmean(e0.elapsed_time(e1) for e0, e1 in ev)
     return total_ms, attn_ms, out
 
 
 def time_e2e(torch, pa, b, steps):
-    """Each step: H2D of the step's inputs from pinned memory, the step, D2H of out."""
+    """Each step copies its inputs from pinned host memory to the device and its
+    output back, all inside the timed region.  The copies run on their own
+    streams with two sets of device buffers, so step i+1's inputs move while
+    step i computes and step i's output returns while step i+1 computes (a
+    serving loop's overlap); events order every reuse of a buffer."""
     names = ["q", "k_new", "v_new", "slot_mapping", "block_tables", "seq_lens", "query_start_loc"]
     host = {n: getattr(b, n).cpu().pin_memory() for n in names}
-    dev = {n: torch.empty_like(getattr(b, n)) for n in names}
-    out = torch.empty_like(b.q)
-    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    comp = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    bufs = []
+    for _ in range(2):
+        bufs.append({"dev": {n: torch.empty_like(getattr(b, n)) for n in names},
+                     "out": torch.empty_like(b.q),
+                     "out_host": torch.empty(b.q.shape, dtype=b.q.dtype, pin_memory=True),
+                     "ready": torch.cuda.Event(), "computed": torch.cuda.Event(),
+                     "returned": torch.cuda.Event(), "used": False})
     ws = workspace_for(pa, b)
 
-    def step():
-        for n in names:
-            dev[n].copy_(host[n], non_blocking=True)
+    def step(i):
+        buf = bufs[i % 2]
+        dev = buf["dev"]
+        with torch.cuda.stream(h2d_s):
+            if buf["used"]:
+                h2d_s.wait_event(buf["computed"])     # step i-2 has read these inputs
+            for n in names:
+                dev[n].copy_(host[n], non_blocking=True)
+            buf["ready"].record(h2d_s)
+        comp.wait_event(buf["ready"])
+        if buf["used"]:
+            comp.wait_event(buf["returned"])          # step i-2's output has left
         cache_write(pa, b, dev["k_new"], dev["v_new"], dev["slot_mapping"])
-        attention(pa, b, out, dev["q"], dev["block_tables"], dev["seq_lens"],
+        attention(pa, b, buf["out"], dev["q"], dev["block_tables"], dev["seq_lens"],
                   dev["query_start_loc"], ws)
-        out_host.copy_(out, non_blocking=True)
+        buf["computed"].record(comp)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(buf["computed"])
+            buf["out_host"].copy_(buf["out"], non_blocking=True)
+            buf["returned"].record(d2h_s)
+        buf["used"] = True
 
-    for _ in range(5):
-        step()
+    for i in range(5):
+        step(i)
     torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(steps):
-        step()
-    end.record(stream)
+    start.record(comp)
+    h2d_s.wait_event(start)
+    for i in range(steps):
+        step(i)
+    for buf in bufs:
+        comp.wait_event(buf["returned"])
+    end.record(comp)
     torch.cuda.synchronize()
     pa.pa_get_device_error()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = bufs[0]["out_host"].numel() * bufs[0]["out_host"].element_size()
     return start.elapsed_time(end) / steps, h2d, d2h
 
 
@@ -532,7 +569,8 @@ def run_ours(args):
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(args.workload),
                      "kernel": "pa_decode/pa_varlen call (schedule + attention + split-K reduce "
-                               "kernels), CUDA events on the launching stream",
+                               "kernels), CUDA events on the launching stream around "
+                               "every 10th call of the timed steps",
                      "algorithmic_bytes_per_launch": acc["total"],
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6650 GB/s"},

@@ -651,7 +651,8 @@ pa_status pa_rope_reshape_and_cache(void* q, const void* k, const void* v, void*
   // quads of four elements line up with both pair layouts when rot_dim is a
   // multiple of 8; the table rows then start 16-byte aligned if the base is
   const bool vec = rot_dim % 8 == 0 && aligned(cos_sin, 16);
-  const long long parts = vec ? (num_q_heads + 7) / 8 + (num_kv_heads + 7) / 8
+  constexpr int kH = pa::kRopeHeads;
+  const long long parts = vec ? (num_q_heads + kH - 1) / kH + (num_kv_heads + kH - 1) / kH
                               : static_cast<long long>(num_q_heads) + num_kv_heads;
   const long long warps = static_cast<long long>(num_tokens) * parts;
   const long long blocks = (warps * 32 + 255) / 256;

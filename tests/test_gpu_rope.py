@@ -32,7 +32,7 @@ def within_ulp(got: np.ndarray, ref: np.ndarray, dtype: str, what: str):
 
 # (q dtype, head_dim, rot_dim, NeoX pairs, block_size, q heads, KV heads, table
 # offset in floats).  rot_dim a multiple of 8 with an aligned table takes the
-# vector kernel (8-head parts: 24/12 heads make ragged parts); rot_dim 36 or 62,
+# vector kernel (16-head parts: 24 q heads make a ragged second part); rot_dim 36 or 62,
 # or a table 4 bytes off alignment, take the per-element kernel.
 ROPE_CASES = [("bf16", 128, 128, True, 16, 8, 2, 0),
               ("f16", 64, 32, False, 8, 8, 2, 0),
@@ -43,7 +43,8 @@ ROPE_CASES = [("bf16", 128, 128, True, 16, 8, 2, 0),
               ("f32", 64, 56, False, 16, 4, 4, 0),
               ("bf16", 128, 36, True, 16, 8, 2, 0),
               ("f16", 64, 62, False, 8, 8, 4, 0),
-              ("bf16", 128, 128, True, 16, 8, 2, 1)]
+              ("bf16", 128, 128, True, 16, 8, 2, 1),
+              ("bf16", 64, 64, True, 16, 20, 20, 0)]
 
 
 @pytest.mark.parametrize("dtype,d,rot,neox,bs,hq,hkv,offset", ROPE_CASES)
