@@ -614,14 +614,23 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       cm[warp * kRows + r1] = m1;
       cl[warp * kRows + r1] = l1;
     }
+    if constexpr (fp8_direct) {
+      // n-tile t, columns 2q, 2q+1 hold head dims 32q + t and 32q + 16 + t: this
+      // lane has dims 32q .. 32q+31 of rows r0 and r1, stored as eight float4
+      // chunks per row in the swizzled layout (conflict-free; plain offsets put
+      // the four quads of a warp on one bank)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      if constexpr (fp8_direct) {  // n-tile t, columns 2q, 2q+1: head dims 32q + t, 32q + 16 + t
-        co[warp][r0][32 * quad + t] = o[t][0];
-        co[warp][r0][32 * quad + 16 + t] = o[t][1];
-        co[warp][r1][32 * quad + t] = o[t][2];
-        co[warp][r1][32 * quad + 16 + t] = o[t][3];
-      } else {
+      for (int kk = 0; kk < 8; ++kk) {
+        const int h = kk >> 2, t0 = 4 * (kk & 3);
+        const int off = co_swizzled(8 * quad + kk);
+        *reinterpret_cast<float4*>(&co[warp][r0][off]) =
+            make_float4(o[t0][h], o[t0 + 1][h], o[t0 + 2][h], o[t0 + 3][h]);
+        *reinterpret_cast<float4*>(&co[warp][r1][off]) =
+            make_float4(o[t0][2 + h], o[t0 + 1][2 + h], o[t0 + 2][2 + h], o[t0 + 3][2 + h]);
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
         *reinterpret_cast<float2*>(&co[warp][r0][t * 8 + 2 * quad]) =
             make_float2(o[t][0], o[t][1]);
         *reinterpret_cast<float2*>(&co[warp][r1][t * 8 + 2 * quad]) =
@@ -629,7 +638,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       }
     }
     if (!consumers_sync()) return;
-    epilogue<T, D, NCW>(s, u, cm, cl, co, out, w, tid, NCW * 32);
+    epilogue<T, D, NCW, fp8_direct>(s, u, cm, cl, co, out, w, tid, NCW * 32);
     if (!consumers_sync()) return;
   }
 }

@@ -348,11 +348,23 @@ __device__ __forceinline__ void store_row8(const Shape& s, T* __restrict__ out, 
   }
 }
 
-template <typename T, int D, int NW>
+// Float offset, inside a merge-buffer row, of the 4-float chunk `ch` (dims
+// 4ch .. 4ch+3) in the swizzled layout: within each run of 8 chunks (32 dims)
+// the chunk index is XORed with 0, 4, 1, 5 for runs 0..3.  A warp whose lanes
+// (g, q) hold dims 32q .. 32q+31 of rows g and g+8 then stores its run
+// conflict-free with float4 stores at a row stride of D + 8 floats.
+__device__ __forceinline__ int co_swizzled(int ch) {
+  const int run = ch >> 3;
+  const int x = ((run & 1) << 2) | ((run >> 1) & 1);
+  return 4 * ((ch & ~7) | ((ch & 7) ^ x));
+}
+
+template <typename T, int D, int NW, bool kSwizzledCo = false>
 __device__ __forceinline__ void epilogue(const Shape& s, const Unit& u, const float* cm,
                                          const float* cl, const float (*co)[kRows][D + 8],
                                          T* __restrict__ out, const Work& w, int tid,
                                          int nthreads) {
+  static_assert(!kSwizzledCo || D <= 128, "the swizzle covers four runs of 32 dims");
   constexpr int kChunks = D / 8;
   for (int task = tid; task < kRows * kChunks; task += nthreads) {
     const int r = task / kChunks, c = task % kChunks;
@@ -371,8 +383,10 @@ __device__ __forceinline__ void epilogue(const Shape& s, const Unit& u, const fl
     for (int q = 0; q < NW; ++q) {
       const float f = exp2f(cm[q * kRows + r] - mx);
       L += f * cl[q * kRows + r];
-      const float4 a = *reinterpret_cast<const float4*>(&co[q][r][c * 8]);
-      const float4 b = *reinterpret_cast<const float4*>(&co[q][r][c * 8 + 4]);
+      const int oa = kSwizzledCo ? co_swizzled(2 * c) : c * 8;
+      const int ob = kSwizzledCo ? co_swizzled(2 * c + 1) : c * 8 + 4;
+      const float4 a = *reinterpret_cast<const float4*>(&co[q][r][oa]);
+      const float4 b = *reinterpret_cast<const float4*>(&co[q][r][ob]);
       acc[0] += f * a.x; acc[1] += f * a.y; acc[2] += f * a.z; acc[3] += f * a.w;
       acc[4] += f * b.x; acc[5] += f * b.y; acc[6] += f * b.z; acc[7] += f * b.w;
     }
