@@ -127,6 +127,27 @@ pa_status make_map_2d(CUtensorMap* map, const void* base, pa_dtype dt, uint64_t 
   return PA_OK;
 }
 
+// 4-D view of a 16-bit K or V cache of `rows` rows x d elements (rows a
+// multiple of 8): (64 elements of a half, row within a group of 8, half,
+// row group), strides 2 B, d * 2 B, 128 B, 8 * d * 2 B.  A box {64, 8, d/64,
+// groups} lands in shared memory as [group][half][8 rows][128 B], 128 B-swizzled.
+pa_status make_map_kv(CUtensorMap* map, const void* base, pa_dtype dt, uint64_t d,
+                      uint64_t rows, uint32_t groups) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[4] = {64, 8, d / 64, rows / 8};
+  const cuuint64_t strides[3] = {d * 2, 128, 8 * d * 2};
+  const cuuint32_t box[4] = {64, 8, static_cast<cuuint32_t>(d / 64), groups};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (kv) failed: %d", r);
+  return PA_OK;
+}
+
 // 2-D view [rows][inner] of a 1-byte tensor (FP8 codes), box {inner, box_rows};
 // 128-byte rows are 128 B-swizzled (the consumers read them with swizzled
 // 16-byte loads), 64-byte rows are not.
@@ -357,10 +378,10 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
   const int box_rows = a.block_size < pa::kBlock ? a.block_size : pa::kBlock;
   pa_status st = KV8 ? make_map_2d_u8(&tk, a.k_cache, D, rows, box_rows)
-                     : make_map_2d(&tk, a.k_cache, a.dtype, D, rows, box_rows);
+                     : make_map_kv(&tk, a.k_cache, a.dtype, D, rows, box_rows / 8);
   if (st != PA_OK) return st;
   st = KV8 ? make_map_2d_u8(&tv, a.v_cache, D, rows, box_rows)
-           : make_map_2d(&tv, a.v_cache, a.dtype, D, rows, box_rows);
+           : make_map_kv(&tv, a.v_cache, a.dtype, D, rows, box_rows / 8);
   if (st != PA_OK) return st;
   st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.qpt);
   if (st != PA_OK) return st;

@@ -10,10 +10,13 @@
 //   so that the dependent global loads of that lookup never delay the stream.
 // * The TMA warp takes each slot and issues cp.async.bulk.tensor loads of the
 //   tile's query rows and of every 16-key K tile and V tile of the unit --
-//   16 tokens x head_dim, 4 KB each at bf16 x 128; one box of a 16- or
-//   32-token block, or two 8-row boxes of two 8-token blocks -- into a
-//   STAGES-deep ring of shared-memory stages completed on mbarriers.  The tensor maps use 128-byte
-//   swizzling, so the ldmatrix reads below are free of bank conflicts.
+//   16 tokens x head_dim, 4 KB each at bf16 x 128 -- into a STAGES-deep ring
+//   of shared-memory stages completed on mbarriers.  A 16-bit tile lands as
+//   [8-row group][64-dim half][8 rows][128 B]: one 4-D box per tile for 16-
+//   and 32-token blocks, one 3-D box per block for two 8-token blocks (the
+//   count and size of boxes set the achievable bandwidth: 1 KB boxes cap it
+//   near 73% of the copy rate, 4 KB boxes do not).  The tensor maps use
+//   128-byte swizzling, so the ldmatrix reads below are free of bank conflicts.
 // * Consumer warp w takes the unit's blocks w, w+NCW, ...: S = Q K^T (16 tile
 //   rows x 16 tokens, m16n8k16 MMAs, fp32 accumulate), masking of keys past
 //   each row's limit, online softmax in the log2 domain (running max m, sum
@@ -50,6 +53,8 @@ struct MmaLayout {
   static constexpr int kHalves = D / 64;             // 64 16-bit elements = one 128 B swizzle row
   static constexpr int kHalfBytes = kBlock * 128;    // 16 rows x 128 B
   static constexpr int kTileBytes = kHalves * kHalfBytes;          // a 16-bit K or V tile
+  // a 16-bit tile is [2 groups of 8 rows][kHalves][8 rows][128 B]
+  static constexpr int kGroupBytes = kHalves * 8 * 128;
   static constexpr int kKVTileBytes = KV8 ? kBlock * D : kTileBytes;  // ... as loaded
   static constexpr int kStageBytes = 2 * kKVTileBytes;  // K tile then V tile
   static constexpr int kQSlotBytes = kHalves * kRows * 128;
@@ -81,6 +86,12 @@ struct MmaLayout {
 // chunk ch ^ (r % 8).
 __device__ __forceinline__ uint32_t swz(int r, int ch) {
   return static_cast<uint32_t>(r * 128 + ((ch ^ (r & 7)) << 4));
+}
+
+// Byte offset of chunk `ch` of row `r` (0..15), half `h`, in a 16-bit K/V
+// tile laid out [r / 8][h][r % 8][128 B] (group stride `group_bytes`).
+__device__ __forceinline__ uint32_t kv_off(int r, int h, int ch, int group_bytes) {
+  return static_cast<uint32_t>((r >> 3) * group_bytes + h * 1024) + swz(r & 7, ch);
 }
 
 // Two e4m3 codes (low byte first) -> f16x2 (exact).
@@ -305,29 +316,37 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
           break;
         ++issued;
         const uint32_t kdst = sbase + st * L::kStageBytes;
-        // boxes per K or V tile: one per 64-dim half (16-bit), or one of D
-        // bytes (FP8); 16 rows, or 8 rows twice with 8-token blocks
-        constexpr int kBoxes = KV8 ? 1 : L::kHalves;
-        constexpr int kBoxBytes = L::kKVTileBytes / kBoxes;
-        if (s.block_size >= kBlock) {
-          mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
-#pragma unroll
-          for (int h = 0; h < kBoxes; ++h) {
-            tma_load_2d(kdst + h * kBoxBytes, &tm_k, full_bar(st), h * 64, y);
-            tma_load_2d(kdst + L::kKVTileBytes + h * kBoxBytes, &tm_v, full_bar(st), h * 64, y);
+        const uint32_t vdst = kdst + L::kKVTileBytes;
+        if constexpr (KV8) {
+          // one box of D bytes x 16 rows, or of 8 rows twice with 8-token blocks
+          if (s.block_size >= kBlock) {
+            mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
+            tma_load_2d(kdst, &tm_k, full_bar(st), 0, y);
+            tma_load_2d(vdst, &tm_v, full_bar(st), 0, y);
+          } else {
+            const int y1 = meta[ms].y1[jj];
+            mbar_arrive_expect_tx(full_bar(st), y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
+            tma_load_2d(kdst, &tm_k, full_bar(st), 0, y);
+            tma_load_2d(vdst, &tm_v, full_bar(st), 0, y);
+            if (y1 >= 0) {
+              tma_load_2d(kdst + L::kKVTileBytes / 2, &tm_k, full_bar(st), 0, y1);
+              tma_load_2d(vdst + L::kKVTileBytes / 2, &tm_v, full_bar(st), 0, y1);
+            }
           }
-        } else {  // 8-token blocks: rows 0-7 and, if the tile has them, rows 8-15
+        } else if (s.block_size >= kBlock) {
+          // the maps view the cache as (64 dims, 8 rows, half, row group): one
+          // box of 2 row groups is the whole tile
+          mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
+          tma_load_4d(kdst, &tm_k, full_bar(st), 0, 0, 0, y >> 3);
+          tma_load_4d(vdst, &tm_v, full_bar(st), 0, 0, 0, y >> 3);
+        } else {  // 8-token blocks: one row group per block, the second if present
           const int y1 = meta[ms].y1[jj];
           mbar_arrive_expect_tx(full_bar(st), y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
-#pragma unroll
-          for (int h = 0; h < kBoxes; ++h) {
-            tma_load_2d(kdst + h * kBoxBytes, &tm_k, full_bar(st), h * 64, y);
-            tma_load_2d(kdst + L::kKVTileBytes + h * kBoxBytes, &tm_v, full_bar(st), h * 64, y);
-            if (y1 >= 0) {
-              tma_load_2d(kdst + h * kBoxBytes + kBoxBytes / 2, &tm_k, full_bar(st), h * 64, y1);
-              tma_load_2d(kdst + L::kKVTileBytes + h * kBoxBytes + kBoxBytes / 2, &tm_v,
-                          full_bar(st), h * 64, y1);
-            }
+          tma_load_4d(kdst, &tm_k, full_bar(st), 0, 0, 0, y >> 3);
+          tma_load_4d(vdst, &tm_v, full_bar(st), 0, 0, 0, y >> 3);
+          if (y1 >= 0) {
+            tma_load_4d(kdst + L::kGroupBytes, &tm_k, full_bar(st), 0, 0, 0, y1 >> 3);
+            tma_load_4d(vdst + L::kGroupBytes, &tm_v, full_bar(st), 0, 0, 0, y1 >> 3);
           }
         }
       }
@@ -484,7 +503,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
         for (int kk = 0; kk < KSTEPS; ++kk) {
           uint32_t b0, b1, b2, b3;
           const int ch = (kk & 3) * 2 + (mi & 1);
-          ldsm_x4(kb + (kk >> 2) * L::kHalfBytes + swz(tk, ch), b0, b1, b2, b3);
+          ldsm_x4(kb + kv_off(tk, kk >> 2, ch, L::kGroupBytes), b0, b1, b2, b3);
           mma_16816<MT>(sacc[0], qa[kk], b0, b1);
           mma_16816<MT>(sacc[1], qa[kk], b2, b3);
         }
@@ -575,7 +594,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
           for (int jj = 0; jj < KSTEPS; ++jj) {
             uint32_t b0, b1, b2, b3;
             const int ch = (jj & 3) * 2 + (mi >> 1);
-            ldsm_x4_t(vb + (jj >> 2) * L::kHalfBytes + swz(tk, ch), b0, b1, b2, b3);
+            ldsm_x4_t(vb + kv_off(tk, jj >> 2, ch, L::kGroupBytes), b0, b1, b2, b3);
             if (masked) {
               b0 &= vm0;
               b1 &= vm1;
