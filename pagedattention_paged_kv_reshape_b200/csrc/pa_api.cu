@@ -109,24 +109,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D view [rows][inner] of a 16-bit tensor, box {64, box_rows}, 128 B swizzle.
-pa_status make_map_2d(CUtensorMap* map, const void* base, pa_dtype dt, uint64_t inner,
-                      uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {64, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                        2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (2d) failed: %d", r);
-  return PA_OK;
-}
-
 // 4-D view of a 16-bit K or V cache of `rows` rows x d elements (rows a
 // multiple of 8): (64 elements of a half, row within a group of 8, half,
 // row group), strides 2 B, d * 2 B, 128 B, 8 * d * 2 B.  A box {64, 8, d/64,
@@ -406,9 +388,9 @@ pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   // one box = 16 cache rows, or one whole 8-token block
   const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
   const int box_rows = a.block_size < pa::kBlock ? a.block_size : pa::kBlock;
-  pa_status st = make_map_2d(&tk, a.k_cache, a.dtype, D, rows, box_rows);
+  pa_status st = make_map_kv(&tk, a.k_cache, a.dtype, D, rows, box_rows / 8);
   if (st != PA_OK) return st;
-  st = make_map_2d(&tv, a.v_cache, a.dtype, D, rows, box_rows);
+  st = make_map_kv(&tv, a.v_cache, a.dtype, D, rows, box_rows / 8);
   if (st != PA_OK) return st;
   st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.chunk_qt);
   if (st != PA_OK) return st;

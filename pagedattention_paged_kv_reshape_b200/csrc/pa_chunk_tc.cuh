@@ -9,12 +9,13 @@
 // * work item = (chunk row, tile of 128/gs query tokens x gs query heads =
 //   128 tile rows, KV head slice); a persistent grid walks the items listed
 //   by the prep kernel, each CTA its items one after another;
-// * a load warp brings Q (one 3-D TMA box, two buffers) and K, V (one TMA box
-//   of 16 rows per 16 keys, two of 8 rows with 8-token blocks; K and V
-//   rings of 128-key tiles) into shared memory
-//   with 128-byte swizzling, which is exactly the canonical K-major layout
-//   (Q, K) and MN-major layout (V) the tcgen05 shared-memory descriptors
-//   describe.  It walks the CTA's tiles as one sequence, K one tile ahead of
+// * a load warp brings Q (one 3-D TMA box per 64-dim half, two buffers) and
+//   K, V (K and V rings of 128-key tiles; one 4-D box of all halves per 16
+//   keys, or per 8-token block) into shared memory with 128-byte swizzling.
+//   Q lands as [half][128 rows][128 B], K and V as [8-key group][half][8
+//   rows][128 B]: canonical K-major (Q, K) and MN-major (V) layouts for the
+//   tcgen05 shared-memory descriptors, with the 8-row group stride as the
+//   descriptors' stride byte offset.  It walks the CTA's tiles as one sequence, K one tile ahead of
 //   V, runs ahead of the tensor core as far as the rings allow, fetches item
 //   metadata one to two items ahead, and hands it to the other warps through
 //   shared memory;
@@ -62,6 +63,7 @@ struct TcLayout {
   static constexpr int kHalves = D / 64;            // 128-byte swizzle rows per token row
   static constexpr int kHalfBytes = 128 * 128;      // 128 rows x 128 B
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // one Q, K or V tile
+  static constexpr int kGroupBytes = kHalves * 1024;        // 8 keys of a K or V tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQStages * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
@@ -236,12 +238,9 @@ __global__ void __launch_bounds__(320, 1)
                                 static_cast<uint32_t>(p.nb * L::kHalves * box_rows * 128));
       }
       r = __shfl_sync(0xffffffffu, r, 0);
-      if (r && lane < p.nb) {
-#pragma unroll
-        for (int h = 0; h < L::kHalves; ++h)
-          tma_load_2d(v_smem(vs) + h * L::kHalfBytes + lane * box_rows * 128, &tm_v, vfull(vs),
-                      h * 64, p.y);
-      }
+      if (r && lane < p.nb)
+        tma_load_4d(v_smem(vs) + lane * (box_rows / 8) * L::kGroupBytes, &tm_v, vfull(vs), 0, 0,
+                    0, p.y >> 3);
       return r;
     };
     int2 ent1 = entry_of(1);
@@ -275,12 +274,9 @@ __global__ void __launch_bounds__(320, 1)
         }
         ok = __shfl_sync(0xffffffffu, r, 0);
         if (!ok) break;
-        if (lane < nb) {
-#pragma unroll
-          for (int h = 0; h < L::kHalves; ++h)
-            tma_load_2d(k_smem(ks) + h * L::kHalfBytes + lane * box_rows * 128, &tm_k, kfull(ks),
-                        h * 64, y);
-        }
+        if (lane < nb)
+          tma_load_4d(k_smem(ks) + lane * (box_rows / 8) * L::kGroupBytes, &tm_k, kfull(ks), 0, 0,
+                      0, y >> 3);
         // queue this tile's V; issue the previous tile's
         if (npend == 0) {
           va = Pending{y, nb, gt};
@@ -343,9 +339,10 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
-            umma_ss(t_s(gt & 1), smem_desc_sw128(q_smem(qb) + off, 16, 1024),
-                    smem_desc_sw128(k_smem(ks) + off, 16, 1024), kIdescS, kk > 0);
+            const uint32_t qoff = (kk >> 2) * L::kHalfBytes + (kk & 3) * 32;
+            const uint32_t koff = (kk >> 2) * 1024 + (kk & 3) * 32;
+            umma_ss(t_s(gt & 1), smem_desc_sw128(q_smem(qb) + qoff, 16, 1024),
+                    smem_desc_sw128(k_smem(ks) + koff, 16, L::kGroupBytes), kIdescS, kk > 0);
           }
           umma_commit(sfull(gt & 1));
           umma_commit(kempty(ks));
@@ -370,8 +367,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int ch = lane; ch < nchunks; ch += 32) {
           const int row = valid + ch / (L::kHalves * 8);
           const int h = (ch / 8) % L::kHalves;
-          *reinterpret_cast<uint4*>(smem + L::kOffV + vs * L::kTileBytes + h * L::kHalfBytes +
-                                    row * 128 + (ch % 8) * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(smem + L::kOffV + vs * L::kTileBytes +
+                                    (row >> 3) * L::kGroupBytes + h * 1024 + (row & 7) * 128 +
+                                    (ch % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
@@ -381,8 +379,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < kTcKeys / 16; ++kk) {
           umma_ts(t_o, t_p(b) + kk * 8,
-                  smem_desc_sw128(v_smem(vs) + kk * 2048, L::kHalfBytes, 1024), kIdescPV,
-                  (c.t > 0 || kk > 0) ? 1u : 0u);
+                  smem_desc_sw128(v_smem(vs) + kk * 2 * L::kGroupBytes, 1024, L::kGroupBytes),
+                  kIdescPV, (c.t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(pfree(b));
         umma_commit(vempty(vs));
