@@ -439,13 +439,15 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
     }
   }
   if (p.s.p_stride <= 1) return PA_OK;
-  // one CTA per (request, 16-token slice, 8 heads) of the rows the attention kernels split
+  // one CTA per (request, 16-token slice, 8 heads) of the rows the attention
+  // kernels split; with 16 or more partitions per row, one per query head
+  const bool wide = p.s.p_stride >= 16;
   int max_q = a.qsl ? a.max_query_len : 1;
   if (p.s.chunk_qt > 0 && max_q >= p.s.chunk_qt) max_q = p.s.chunk_qt - 1;
   const int slices = (max_q + pa::kReduceTokens - 1) / pa::kReduceTokens;
   const dim3 grid(static_cast<unsigned>(a.num_seqs),
                   static_cast<unsigned>(slices < 65535 ? slices : 65535),
-                  static_cast<unsigned>((a.num_q_heads + 7) / 8));
+                  static_cast<unsigned>(wide ? a.num_q_heads : (a.num_q_heads + 7) / 8));
   if (grid.y == 0) return PA_OK;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -456,14 +458,17 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = a.head_dim == 256
-          ? cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 256>, p.s, a.qsl, a.seq_lens, w,
-                               static_cast<T*>(a.out))
-      : a.head_dim == 128
-          ? cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 128>, p.s, a.qsl, a.seq_lens, w,
-                               static_cast<T*>(a.out))
-          : cudaLaunchKernelEx(&cfg, pa::reduce_kernel<T, 64>, p.s, a.qsl, a.seq_lens, w,
-                               static_cast<T*>(a.out));
+  auto launch = [&](auto kern) {
+    return cudaLaunchKernelEx(&cfg, kern, p.s, a.qsl, a.seq_lens, w, static_cast<T*>(a.out));
+  };
+  if (wide)
+    e = a.head_dim == 256   ? launch(pa::reduce_wide_kernel<T, 256>)
+        : a.head_dim == 128 ? launch(pa::reduce_wide_kernel<T, 128>)
+                            : launch(pa::reduce_wide_kernel<T, 64>);
+  else
+    e = a.head_dim == 256   ? launch(pa::reduce_kernel<T, 256>)
+        : a.head_dim == 128 ? launch(pa::reduce_kernel<T, 128>)
+                            : launch(pa::reduce_kernel<T, 64>);
   if (e != cudaSuccess) return cuda_fail(e, "reduce kernel launch");
   return PA_OK;
 }

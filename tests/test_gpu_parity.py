@@ -260,6 +260,37 @@ def test_head_dim_256_refuses_cuda_core_paths():
     assert e.value.status == pa.Status.UNSUPPORTED
 
 
+# Batches whose longest row has 16 or more 512-key partitions take the wide
+# split-K reduce (one CTA per query head, warps splitting the partitions);
+# short rows of the same batch go through it too.
+WIDE_REDUCE_CASES = [
+    # (rows (seq_len, q_len), hq, hkv, d, dtype, kv cache dtype, path)
+    ([(9000, 1), (17, 1), (8200, 1), (600, 1), (16385, 1)], 8, 2, 128, "bf16", None, "auto"),
+    ([(8193, 1), (3, 1), (12000, 1)], 4, 4, 64, "f32", None, "simt"),
+    ([(9100, 1), (530, 1)], 8, 4, 256, "bf16", None, "auto"),
+    ([(9000, 37), (1, 1), (8300, 1), (700, 200)], 8, 2, 128, "f16", None, "mma"),
+    ([(10000, 1), (45, 1), (8500, 9)], 16, 2, 128, "bf16", "fp8", "auto"),
+]
+
+
+@pytest.mark.parametrize("case", range(len(WIDE_REDUCE_CASES)))
+def test_wide_split_k_reduce_matches_oracle(case):
+    rows, hq, hkv, d, dtype, kv_dtype, path = WIDE_REDUCE_CASES[case]
+    if path == "simt":
+        pa.pa_set_path(pa.Path.SIMT)
+    elif path == "mma":
+        pa.pa_set_path(pa.Path.MMA)
+    extra = {"kv_dtype": kv_dtype} if kv_dtype else {}
+    b = W.build_batch([W.Request(L, q) for L, q in rows], num_q_heads=hq, num_kv_heads=hkv,
+                      head_dim=d, dtype=dtype, seed=900 + case, device=DEV, pool_factor=1.2,
+                      **extra)
+    assert math.ceil(b.max_seq_len / 512) >= 16
+    varlen = any(q_ != 1 for _, q_ in rows)
+    out, _, _ = gpu_step(b, varlen=varlen)
+    ref, _, _ = oracle_step(b, varlen=varlen)
+    assert_close(out, ref, dtype, f"wide reduce case {case} ({path})")
+
+
 def test_chunk_kernel_agrees_with_decode_kernel_tiles():
     """The tcgen05 chunk tiles and the decode kernel's 16-row tiles compute the
     same rows; both are within tolerance of each other as well as the oracle."""
