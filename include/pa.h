@@ -154,6 +154,10 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
  * Each result is computed in fp32 and rounded once to `dtype`.  A position
  * outside [0, max_position) leaves that token's q and cache rows untouched
  * and is recorded as PA_ERR_DEVICE_BOUNDS; slots as for pa_reshape_and_cache.
+ * rot_dim must be even and at most head_dim (else PA_ERR_INVALID_ARG).  With
+ * rot_dim a multiple of 8 and cos_sin 16-byte aligned the call runs a
+ * vectorised kernel; other shapes run a per-element one with the same
+ * arithmetic.
  */
 pa_status pa_rope_reshape_and_cache(void* q, const void* k, const void* v, void* k_cache,
                                     void* v_cache, const int32_t* slot_mapping,
