@@ -299,10 +299,11 @@ def launches_per_step(b) -> int:
 
 
 def time_steps(torch, pa, b, steps, warmup, sample_every=10):
-    """Device time of ``steps`` steps and the mean duration of the attention
-    call, taken with events around the call of every ``sample_every``-th step
-    inside the same timed region (events around every call cost ~2% of the
-    step time on B200; one in ten costs nothing measurable)."""
+    """Device time of ``steps`` steps, the mean duration of the attention call
+    and of the cache write, taken with events around both calls of every
+    ``sample_every``-th step inside the same timed region (events around every
+    call cost ~2% of the step time on B200; one in ten costs nothing
+    measurable).  Returns (total_ms, attention_ms, cache_write_ms, out)."""
     out = torch.empty_like(b.q)
     ws = workspace_for(pa, b)
     step, attend = make_step(pa, b, out, ws)
@@ -319,18 +320,20 @@ def time_steps(torch, pa, b, steps, warmup, sample_every=10):
         if i % every:
             step()
             continue
+        ew, e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        ew.record(stream)
         cache_write(pa, b, b.k_new, b.v_new, b.slot_mapping)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         attend()
         e1.record(stream)
-        ev.append((e0, e1))
+        ev.append((ew, e0, e1))
     end.record(stream)
     torch.cuda.synchronize()
     pa.pa_get_device_error()
     total_ms = start.elapsed_time(end)
-    attn_ms = statistics.fmean(e0.elapsed_time(e1) for e0, e1 in ev)
-    return total_ms, attn_ms, out
+    attn_ms = statistics.fmean(e0.elapsed_time(e1) for _, e0, e1 in ev)
+    write_ms = statistics.fmean(ew.elapsed_time(e0) for ew, e0, _ in ev)
+    return total_ms, attn_ms, write_ms, out
 
 
 def time_e2e(torch, pa, b, steps):
@@ -528,7 +531,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    total_ms, attn_ms, _ = time_steps(torch, pa, b, args.steps, args.warmup)
+    total_ms, attn_ms, write_ms, _ = time_steps(torch, pa, b, args.steps, args.warmup)
     clocks = sampler.stop() if sampler else None
 
     max_ms, value, tok_per_s = combine_over_ranks(total_ms, step_bytes * args.steps,
@@ -576,6 +579,10 @@ def run_ours(args):
                      if peak_kind == "measured" else "fallback 6650 GB/s"},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e.item(), 5)},
+        "cache_write": {"ms": round(write_ms, 5), "bytes": A.reshape_bytes(b),
+                        "gbs": round(A.reshape_bytes(b) / (write_ms / 1e3) / 1e9, 1),
+                        "note": "pa_reshape_and_cache of the step's new rows, CUDA events "
+                                "around every 10th call of the timed steps"},
         "gpu_launches": launches_per_step(b) * args.steps,
         "clocks": clocks,
     }
@@ -591,13 +598,15 @@ def run_ours(args):
             torch.cuda.empty_cache()
             b = W.make_config(name, seed=args.seed + rank, device=dev)
             a2 = A.attention_bytes(b)
-            tot, attn, _ = time_steps(torch, pa, b, args.per_config_steps, max(3, args.warmup // 4))
+            tot, attn, wr, _ = time_steps(torch, pa, b, args.per_config_steps,
+                                          max(3, args.warmup // 4))
             sb = a2["total"] + A.reshape_bytes(b)
             ent = {"step_gbs": round(sb / (tot / args.per_config_steps / 1e3) / 1e9, 1),
                    "attention_gbs": round(a2["total"] / (attn / 1e3) / 1e9, 1),
                    "pct_of_hbm_peak": round(100 * a2["total"] / (attn / 1e3) / 1e9 / peak, 1),
                    "ms_per_step": round(tot / args.per_config_steps, 4),
                    "attention_ms": round(attn, 4),
+                   "cache_write_ms": round(wr, 4),
                    "tokens_per_s": round(b.total_q / (tot / args.per_config_steps / 1e3), 1)}
             if name == "mixed_2048":
                 ent["unique_vs_logical_kv"] = [a2["kv_unique"], a2["kv_logical"]]
@@ -606,7 +615,8 @@ def run_ours(args):
                 tflops = A.chunk_flops(b) / (attn / 1e3) / 1e12
                 ent = {"chunk_tflops": round(tflops, 1),
                        "pct_of_bf16_peak": round(100 * tflops / tensor_peak, 1),
-                       "attention_ms": round(attn, 4), "chunk_gflop": round(A.chunk_flops(b) / 1e9, 1),
+                       "attention_ms": round(attn, 4), "cache_write_ms": round(wr, 4),
+                       "chunk_gflop": round(A.chunk_flops(b) / 1e9, 1),
                        "peak_kind": "measured bf16_tflops (burst)",
                        "tokens_per_s": round(b.total_q / (attn / 1e3), 1)}
             per[name] = ent
