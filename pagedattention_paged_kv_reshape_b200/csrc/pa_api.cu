@@ -408,9 +408,8 @@ pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
 template <typename T>
 pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   const pa::Work w = carve(a.workspace, p);
-  pa::schedule_kernel<T><<<1, 1024, 0, a.stream>>>(p.s, a.qsl, a.seq_lens, w,
-                                                   static_cast<T*>(a.out));
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(pa::schedule_kernel<T>, 1, 1024, 0, a.stream, p.s, a.qsl,
+                             a.seq_lens, w, static_cast<T*>(a.out));
   if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
   pa_status st;
   const bool d128 = a.head_dim == 128;
@@ -569,12 +568,12 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void
   const long long warps = static_cast<long long>(num_tokens) * num_kv_heads;
   const long long blocks = (warps * 32 + 255) / 256;
   if (blocks > 0x7fffffffLL) return fail(PA_ERR_UNSUPPORTED, "too many tokens");
-  pa::reshape_and_cache_kernel<<<static_cast<unsigned>(blocks), 256, 0,
-                                 static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, row_vecs, block_size,
+  const cudaError_t e = launch_pdl(
+      pa::reshape_and_cache_kernel, static_cast<unsigned>(blocks), 256, 0,
+      static_cast<cudaStream_t>(stream), static_cast<const uint4*>(k),
+      static_cast<const uint4*>(v), static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+      slot_mapping, num_tokens, num_kv_heads, row_vecs, block_size,
       static_cast<long long>(num_blocks) * block_size);
-  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache launch");
   return PA_OK;
 }

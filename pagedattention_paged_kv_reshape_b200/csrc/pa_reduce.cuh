@@ -32,6 +32,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) reduce_kernel(Shape s, const int* __restrict__ qsl,
                                                      const int* __restrict__ seq_lens, Work w,
                                                      T* __restrict__ out) {
+  // the next kernel on the stream may be scheduled now; it waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kPer = D / 32;  // dims per lane
   constexpr int kUnroll = 8;
@@ -120,6 +122,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) reduce_wide_kernel(Shape s, const int* __restrict__ qsl,
                                                           const int* __restrict__ seq_lens,
                                                           Work w, T* __restrict__ out) {
+  // the next kernel on the stream may be scheduled now; it waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kPer = D / 32;  // dims per lane
   constexpr int kWarps = 8, kUnroll = 8;

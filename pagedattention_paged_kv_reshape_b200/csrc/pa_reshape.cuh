@@ -21,6 +21,10 @@ __global__ void __launch_bounds__(256)
                              const int* __restrict__ slot_mapping, int num_tokens,
                              int num_kv_heads, int row_vecs, int block_size,
                              long long num_slots) {
+  // launched with programmatic dependent launch: let the next kernel be
+  // scheduled, and touch memory only once the previous grid is done
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= static_cast<long long>(num_tokens) * num_kv_heads) return;

@@ -243,6 +243,9 @@ __global__ void __launch_bounds__(1024) schedule_kernel(Shape s, const int* __re
                                                         const int* __restrict__ seq_lens,
                                                         Work w, T* __restrict__ out) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // launched behind the cache write with programmatic dependent launch: the
+  // workspace and the rows are touched only after the previous grid is done
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int warp_tot[2][32];
   __shared__ int carry_s[2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
