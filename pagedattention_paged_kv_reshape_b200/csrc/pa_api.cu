@@ -608,23 +608,15 @@ pa_status pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, 
   const unsigned g = static_cast<unsigned>(blocks);
   auto* kc = static_cast<uint8_t*>(k_cache);
   auto* vc = static_cast<uint8_t*>(v_cache);
-  switch (dtype) {
-    case PA_BF16:
-      pa::reshape_and_cache_fp8_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), kc, vc,
-          slot_mapping, k_scale, v_scale, num_tokens, num_kv_heads, head_dim, block_size, slots);
-      break;
-    case PA_F16:
-      pa::reshape_and_cache_fp8_kernel<__half><<<g, 256, 0, st>>>(
-          static_cast<const __half*>(k), static_cast<const __half*>(v), kc, vc, slot_mapping,
-          k_scale, v_scale, num_tokens, num_kv_heads, head_dim, block_size, slots);
-      break;
-    default:
-      pa::reshape_and_cache_fp8_kernel<float><<<g, 256, 0, st>>>(
-          static_cast<const float*>(k), static_cast<const float*>(v), kc, vc, slot_mapping,
-          k_scale, v_scale, num_tokens, num_kv_heads, head_dim, block_size, slots);
-  }
-  const cudaError_t e = cudaGetLastError();
+  auto launch = [&](auto* tag) {
+    using T = std::remove_pointer_t<decltype(tag)>;
+    return launch_pdl(pa::reshape_and_cache_fp8_kernel<T>, g, 256, 0, st,
+                      static_cast<const T*>(k), static_cast<const T*>(v), kc, vc, slot_mapping,
+                      k_scale, v_scale, num_tokens, num_kv_heads, head_dim, block_size, slots);
+  };
+  const cudaError_t e = dtype == PA_BF16 ? launch(static_cast<__nv_bfloat16*>(nullptr))
+                        : dtype == PA_F16 ? launch(static_cast<__half*>(nullptr))
+                                          : launch(static_cast<float*>(nullptr));
   if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache_fp8 launch");
   return PA_OK;
 }
@@ -670,23 +662,15 @@ pa_status pa_rope_reshape_and_cache(void* q, const void* k, const void* v, void*
   auto launch = [&](auto* tag) {
     using T = std::remove_pointer_t<decltype(tag)>;
     auto kern = vec ? pa::rope_reshape_and_cache_vec_kernel<T> : pa::rope_reshape_and_cache_kernel<T>;
-    kern<<<g, 256, 0, st>>>(static_cast<T*>(q), static_cast<const T*>(k),
-                            static_cast<const T*>(v), static_cast<T*>(k_cache),
-                            static_cast<T*>(v_cache), slot_mapping, positions, cos_sin,
-                            max_position, rot_dim, neox != 0, num_tokens, num_q_heads,
-                            num_kv_heads, head_dim, block_size, slots);
+    return launch_pdl(kern, g, 256, 0, st, static_cast<T*>(q), static_cast<const T*>(k),
+                      static_cast<const T*>(v), static_cast<T*>(k_cache),
+                      static_cast<T*>(v_cache), slot_mapping, positions, cos_sin, max_position,
+                      rot_dim, neox != 0, num_tokens, num_q_heads, num_kv_heads, head_dim,
+                      block_size, slots);
   };
-  switch (dtype) {
-    case PA_BF16:
-      launch(static_cast<__nv_bfloat16*>(nullptr));
-      break;
-    case PA_F16:
-      launch(static_cast<__half*>(nullptr));
-      break;
-    default:
-      launch(static_cast<float*>(nullptr));
-  }
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = dtype == PA_BF16 ? launch(static_cast<__nv_bfloat16*>(nullptr))
+                        : dtype == PA_F16 ? launch(static_cast<__half*>(nullptr))
+                                          : launch(static_cast<float*>(nullptr));
   if (e != cudaSuccess) return cuda_fail(e, "rope_reshape_and_cache launch");
   return PA_OK;
 }

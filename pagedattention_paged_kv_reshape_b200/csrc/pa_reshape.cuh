@@ -62,6 +62,10 @@ __global__ void __launch_bounds__(256)
                                  const float* __restrict__ v_scale, int num_tokens,
                                  int num_kv_heads, int head_dim, int block_size,
                                  long long num_slots) {
+  // launched with programmatic dependent launch: let the next kernel be
+  // scheduled, and touch memory only once the previous grid is done
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= static_cast<long long>(num_tokens) * num_kv_heads) return;
@@ -109,6 +113,10 @@ __global__ void __launch_bounds__(256)
                                   int rot_dim, bool neox, int num_tokens, int num_q_heads,
                                   int num_kv_heads, int head_dim, int block_size,
                                   long long num_slots) {
+  // launched with programmatic dependent launch: let the next kernel be
+  // scheduled, and touch memory only once the previous grid is done
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int heads = num_q_heads + num_kv_heads;
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -217,6 +225,10 @@ __global__ void __launch_bounds__(256)
                                       int rot_dim, bool neox, int num_tokens, int num_q_heads,
                                       int num_kv_heads, int head_dim, int block_size,
                                       long long num_slots) {
+  // launched with programmatic dependent launch: let the next kernel be
+  // scheduled, and touch memory only once the previous grid is done
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   using Q = Quad<T>;
   using Raw = typename Q::Raw;
   constexpr int kHeads = kRopeHeads, kBatch = PA_ROPE_BATCH;
