@@ -106,7 +106,10 @@ typedef enum {
   PA_PATH_AUTO = 0,
   PA_PATH_SIMT = 1,     /* CUDA-core kernel, plain vector loads (any dtype) */
   PA_PATH_MMA = 2,      /* TMA bulk-tensor loads + warp-level bf16/f16 tensor-core MMA */
-  PA_PATH_TCGEN05 = 3   /* as PA_PATH_MMA, with prefill chunks on tcgen05/TMEM tiles */
+  PA_PATH_TCGEN05 = 3,  /* as PA_PATH_MMA, with prefill chunks on tcgen05/TMEM tiles */
+  PA_PATH_TCGEN05_PAIRS = 4  /* as PA_PATH_TCGEN05, chunk items of two query tiles
+                                sharing each K/V tile (slower than PA_PATH_TCGEN05 on
+                                B200 as measured; never chosen by PA_PATH_AUTO) */
 } pa_path;
 
 /*

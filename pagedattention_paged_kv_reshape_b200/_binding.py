@@ -37,6 +37,7 @@ class Path(enum.IntEnum):
     SIMT = 1
     MMA = 2
     TCGEN05 = 3
+    TCGEN05_PAIRS = 4
 
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}

@@ -16,8 +16,10 @@
 #include "pa_attn_mma.cuh"
 #include "pa_attn_simt.cuh"
 #include "pa_blocks.cuh"
+#include "pa_chunk_pair.cuh"
 #include "pa_chunk_tc.cuh"
 #include "pa_reduce.cuh"
+
 #include "pa_reshape.cuh"
 #include "pa_sched.cuh"
 
@@ -232,6 +234,7 @@ Plan make_plan(int num_seqs, int total_q, int hq, int hkv, int d, int max_len, b
   s.p_stride = max_len > 0 ? (max_len + pa::kPart - 1) / pa::kPart : 1;
   s.chunk_qt = 0;
   s.chunk_cap = 0;
+  s.chunk_span = 0;
   const size_t rows = static_cast<size_t>(num_seqs) + 1;
   p.off_row_a = sizeof(pa::Sched);
   p.off_row_b = p.off_row_a + rows * 4;
@@ -405,6 +408,34 @@ pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   return PA_OK;
 }
 
+template <typename T, int D>
+pa_status launch_chunk_pair(const AttnArgs& a, const Plan& p, const pa::Work& w) {
+  using L = pa::TcPairLayout<D>;
+  auto kern = pa::chunk_pair_kernel<T, D>;
+  int occ = 0;
+  cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk pair kernel set-up");
+  CUtensorMap tk, tv, tq;
+  // one box = 16 cache rows, or one whole 8-token block
+  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
+  const int box_rows = a.block_size < pa::kBlock ? a.block_size : pa::kBlock;
+  pa_status st = make_map_kv(&tk, a.k_cache, a.dtype, D, rows, box_rows / 8);
+  if (st != PA_OK) return st;
+  st = make_map_kv(&tv, a.v_cache, a.dtype, D, rows, box_rows / 8);
+  if (st != PA_OK) return st;
+  st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.chunk_qt);
+  if (st != PA_OK) return st;
+  long long grid = sm_count();
+  const long long items = p.chunk_cap * a.num_kv_heads * p.s.ns;
+  if (items < grid) grid = items;
+  if (grid < 1) grid = 1;
+  e = launch_pdl(kern, static_cast<unsigned>(grid), L::kThreads, L::kSmem, a.stream, tk, tv, tq,
+                 p.s, static_cast<T*>(a.out), a.block_tables, a.qsl, a.seq_lens, w,
+                 static_cast<float>(a.scale * M_LOG2E));
+  if (e != cudaSuccess) return cuda_fail(e, "chunk pair kernel launch");
+  return PA_OK;
+}
+
 template <typename T>
 pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   const pa::Work w = carve(a.workspace, p);
@@ -433,7 +464,11 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   if (st != PA_OK) return st;
   if constexpr (sizeof(T) == 2) {
     if (p.s.chunk_qt > 0) {
-      st = a.head_dim == 128 ? launch_chunk<T, 128>(a, p, w) : launch_chunk<T, 64>(a, p, w);
+      if (p.s.chunk_span > p.s.chunk_qt)
+        st = a.head_dim == 128 ? launch_chunk_pair<T, 128>(a, p, w)
+                               : launch_chunk_pair<T, 64>(a, p, w);
+      else
+        st = a.head_dim == 128 ? launch_chunk<T, 128>(a, p, w) : launch_chunk<T, 64>(a, p, w);
       if (st != PA_OK) return st;
     }
   }
@@ -495,7 +530,7 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
     return fail(PA_ERR_INVALID_ARG, "bad k_scale / v_scale pointer");
   const int path = g_path.load();
   const bool sixteen = a.dtype != PA_F32;
-  if (path == PA_PATH_MMA || path == PA_PATH_TCGEN05) {
+  if (path == PA_PATH_MMA || path == PA_PATH_TCGEN05 || path == PA_PATH_TCGEN05_PAIRS) {
     if (!sixteen)
       return fail(PA_ERR_UNSUPPORTED, "tensor-core path needs bf16 or f16 (got fp32)");
   }
@@ -510,6 +545,8 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
                      ? p.chunk_qt
                      : 0;
   p.s.chunk_cap = static_cast<int>(p.chunk_cap);
+  // one query tile per chunk item, or two with PA_PATH_TCGEN05_PAIRS
+  p.s.chunk_span = path == PA_PATH_TCGEN05_PAIRS ? 2 * p.s.chunk_qt : p.s.chunk_qt;
   switch (a.dtype) {
     case PA_BF16: return run_typed<__nv_bfloat16>(a, p, use_mma);
     case PA_F16: return run_typed<__half>(a, p, use_mma);

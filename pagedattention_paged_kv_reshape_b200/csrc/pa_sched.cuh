@@ -49,6 +49,8 @@ struct Shape {
   int chunk_qt;     // > 0: rows with q_len >= chunk_qt go to the tcgen05 chunk kernel
                     // as tiles of chunk_qt query tokens (128 / gs)
   int chunk_cap;    // capacity of the chunk-tile list
+  int chunk_span;   // query tokens per chunk-list entry: chunk_qt, or 2 chunk_qt when
+                    // the chunk kernel takes two tiles per item
 };
 
 // Schedule block at the start of the workspace.
@@ -264,10 +266,10 @@ __global__ void __launch_bounds__(1024) schedule_kernel(Shape s, const int* __re
       if (!ri.ok) report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, r, ri.seq_len);
       row_units(s, ri, va, vb);
       if (ri.ok && is_chunk_row(s, ri)) {
-        const int n = ceil_div(ri.q_len, s.chunk_qt);
+        const int n = ceil_div(ri.q_len, s.chunk_span);
         const int at = atomicAdd(&w.sched->chunk_count, n);
         if (at + n <= s.chunk_cap) {
-          for (int j = 0; j < n; ++j) w.chunk_list[at + j] = make_int2(r, j * s.chunk_qt);
+          for (int j = 0; j < n; ++j) w.chunk_list[at + j] = make_int2(r, j * s.chunk_span);
         } else {  // rows overlap in query_start_loc: more tiles than tokens allow
           report_error(PA_ERR_DEVICE_BOUNDS, kWhereRowMeta, r, at + n);
         }

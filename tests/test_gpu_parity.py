@@ -156,16 +156,16 @@ VARLEN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["auto", "mma", "simt"])
+@pytest.mark.parametrize("path", ["auto", "mma", "simt", "pairs"])
 @pytest.mark.parametrize("case", range(len(VARLEN_CASES)))
 def test_varlen_matches_oracle(case, path):
     rows, hq, hkv, d, dtype = VARLEN_CASES[case]
     if path == "simt":
         pa.pa_set_path(pa.Path.SIMT)
-    elif path == "mma":
+    elif path in ("mma", "pairs"):
         if dtype == "f32":
             pytest.skip("tensor-core paths need 16-bit inputs")
-        pa.pa_set_path(pa.Path.MMA)
+        pa.pa_set_path(pa.Path.MMA if path == "mma" else pa.Path.TCGEN05_PAIRS)
     b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
                       head_dim=d, dtype=dtype, seed=100 + case, device=DEV, pool_factor=1.2)
     out, _, _ = gpu_step(b, varlen=True)
@@ -202,16 +202,16 @@ BLOCK_SIZE_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["auto", "mma", "simt"])
+@pytest.mark.parametrize("path", ["auto", "mma", "simt", "pairs"])
 @pytest.mark.parametrize("case", range(len(BLOCK_SIZE_CASES)))
 def test_block_sizes_match_oracle(case, path):
     rows, hq, hkv, d, dtype, bs = BLOCK_SIZE_CASES[case]
     if path == "simt":
         pa.pa_set_path(pa.Path.SIMT)
-    elif path == "mma":
+    elif path in ("mma", "pairs"):
         if dtype == "f32":
             pytest.skip("tensor-core paths need 16-bit inputs")
-        pa.pa_set_path(pa.Path.MMA)
+        pa.pa_set_path(pa.Path.MMA if path == "mma" else pa.Path.TCGEN05_PAIRS)
     b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
                       head_dim=d, dtype=dtype, seed=300 + case, device=DEV, pool_factor=1.2,
                       block_size=bs)
@@ -303,6 +303,10 @@ def test_chunk_kernel_agrees_with_decode_kernel_tiles():
     mma = gpu_attention(b, kc, vc, varlen=True)
     assert_close(tc, f64(mma), "bf16", "tcgen05 vs mma tiles")
     assert torch.equal(tc[-1], mma[-1])   # the decode row takes the same kernel on both
+    pa.pa_set_path(pa.Path.TCGEN05_PAIRS)  # two query tiles per chunk item
+    pairs = gpu_attention(b, kc, vc, varlen=True)
+    assert_close(pairs, f64(mma), "bf16", "tcgen05 pairs vs mma tiles")
+    assert torch.equal(pairs[-1], mma[-1])
 
 
 def test_varlen_decode_rows_equal_decode():
