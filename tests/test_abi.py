@@ -43,6 +43,22 @@ def test_header_declares_the_boundary():
         assert must in names
 
 
+def _header_enum(prefix):
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    return {m.group(1): int(m.group(2))
+            for m in re.finditer(r"\b(" + prefix + r"[A-Z0-9_]*)\s*=\s*(\d+)", text)}
+
+
+def test_binding_enums_mirror_the_header():
+    """The Python enums carry the header's values, so a new path or status
+    cannot drift between the C ABI and the binding."""
+    paths = _header_enum("PA_PATH_")
+    assert paths == {"PA_PATH_" + p.name: int(p) for p in pa.Path}
+    statuses = _header_enum("PA_(?:OK|ERR_)")
+    assert statuses == {("PA_OK" if s.name == "OK" else "PA_ERR_" + s.name): int(s)
+                        for s in pa.Status}
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), f"{name} missing from libpa.so"
