@@ -4,10 +4,12 @@ The hot path of a paged-KV serving engine's attention layer as a C-ABI
 library (``libpa.so``, declared in ``include/pa.h``) with hand-written CUDA
 kernels, and this thin Python binding of it:
 
-* :func:`pa_reshape_and_cache` -- scatter new K/V rows into 16-token blocks;
+* :func:`pa_reshape_and_cache` -- scatter new K/V rows into 8-, 16- or 32-token
+  blocks;
 * :func:`pa_decode` -- block-table-indirected decode attention (GQA, online
   softmax, split-K with a log-sum-exp reduce);
-* :func:`pa_varlen` -- mixed batches of decode rows and causal prefill chunks;
+* :func:`pa_varlen` -- mixed batches of decode rows and causal prefill chunks
+  (the chunks on tcgen05 tensor cores with TMEM accumulators);
 * :func:`pa_copy_blocks` / :func:`pa_swap_blocks` -- copy-on-write copies
   inside a pool, swap-out / swap-in between the device and a host pool;
 * :func:`pa_reshape_and_cache_fp8`, :func:`pa_decode_fp8`,
