@@ -3,14 +3,19 @@
 
 One step = one pass of the whole hot path over one seeded synthetic batch:
 ``pa_reshape_and_cache`` of the step's new K/V rows, then paged attention
-(``pa_decode`` for decode batches, ``pa_varlen`` for the mixed batch), all
+(``pa_varlen`` for mixed batches, ``pa_decode`` for decode batches), all
 through the C ABI.  The KV cache is resident in HBM (it is the engine's state);
-``value`` is the step's algorithmic bytes (every visible K/V row once, q, out,
-block-table entries, the cache write) over the device time of the step, in
-GB/s.  ``e2e`` repeats the measurement with each step's inputs copied from
-pinned host memory and its output copied back inside the timed region (the
-copies on their own streams, double-buffered, overlapping the compute of the
-neighbouring steps).
+``value`` is the step's algorithmic bytes (every visible K/V row once, a
+shared prefix once, q, out, block-table entries, the cache write) over the
+device time of the step, in GB/s.  The headline workload is the mixed
+scheduler iteration (a 512-token causal prefill chunk next to 1536 decode
+rows, half of them sharing a 512-token prefix): the largest batch, and the
+one that runs both halves of the path.
+
+``roofline`` times the attention call alone in a loop of back-to-back calls
+(events around the loop only), so its duration is at most a step's.  ``e2e``
+repeats the step with each step's inputs copied from pinned host memory and
+its output copied back inside the timed region.
 
 Usage:  python bench.py [--gpus N --steps K --warmup W] [--workload NAME]
         python bench.py --impl reference ...   (the fp64 oracle on host cores)
@@ -29,55 +34,50 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = ("paged-attn decode KV-read GB/s (% of B200 HBM peak); decode tokens/s per config")
-HEADLINE = "mha_bs64"
+HEADLINE = "mixed_2048"
+PER_CONFIG = ("mha_bs64", "gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512",
+              "gqa_bs256_b8", "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--per-config-steps", type=int, default=300)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--per-config-steps", type=int, default=100)
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU-seconds of oracle work in the cpu_baseline sample")
     return ap.parse_args()
 
 
-FALLBACK_BF16_TFLOPS = 1590.0
-
-
 def measured_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    try:
-        with open(path) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
-
-
-def measured_tensor_peak() -> float:
+    """(HBM GB/s, bf16 TFLOP/s, kind): MEASURED_PEAKS.json, else the fallback."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            return float(json.load(f)["bf16_tflops"])
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except Exception:
-        return FALLBACK_BF16_TFLOPS
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-# Sources the attention kernel is compiled from (its traffic record is keyed to them).
-ATTENTION_SOURCES = ("pa_common.cuh", "pa_sched.cuh", "pa_attn_mma.cuh")
+# Sources the attention kernels are compiled from (traffic records are keyed to them).
+ATTENTION_SOURCES = ("pa_common.cuh", "pa_sched.cuh", "pa_attn_mma.cuh", "pa_chunk_tc.cuh",
+                     "pa_tcgen05.cuh", "pa_reduce.cuh")
 
 
 def kernel_source_hash() -> str:
@@ -90,38 +90,49 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per launch of the attention kernel from the committed ncu
-    summary, if it was taken on the current kernel sources."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes of one attention call from the committed ncu summary, if it
+    was taken on the current kernel sources."""
     try:
-        with open(path) as f:
-            d = json.load(f)
-        e = d.get(workload)
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            e = json.load(f).get(workload)
         if e and e.get("source_hash") == kernel_source_hash():
-            return e.get("dram_bytes_per_launch")
+            return e.get("dram_bytes_per_call")
     except Exception:
         pass
     return None
 
 
 # ---------------------------------------------------------------------------
-# clocks during the timed region
+# clocks: nvidia-smi sampled from the first warm-up step to the end of the run
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, uuid: str):
         self.uuid = uuid.lower().replace("gpu-", "")
+        self.marks = {}
+        self.lines = []
         self.proc = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.INTERVAL_MS)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
         except Exception:
             self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
+    def mark(self, name: str) -> None:
+        self.marks[name] = time.time()
 
     def stop(self) -> dict:
         if self.proc is None:
@@ -129,119 +140,110 @@ class ClockSampler:
                     "note": "nvidia-smi unavailable"}
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=10)
+            self.proc.wait(timeout=10)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
-        for line in out.splitlines():
+        self.reader.join(timeout=5)
+        rows = []
+        for line in self.lines:
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9 or f[0].lower().replace("gpu-", "") != self.uuid:
+            if len(f) < 10 or f[1].lower().replace("gpu-", "") != self.uuid:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]), float(f[5]),
+                             {n for n, v in zip(self.REASONS, f[6:10])
+                              if v.lower().startswith("active")}))
             except ValueError:
                 continue
-            for name, val in zip(self.REASONS, f[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        load = [r for r in rows if r[3] >= 30.0]
+        t0, t1 = self.marks.get("timed_start"), self.marks.get("timed_end")
+        timed = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        reasons = sorted(set().union(*[r[4] for r in load])) if load else []
+        return {"sm_mhz": statistics.median(r[1] for r in load) if load else None,
+                "sm_max_mhz": max(r[2] for r in rows) if rows else None,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "samples_in_timed_region": len(timed),
+                "timed_region_sm_mhz": statistics.median(r[1] for r in timed) if timed else None,
+                "interval_ms": self.INTERVAL_MS,
+                "note": "nvidia-smi from the first warm-up step to the end of the run "
+                        "(per_config and e2e included); 'under load' = utilization >= 30%"}
 
 
 # ---------------------------------------------------------------------------
-# oracle timing (cpu_baseline and the reference arm)
+# the fp64 oracle on host cores (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
-def oracle_units(batch, n_units: int, start: int = 0):
-    """The next ``n_units`` (request, kv head) sub-problems of ``batch``."""
-    units = []
-    for u in range(start, start + n_units):
-        r = u % batch.num_seqs
-        g = (u // batch.num_seqs) % batch.num_kv_heads
-        units.append((r, g))
-    return units
+def host_sample_batch(W, workload: str, seed: int, max_requests: int):
+    """A host (CPU) batch of the workload's recipe holding its first requests
+    (the chunk rows of a mixed batch are kept): the oracle's sample."""
+    spec = dict(W.CONFIGS[workload])
+    reqs = spec.pop("requests")(seed)
+    spec.pop("kind")
+    spec.pop("about")
+    chunks = [r for r in reqs if r.q_len > 1]
+    decode = [r for r in reqs if r.q_len <= 1]
+    keep = decode[:max(0, max_requests - len(chunks[:2]))] + chunks[:2]
+    if not any(r.shares_prefix for r in keep):
+        spec.pop("shared_prefix_len", None)
+    return W.build_batch(keep, seed=seed, device="cpu", name=workload, **spec)
 
 
-def time_oracle(batch, units):
-    """Run the oracle on (request, kv head) sub-problems; returns (seconds, bytes)."""
+def oracle_pool_for(batch, workers=None):
+    """An oracle.parallel pool over the host batch (its tensors in shared memory)."""
     import numpy as np
     import torch
 
-    import oracle as O
-    from pagedattention_paged_kv_reshape_b200 import workload as W
+    from oracle.parallel import OraclePool
 
-    def host(t):
-        t = t.detach().cpu().contiguous()
-        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 \
-            else t.numpy()
-
-    elem = W.ELEMENT_BYTES[batch.dtype]
-    G = batch.num_q_heads // batch.num_kv_heads
-    D = batch.head_dim
-    total_s, total_b = 0.0, 0
-    for r, g in units:
-        L = int(batch.host_seq_lens[r])
-        nb = -(-L // batch.block_size)
-        q0, q1 = int(batch.host_qsl[r]), int(batch.host_qsl[r + 1])
-        blocks = [int(x) for x in batch.host_tables[r, :nb]]
-        idx = torch.tensor(blocks, dtype=torch.long, device=batch.k_cache.device)
-        kc = host(batch.k_cache.index_select(0, idx)[:, g:g + 1])
-        vc = host(batch.v_cache.index_select(0, idx)[:, g:g + 1])
-        table = np.arange(nb, dtype=np.int32)[None, :]
-        tok = slice(q0, q1)
-        q = host(batch.q[tok, g * G:(g + 1) * G])
-        kn, vn = host(batch.k_new[tok, g:g + 1]), host(batch.v_new[tok, g:g + 1])
-        remap = {b: i for i, b in enumerate(blocks)}
-        slots = np.array([remap[int(s) // 16] * 16 + int(s) % 16 for s in batch.host_slots[q0:q1]],
-                         dtype=np.int32)
-        t0 = time.perf_counter()
-        kc2, vc2 = O.reshape_and_cache(kc, vc, kn, vn, slots)
-        if q1 - q0 == 1 and batch.is_decode:
-            O.paged_decode(q, kc2, vc2, table, np.array([L]), batch.scale, batch.dtype)
+    pool = OraclePool(workers)
+    for name in ("k_cache", "v_cache", "q", "k_new", "v_new"):
+        t = getattr(batch, name)
+        if t.dtype == torch.bfloat16:
+            arr = pool.array(name, tuple(t.shape), np.uint16)
+            torch.from_numpy(arr.view(np.int16)).copy_(t.view(torch.int16))
         else:
-            O.paged_varlen(q, kc2, vc2, table, np.array([0, q1 - q0], np.int32), np.array([L]),
-                           batch.scale, batch.dtype)
-        total_s += time.perf_counter() - t0
-        total_b += L * 2 * D * elem + 2 * (q1 - q0) * G * D * elem + 4 * nb
-    return total_s, total_b
+            arr = pool.array(name, tuple(t.shape), t.numpy().dtype)
+            arr[...] = t.numpy()
+    pool.start(tables=batch.host_tables, seq_lens=batch.host_seq_lens, qsl=batch.host_qsl,
+               slots=batch.host_slots, num_q_heads=batch.num_q_heads,
+               num_kv_heads=batch.num_kv_heads, block_size=batch.block_size, dtype=batch.dtype,
+               scale=batch.scale, varlen=not batch.is_decode, fp8=batch.fp8,
+               k_scale=None if not batch.fp8 else batch.k_scale.numpy(),
+               v_scale=None if not batch.fp8 else batch.v_scale.numpy())
+    return pool
 
 
-def oracle_threads() -> int:
+def run_oracle_units(pool, units):
+    """(wall seconds, algorithmic bytes, CPU seconds) of the oracle on ``units``."""
+    t0 = time.perf_counter()
+    res = pool.map(units)
+    wall = time.perf_counter() - t0
+    return wall, sum(r[5] for r in res), sum(r[6] for r in res)
+
+
+def cpu_baseline(W, workload: str, seed: int, cpu_seconds: float) -> dict:
+    """The oracle, as it stands, on every host core over a bounded sample of
+    the workload's (request, KV head) sub-problems."""
+    from oracle.parallel import units_of
+
+    batch = host_sample_batch(W, workload, seed, max_requests=48)
+    pool = oracle_pool_for(batch)
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
-        return 1
-
-
-def run_oracle_limited(fn):
-    """Run ``fn`` with BLAS limited to one thread, so ``cores`` is exact."""
-    try:
-        from threadpoolctl import threadpool_limits
-        with threadpool_limits(limits=1):
-            return fn(), 1
-    except Exception:
-        return fn(), oracle_threads()
-
-
-def cpu_baseline(batch, seconds: float) -> dict:
-    units_done, s, b, u = 0, 0.0, 0, 0
-
-    def go():
-        nonlocal s, b, u
-        while s < seconds and u < batch.num_seqs * batch.num_kv_heads:
-            ds, db = time_oracle(batch, oracle_units(batch, 1, u))
-            s += ds
-            b += db
-            u += 1
-
-    _, cores = run_oracle_limited(go)
-    return {"value": b / s / 1e9 if s else None, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{u} (request, kv head) sub-problems of {batch.name} "
-                      f"({b / 1e6:.1f} MB of algorithmic bytes, {s:.1f} s)"}
+        units = units_of(batch.num_seqs, batch.num_kv_heads)
+        run_oracle_units(pool, units[:pool.workers])          # workers warm
+        wall = nbytes = cpu = 0.0
+        rounds = 0
+        while cpu < cpu_seconds and rounds < 50:
+            w_, b_, c_ = run_oracle_units(pool, units)
+            wall, nbytes, cpu, rounds = wall + w_, nbytes + b_, cpu + c_, rounds + 1
+        return {"value": round(nbytes / wall / 1e9, 5), "unit": "GB/s", "cores": pool.workers,
+                "kind": "oracle",
+                "sample": f"{rounds} pass(es) over the {len(units)} (request, KV head) "
+                          f"sub-problems of a host batch of {batch.num_seqs} requests of "
+                          f"{workload}'s recipe ({nbytes / 1e6:.1f} MB of algorithmic bytes, "
+                          f"{cpu:.1f} CPU-s in {wall:.2f} s on {pool.workers} worker processes)"}
+    finally:
+        pool.close()
 
 
 # ---------------------------------------------------------------------------
@@ -272,17 +274,6 @@ def attention(pa, b, out, q, tables, lens, qsl, ws):
         pa.pa_decode(out, q, b.k_cache, b.v_cache, tables, lens, b.max_seq_len, b.scale, ws)
 
 
-def make_step(pa, b, out, ws):
-    def step():
-        cache_write(pa, b, b.k_new, b.v_new, b.slot_mapping)
-        attend()
-
-    def attend():
-        attention(pa, b, out, b.q, b.block_tables, b.seq_lens, b.query_start_loc, ws)
-
-    return step, attend
-
-
 def workspace_for(pa, b):
     if b.is_decode:
         n = pa.pa_decode_workspace_size(b.num_seqs, b.num_q_heads, b.num_kv_heads, b.head_dim,
@@ -294,46 +285,65 @@ def workspace_for(pa, b):
 
 
 def launches_per_step(b) -> int:
+    """Our kernels per step: cache write, schedule, attention, then the
+    tcgen05 chunk kernel (rows of >= one 128-row tile of new tokens) and the
+    split-K reduce (contexts over one 512-key partition) when the batch has them."""
+    group = b.num_q_heads // b.num_kv_heads
+    gs = min(group, 16)
+    chunk_qt = 128 // gs if gs in (1, 2, 4, 8, 16) else 0
+    chunk = (not b.is_decode and not b.fp8 and b.head_dim != 256 and chunk_qt > 0
+             and b.max_query_len >= chunk_qt)
     split = math.ceil(b.max_seq_len / 512) > 1
-    return 1 + 2 + (1 if split else 0)   # cache write + schedule + attention (+ reduce)
+    return 3 + int(chunk) + int(split)
 
 
-def time_steps(torch, pa, b, steps, warmup, sample_every=10):
-    """Device time of ``steps`` steps, the mean duration of the attention call
-    and of the cache write, taken with events around both calls of every
-    ``sample_every``-th step inside the same timed region (events around every
-    call cost ~2% of the step time on B200; one in ten costs nothing
-    measurable).  Returns (total_ms, attention_ms, cache_write_ms, out)."""
+def timed_loop(torch, fn, n: int, warmup: int = 3) -> float:
+    """Mean ms of ``fn`` over ``n`` back-to-back calls, CUDA events on the
+    launching stream around the loop only."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(n):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / n
+
+
+def measure_workload(torch, pa, b, steps: int, warmup: int, sampler=None):
+    """(step ms, attention-call ms, cache-write ms): K steps (cache write +
+    attention) between two events after W warm-up steps, then the attention
+    call alone and the cache write alone, each in its own loop of K calls.
+    Every input is larger than the L2 except the cache write's few MB."""
     out = torch.empty_like(b.q)
     ws = workspace_for(pa, b)
-    step, attend = make_step(pa, b, out, ws)
+
+    def write():
+        cache_write(pa, b, b.k_new, b.v_new, b.slot_mapping)
+
+    def attend():
+        attention(pa, b, out, b.q, b.block_tables, b.seq_lens, b.query_start_loc, ws)
+
+    def step():
+        write()
+        attend()
+
     for _ in range(warmup):
         step()
     pa.pa_get_device_error()
     torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-    every = sample_every if steps >= sample_every else 1
-    ev = []
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(steps):
-        if i % every:
-            step()
-            continue
-        ew, e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        ew.record(stream)
-        cache_write(pa, b, b.k_new, b.v_new, b.slot_mapping)
-        e0.record(stream)
-        attend()
-        e1.record(stream)
-        ev.append((ew, e0, e1))
-    end.record(stream)
-    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark("timed_start")
+    step_ms = timed_loop(torch, step, steps, warmup=0)
+    if sampler:
+        sampler.mark("timed_end")
+    attn_ms = timed_loop(torch, attend, steps)
+    write_ms = timed_loop(torch, write, steps)
     pa.pa_get_device_error()
-    total_ms = start.elapsed_time(end)
-    attn_ms = statistics.fmean(e0.elapsed_time(e1) for _, e0, e1 in ev)
-    write_ms = statistics.fmean(ew.elapsed_time(e0) for ew, e0, _ in ev)
-    return total_ms, attn_ms, write_ms, out
+    return step_ms, attn_ms, write_ms
 
 
 def time_e2e(torch, pa, b, steps):
@@ -431,22 +441,9 @@ def measure_block_ops(torch, pa, dev, peak) -> dict:
     host_v = torch.empty_like(host_k).pin_memory()
     omap = torch.stack([perm[:n_swap], torch.arange(n_swap)], 1).int().to(dev)
     imap = torch.stack([torch.arange(n_swap), perm[2 * n_copy:2 * n_copy + n_swap]], 1).int().to(dev)
-
-    def timed(fn, iters=10):
-        for _ in range(3):
-            fn()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        s.record()
-        for _ in range(iters):
-            fn()
-        e.record()
-        torch.cuda.synchronize()
-        return s.elapsed_time(e) / iters
-
-    copy_ms = timed(lambda: pa.pa_copy_blocks(k, v, cmap))
-    out_ms = timed(lambda: pa.pa_swap_blocks(k, v, host_k, host_v, omap))
-    in_ms = timed(lambda: pa.pa_swap_blocks(host_k, host_v, k, v, imap))
+    copy_ms = timed_loop(torch, lambda: pa.pa_copy_blocks(k, v, cmap), 10)
+    out_ms = timed_loop(torch, lambda: pa.pa_swap_blocks(k, v, host_k, host_v, omap), 10)
+    in_ms = timed_loop(torch, lambda: pa.pa_swap_blocks(host_k, host_v, k, v, imap), 10)
     pa.pa_get_device_error()
     copy_gbs = 2 * n_copy * block_bytes / (copy_ms / 1e3) / 1e9
     return {"copy_blocks": {"pairs": n_copy, "ms": round(copy_ms, 4),
@@ -478,23 +475,36 @@ def measure_rope_write(torch, pa, dev, peak) -> dict:
     inv = 10000.0 ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
     ang = torch.arange(8192, dtype=torch.float64)[:, None] * inv[None, :]
     table = torch.cat([ang.cos(), ang.sin()], 1).float().to(dev)
-    for _ in range(3):
-        pa.pa_rope_reshape_and_cache(q, k, v, kc, vc, slots, positions, table)
-    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    s_ev.record()
-    iters = 20
-    for _ in range(iters):
-        pa.pa_rope_reshape_and_cache(q, k, v, kc, vc, slots, positions, table)
-    e_ev.record()
-    torch.cuda.synchronize()
+    ms = timed_loop(torch, lambda: pa.pa_rope_reshape_and_cache(q, k, v, kc, vc, slots,
+                                                                positions, table), 20)
     pa.pa_get_device_error()
-    ms = s_ev.elapsed_time(e_ev) / iters
     nbytes = (2 * T * hq * d * 2 + 2 * T * hkv * d * 2 + 2 * T * hkv * d * 2 + T * d * 4
               + 8 * T)
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"tokens": T, "ms": round(ms, 4), "algorithmic_bytes": nbytes, "gbs": round(gbs, 1),
             "pct_of_hbm_peak": round(100 * gbs / peak, 1)}
+
+
+def per_config_entry(A, b, step_ms, attn_ms, write_ms, peak, tensor_peak) -> dict:
+    acc = A.attention_bytes(b)
+    sb = acc["total"] + A.reshape_bytes(b)
+    attn_gbs = acc["total"] / (attn_ms / 1e3) / 1e9
+    ent = {"step_gbs": round(sb / (step_ms / 1e3) / 1e9, 1),
+           "attention_gbs": round(attn_gbs, 1),
+           "pct_of_hbm_peak": round(100 * attn_gbs / peak, 1),
+           "ms_per_step": round(step_ms, 4), "attention_ms": round(attn_ms, 4),
+           "cache_write_ms": round(write_ms, 4),
+           "tokens_per_s": round(b.total_q / (step_ms / 1e3), 1)}
+    if A.chunk_flops(b):
+        ent["chunk_gflop"] = round(A.chunk_flops(b) / 1e9, 2)
+    if any(r.shares_prefix for r in b.requests):
+        ent["unique_vs_logical_kv"] = [acc["kv_unique"], acc["kv_logical"]]
+    if all(r.q_len > 1 for r in b.requests):   # dense causal chunks: a tensor-core roofline
+        tflops = A.chunk_flops(b) / (attn_ms / 1e3) / 1e12
+        ent.update({"chunk_tflops": round(tflops, 1),
+                    "pct_of_bf16_peak": round(100 * tflops / tensor_peak, 1),
+                    "tokens_per_s": round(b.total_q / (attn_ms / 1e3), 1)})
+    return ent
 
 
 def run_ours(args):
@@ -522,6 +532,7 @@ def run_ours(args):
     pa.lib()
 
     dev = torch.device("cuda", local)
+    peak, tensor_peak, peak_kind = measured_peaks()
     b = W.make_config(args.workload, seed=args.seed + rank, device=dev)
     acc = A.attention_bytes(b)
     step_bytes = acc["total"] + A.reshape_bytes(b)
@@ -531,11 +542,15 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    total_ms, attn_ms, write_ms, _ = time_steps(torch, pa, b, args.steps, args.warmup)
-    clocks = sampler.stop() if sampler else None
-
-    max_ms, value, tok_per_s = combine_over_ranks(total_ms, step_bytes * args.steps,
+    step_ms, attn_ms, write_ms = measure_workload(torch, pa, b, args.steps, args.warmup,
+                                                  sampler)
+    max_ms, value, tok_per_s = combine_over_ranks(step_ms * args.steps,
+                                                  step_bytes * args.steps,
                                                   b.total_q * args.steps, dev)
+    attn_t = torch.tensor([attn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(attn_t, op=dist.ReduceOp.MAX)
+    attn_ms = attn_t.item()
 
     e2e_ms, h2d, d2h = time_e2e(torch, pa, b, args.e2e_steps)
     e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
@@ -543,8 +558,9 @@ def run_ours(args):
         dist.all_reduce(e2e, op=dist.ReduceOp.MAX)
     e2e_value = step_bytes * world / (e2e.item() / 1e3) / 1e9
 
-    peak, peak_kind = measured_peaks()
     achieved = acc["total"] / (attn_ms / 1e3) / 1e9
+    peak_note = ("of measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                 else f"of fallback ({FALLBACK_HBM_GBS:.0f} GB/s; MEASURED_PEAKS.json absent)")
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -571,64 +587,42 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(args.workload),
-                     "kernel": "pa_decode/pa_varlen call (schedule + attention + split-K reduce "
-                               "kernels), CUDA events on the launching stream around "
-                               "every 10th call of the timed steps",
+                     "kernel": ("one pa_varlen call (schedule_kernel + attn_mma_kernel + "
+                                "chunk_tc_kernel + reduce_kernel)" if not b.is_decode else
+                                "one pa_decode call (schedule_kernel + attn_mma_kernel "
+                                "[+ reduce_kernel])"),
+                     "timing": f"CUDA events on the launching stream around a loop of "
+                               f"{args.steps} back-to-back calls (mean {attn_ms:.4f} ms)",
                      "algorithmic_bytes_per_launch": acc["total"],
-                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
-                     if peak_kind == "measured" else "fallback 6650 GB/s"},
+                     "peak_kind": peak_note},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e.item(), 5)},
         "cache_write": {"ms": round(write_ms, 5), "bytes": A.reshape_bytes(b),
-                        "gbs": round(A.reshape_bytes(b) / (write_ms / 1e3) / 1e9, 1),
-                        "note": "pa_reshape_and_cache of the step's new rows, CUDA events "
-                                "around every 10th call of the timed steps"},
+                        "note": "pa_reshape_and_cache alone, a loop of back-to-back calls; "
+                                "launch-latency bound (a few MB), not a bandwidth figure"},
         "gpu_launches": launches_per_step(b) * args.steps,
-        "clocks": clocks,
     }
 
     if not args.no_per_config:
-        tensor_peak = measured_tensor_peak()
-        per = {}
-        for name in ("gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512", "gqa_bs256_b8",
-                     "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256"):
+        per = {args.workload: per_config_entry(A, b, step_ms, attn_ms, write_ms, peak,
+                                               tensor_peak)}
+        for name in PER_CONFIG:
             if name == args.workload:
                 continue
             del b
             torch.cuda.empty_cache()
             b = W.make_config(name, seed=args.seed + rank, device=dev)
-            a2 = A.attention_bytes(b)
-            tot, attn, wr, _ = time_steps(torch, pa, b, args.per_config_steps,
-                                          max(3, args.warmup // 4))
-            sb = a2["total"] + A.reshape_bytes(b)
-            ent = {"step_gbs": round(sb / (tot / args.per_config_steps / 1e3) / 1e9, 1),
-                   "attention_gbs": round(a2["total"] / (attn / 1e3) / 1e9, 1),
-                   "pct_of_hbm_peak": round(100 * a2["total"] / (attn / 1e3) / 1e9 / peak, 1),
-                   "ms_per_step": round(tot / args.per_config_steps, 4),
-                   "attention_ms": round(attn, 4),
-                   "cache_write_ms": round(wr, 4),
-                   "tokens_per_s": round(b.total_q / (tot / args.per_config_steps / 1e3), 1)}
-            if name == "mixed_2048":
-                ent["unique_vs_logical_kv"] = [a2["kv_unique"], a2["kv_logical"]]
-                ent["chunk_gflop"] = round(A.chunk_flops(b) / 1e9, 2)
-            if name == "prefill_16x512":   # dense causal chunks: a tensor-core roofline
-                tflops = A.chunk_flops(b) / (attn / 1e3) / 1e12
-                ent = {"chunk_tflops": round(tflops, 1),
-                       "pct_of_bf16_peak": round(100 * tflops / tensor_peak, 1),
-                       "attention_ms": round(attn, 4), "cache_write_ms": round(wr, 4),
-                       "chunk_gflop": round(A.chunk_flops(b) / 1e9, 1),
-                       "peak_kind": "measured bf16_tflops (burst)",
-                       "tokens_per_s": round(b.total_q / (attn / 1e3), 1)}
-            per[name] = ent
+            s_ms, a_ms, w_ms = measure_workload(torch, pa, b, args.per_config_steps,
+                                                max(3, args.warmup // 4))
+            per[name] = per_config_entry(A, b, s_ms, a_ms, w_ms, peak, tensor_peak)
         result["per_config"] = per
         result["block_ops"] = measure_block_ops(torch, pa, dev, peak)
         result["rope_cache_write"] = measure_rope_write(torch, pa, dev, peak)
+        result["peaks"] = {"hbm_gbs": peak, "bf16_tflops": tensor_peak, "kind": peak_kind}
+    result["clocks"] = sampler.stop() if sampler else None
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        del b
-        torch.cuda.empty_cache()
-        b = W.make_config(args.workload, seed=args.seed, device=dev)
-        result["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(W, args.workload, args.seed, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -644,40 +638,40 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    import torch
-
+    from oracle.parallel import units_of
     from pagedattention_paged_kv_reshape_b200 import workload as W
 
     # the same recipe on the host (values differ from the GPU draw; shapes match)
-    spec = dict(W.CONFIGS[args.workload])
-    reqs = spec.pop("requests")(args.seed)
-    spec.pop("kind")
-    spec.pop("about")
-    b = _host_sample_batch(W, args, reqs, spec)
-    # calibrate sub-problems per step so the whole run stays within ~3 minutes
-    probe_s, _ = run_oracle_limited(lambda: time_oracle(b, oracle_units(b, 2, 0)))[0]
-    per_unit = max(probe_s / 2, 1e-4)
-    budget = min(1.0, 150.0 / max(1, args.steps + args.warmup))
-    per_step = max(1, int(budget / per_unit))
-    u = 2
+    b = host_sample_batch(W, args.workload, args.seed, max_requests=64)
+    pool = oracle_pool_for(b)
+    try:
+        units = units_of(b.num_seqs, b.num_kv_heads)
+        # calibrate the sub-problems per step so the whole run takes ~2-3 minutes
+        w_, _, _ = run_oracle_units(pool, units)
+        per_unit = max(w_ / len(units), 1e-5)
+        budget = min(6.0, 150.0 / max(1, args.steps + args.warmup))
+        per_step = max(pool.workers, int(budget / per_unit))
+        cursor = 0
 
-    def go():
-        nonlocal u
+        def next_units():
+            nonlocal cursor
+            out = [units[(cursor + i) % len(units)] for i in range(per_step)]
+            cursor += per_step
+            return out
+
         for _ in range(args.warmup):
-            time_oracle(b, oracle_units(b, per_step, u))
-            u += per_step
-        s = nb = 0
+            run_oracle_units(pool, next_units())
+        s = nb = cpu = 0.0
         for _ in range(args.steps):
-            ds, db = time_oracle(b, oracle_units(b, per_step, u))
-            u += per_step
-            s += ds
-            nb += db
-        return s, nb
-
-    (s, nb), cores = run_oracle_limited(go)
+            w_, b_, c_ = run_oracle_units(pool, next_units())
+            s, nb, cpu = s + w_, nb + b_, cpu + c_
+        cores = pool.workers
+    finally:
+        pool.close()
     value = nb / s / 1e9
-    sample = (f"{per_step} (request, kv head) sub-problems per step of {args.workload} "
-              f"(host-drawn batch of the same recipe)")
+    sample = (f"{per_step} (request, KV head) sub-problems per step, cycling over a host batch "
+              f"of {b.num_seqs} requests of {args.workload}'s recipe; {cpu:.1f} CPU-s over "
+              f"{cores} worker processes")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -690,12 +684,6 @@ def run_reference(args):
         "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)
-
-
-def _host_sample_batch(W, args, reqs, spec):
-    """A host batch holding the first requests of the workload (enough to sample)."""
-    keep = reqs[:16] if not spec.get("shared_prefix_len") else reqs[:15] + reqs[-1:]
-    return W.build_batch(keep, seed=args.seed, device="cpu", name=args.workload, **spec)
 
 
 def main():

@@ -106,10 +106,7 @@ typedef enum {
   PA_PATH_AUTO = 0,
   PA_PATH_SIMT = 1,     /* CUDA-core kernel, plain vector loads (any dtype) */
   PA_PATH_MMA = 2,      /* TMA bulk-tensor loads + warp-level bf16/f16 tensor-core MMA */
-  PA_PATH_TCGEN05 = 3,  /* as PA_PATH_MMA, with prefill chunks on tcgen05/TMEM tiles */
-  PA_PATH_TCGEN05_PAIRS = 4  /* as PA_PATH_TCGEN05, chunk items of two query tiles
-                                sharing each K/V tile (slower than PA_PATH_TCGEN05 on
-                                B200 as measured; never chosen by PA_PATH_AUTO) */
+  PA_PATH_TCGEN05 = 3   /* as PA_PATH_MMA, with prefill chunks on tcgen05/TMEM tiles */
 } pa_path;
 
 /*
@@ -387,6 +384,27 @@ const char* pa_last_error_message(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int pa_version(void);
+
+/*
+ * SM version the loaded kernels were built for, as the CUDA runtime reports
+ * it for this library's code on the current device (100 = sm_100a), or -1
+ * when no kernel image can be loaded there.
+ */
+int pa_binary_version(void);
+
+/*
+ * Test hook for the bounded waits (no counterpart in the pages).  Every wait
+ * inside the kernels gives up after a limit (about one second), records
+ * PA_ERR_TIMEOUT for pa_get_device_error and lets its CTA leave cleanly
+ * (copies already issued land first; tensor memory is freed).  With
+ * `kernel` = 1 (the decode/varlen attention kernel) or 2 (the tcgen05 chunk
+ * kernel), every CTA of that kernel leaves its first K/V tile unissued in
+ * every later call -- no copy, no arrival -- and the limit drops to about one
+ * millisecond, so the wait for that tile runs out.  0 restores normal
+ * operation.  Process-wide on the current device; synchronous.  Never set
+ * in production.
+ */
+pa_status pa_debug_lost_load(int kernel);
 
 #ifdef __cplusplus
 }

@@ -33,7 +33,6 @@ from .paged_attention import (  # noqa: F401
     softmax_attention,
     paged_decode,
     paged_varlen,
-    default_scale,
 )
 from .block_ops import copy_blocks, swap_blocks  # noqa: F401,E402
 from .fp8 import (  # noqa: F401,E402

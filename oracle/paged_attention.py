@@ -17,8 +17,6 @@ Value encodings accepted everywhere (``dtype`` argument):
 
 from __future__ import annotations
 
-import math
-
 import numpy as np
 
 # [CORE] §核心抽象 2 ("常见为 16"); [ARCH] §1.1 ("默认 16 tokens") and §5.1.
@@ -212,8 +210,3 @@ def paged_varlen(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, s
                 out[first + i, h] = softmax_attention(
                     q_i[h], keys[:visible, g, :], values[:visible, g, :], scale)
     return out
-
-
-def default_scale(head_dim: int) -> float:
-    """``1 / sqrt(d)`` of [DEEP] §2.2 and §3.3."""
-    return 1.0 / math.sqrt(head_dim)

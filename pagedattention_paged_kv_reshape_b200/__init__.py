@@ -30,7 +30,9 @@ from ._binding import (  # noqa: F401
     alloc_workspace,
     lib,
     STATIC_WORKSPACE_BYTES,
+    pa_binary_version,
     pa_copy_blocks,
+    pa_debug_lost_load,
     pa_decode,
     pa_decode_fp8,
     pa_decode_static,

@@ -37,7 +37,6 @@ class Path(enum.IntEnum):
     SIMT = 1
     MMA = 2
     TCGEN05 = 3
-    TCGEN05_PAIRS = 4
 
 
 DTYPE_CODES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
@@ -78,6 +77,8 @@ _SIGNATURES = {
     "pa_status_string": (ctypes.c_char_p, [_c_int]),
     "pa_last_error_message": (ctypes.c_char_p, []),
     "pa_version": (_c_int, []),
+    "pa_binary_version": (_c_int, []),
+    "pa_debug_lost_load": (_c_int, [_c_int]),
 }
 
 _lock = threading.Lock()
@@ -384,3 +385,15 @@ def pa_status_string(status: int) -> str:
 
 def pa_version() -> int:
     return int(lib().pa_version())
+
+
+def pa_binary_version() -> int:
+    """SM version of the loaded kernel image on the current device (100 = sm_100a)."""
+    return int(lib().pa_binary_version())
+
+
+def pa_debug_lost_load(kernel: int) -> None:
+    """Test hook of the bounded waits (see include/pa.h): 1 or 2 makes every CTA
+    of the attention or chunk kernel leave its first K/V tile unissued, with a
+    wait limit of about a millisecond; 0 restores normal operation."""
+    _check(lib().pa_debug_lost_load(int(kernel)))

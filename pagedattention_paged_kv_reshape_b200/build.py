@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import argparse
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -41,15 +42,30 @@ def _sources() -> list[str]:
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+STAMP = LIB + ".sources"  # hash of the sources and flags the library was built from
+
+
+def source_hash() -> str:
+    """SHA-256 over the build flags and every source file (names and bytes)."""
+    h = hashlib.sha256(" ".join(NVCC_FLAGS).encode())
+    for path in _sources():
+        h.update(os.path.relpath(path, ROOT).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    """True when libpa.so exists and was built from exactly the current sources
+    (a library copied in from elsewhere, or built from older sources, is not)."""
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(s) <= t for s in _sources())
+    with open(STAMP) as f:
+        return f.read().strip() == source_hash()
 
 
 def build(force: bool = False, ptxas_info: bool = False, quiet: bool = False) -> str:
-    """Compile libpa.so unless it is newer than every source.  Returns its path."""
+    """Compile libpa.so unless its stamp matches the current sources.  Returns its path."""
     if not force and up_to_date():
         return LIB
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC,
@@ -63,7 +79,11 @@ def build(force: bool = False, ptxas_info: bool = False, quiet: bool = False) ->
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if ptxas_info or not quiet:
         sys.stderr.write(res.stderr)
+    digest = source_hash()
     os.replace(LIB + ".tmp", LIB)
+    with open(STAMP + ".tmp", "w") as f:
+        f.write(digest + "\n")
+    os.replace(STAMP + ".tmp", STAMP)
     return LIB
 
 

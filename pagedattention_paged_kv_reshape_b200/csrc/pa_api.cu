@@ -16,7 +16,6 @@
 #include "pa_attn_mma.cuh"
 #include "pa_attn_simt.cuh"
 #include "pa_blocks.cuh"
-#include "pa_chunk_pair.cuh"
 #include "pa_chunk_tc.cuh"
 #include "pa_reduce.cuh"
 
@@ -305,8 +304,6 @@ pa_status check_common(const AttnArgs& a) {
                 a.num_q_heads, a.num_kv_heads);
   if (a.head_dim != 64 && a.head_dim != 128 && a.head_dim != 256)
     return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128, 256)", a.head_dim);
-  if (a.head_dim == 256 && (a.dtype == PA_F32 || a.kv8()))
-    return fail(PA_ERR_UNSUPPORTED, "head_dim 256 runs on the bf16/f16 tensor-core path only");
   if (!supported_block_size(a.block_size))
     return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", a.block_size);
   if (!(std::isfinite(a.scale))) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
@@ -333,13 +330,14 @@ template <typename T, int D, bool KV8>
 pa_status launch_simt(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   using C = typename std::conditional<KV8, uint8_t, T>::type;  // cache element
   auto kern = pa::attn_simt_kernel<T, D, KV8>;
+  constexpr int smem = pa::simt_smem_bytes<D>();
   int occ = 0;
-  cudaError_t e = prepare(kern, 128, 0, &occ);
+  cudaError_t e = prepare(kern, 128, smem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "simt kernel set-up");
   long long grid = static_cast<long long>(sm_count()) * occ;
   if (p.max_units < grid) grid = p.max_units;
   if (grid < 1) grid = 1;
-  e = launch_pdl(kern, static_cast<unsigned>(grid), 128, 0, a.stream, p.s,
+  e = launch_pdl(kern, static_cast<unsigned>(grid), 128, smem, a.stream, p.s,
                  static_cast<T*>(a.out), static_cast<const T*>(a.q),
                  static_cast<const C*>(a.k_cache), static_cast<const C*>(a.v_cache),
                  a.block_tables, a.qsl, a.seq_lens, w, static_cast<float>(a.scale * M_LOG2E),
@@ -408,32 +406,16 @@ pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   return PA_OK;
 }
 
-template <typename T, int D>
-pa_status launch_chunk_pair(const AttnArgs& a, const Plan& p, const pa::Work& w) {
-  using L = pa::TcPairLayout<D>;
-  auto kern = pa::chunk_pair_kernel<T, D>;
-  int occ = 0;
-  cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
-  if (e != cudaSuccess) return cuda_fail(e, "chunk pair kernel set-up");
-  CUtensorMap tk, tv, tq;
-  // one box = 16 cache rows, or one whole 8-token block
-  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.num_kv_heads * a.block_size;
-  const int box_rows = a.block_size < pa::kBlock ? a.block_size : pa::kBlock;
-  pa_status st = make_map_kv(&tk, a.k_cache, a.dtype, D, rows, box_rows / 8);
-  if (st != PA_OK) return st;
-  st = make_map_kv(&tv, a.v_cache, a.dtype, D, rows, box_rows / 8);
-  if (st != PA_OK) return st;
-  st = make_map_3d(&tq, a.q, a.dtype, D, a.num_q_heads, a.total_q, p.s.gs, p.s.chunk_qt);
-  if (st != PA_OK) return st;
-  long long grid = sm_count();
-  const long long items = p.chunk_cap * a.num_kv_heads * p.s.ns;
-  if (items < grid) grid = items;
-  if (grid < 1) grid = 1;
-  e = launch_pdl(kern, static_cast<unsigned>(grid), L::kThreads, L::kSmem, a.stream, tk, tv, tq,
-                 p.s, static_cast<T*>(a.out), a.block_tables, a.qsl, a.seq_lens, w,
-                 static_cast<float>(a.scale * M_LOG2E));
-  if (e != cudaSuccess) return cuda_fail(e, "chunk pair kernel launch");
-  return PA_OK;
+// The CUDA-core kernel for the call's head_dim and cache type.
+template <typename T>
+pa_status simt_for_dim(const AttnArgs& a, const Plan& p, const pa::Work& w) {
+  switch (a.head_dim) {
+    case 64: return a.kv8() ? launch_simt<T, 64, true>(a, p, w) : launch_simt<T, 64, false>(a, p, w);
+    case 128:
+      return a.kv8() ? launch_simt<T, 128, true>(a, p, w) : launch_simt<T, 128, false>(a, p, w);
+    default:
+      return a.kv8() ? launch_simt<T, 256, true>(a, p, w) : launch_simt<T, 256, false>(a, p, w);
+  }
 }
 
 template <typename T>
@@ -446,29 +428,20 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   const bool d128 = a.head_dim == 128;
   if constexpr (sizeof(T) == 2) {
     if (a.head_dim == 256)
-      st = launch_mma<T, 256, false>(a, p, w);
+      st = a.kv8() ? launch_mma<T, 256, true>(a, p, w) : launch_mma<T, 256, false>(a, p, w);
     else if (use_mma)
       st = a.kv8() ? (d128 ? launch_mma<T, 128, true>(a, p, w) : launch_mma<T, 64, true>(a, p, w))
                    : (d128 ? launch_mma<T, 128, false>(a, p, w)
                            : launch_mma<T, 64, false>(a, p, w));
     else
-      st = a.kv8() ? (d128 ? launch_simt<T, 128, true>(a, p, w)
-                           : launch_simt<T, 64, true>(a, p, w))
-                   : (d128 ? launch_simt<T, 128, false>(a, p, w)
-                           : launch_simt<T, 64, false>(a, p, w));
+      st = simt_for_dim<T>(a, p, w);
   } else {
-    st = a.kv8() ? (d128 ? launch_simt<T, 128, true>(a, p, w) : launch_simt<T, 64, true>(a, p, w))
-                 : (d128 ? launch_simt<T, 128, false>(a, p, w)
-                         : launch_simt<T, 64, false>(a, p, w));
+    st = simt_for_dim<T>(a, p, w);
   }
   if (st != PA_OK) return st;
   if constexpr (sizeof(T) == 2) {
     if (p.s.chunk_qt > 0) {
-      if (p.s.chunk_span > p.s.chunk_qt)
-        st = a.head_dim == 128 ? launch_chunk_pair<T, 128>(a, p, w)
-                               : launch_chunk_pair<T, 64>(a, p, w);
-      else
-        st = a.head_dim == 128 ? launch_chunk<T, 128>(a, p, w) : launch_chunk<T, 64>(a, p, w);
+      st = a.head_dim == 128 ? launch_chunk<T, 128>(a, p, w) : launch_chunk<T, 64>(a, p, w);
       if (st != PA_OK) return st;
     }
   }
@@ -530,13 +503,11 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
     return fail(PA_ERR_INVALID_ARG, "bad k_scale / v_scale pointer");
   const int path = g_path.load();
   const bool sixteen = a.dtype != PA_F32;
-  if (path == PA_PATH_MMA || path == PA_PATH_TCGEN05 || path == PA_PATH_TCGEN05_PAIRS) {
+  if (path == PA_PATH_MMA || path == PA_PATH_TCGEN05) {
     if (!sixteen)
       return fail(PA_ERR_UNSUPPORTED, "tensor-core path needs bf16 or f16 (got fp32)");
   }
   const bool use_mma = sixteen && path != PA_PATH_SIMT;
-  if (a.head_dim == 256 && !use_mma)
-    return fail(PA_ERR_UNSUPPORTED, "head_dim 256 has no CUDA-core path");
   // Prefill-chunk rows (q_len >= one 128-row tile) go to the tcgen05 kernel
   // unless a family without it was forced.
   p.s.chunk_qt = (use_mma && !a.kv8() && a.head_dim != 256 && path != PA_PATH_MMA &&
@@ -545,8 +516,7 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
                      ? p.chunk_qt
                      : 0;
   p.s.chunk_cap = static_cast<int>(p.chunk_cap);
-  // one query tile per chunk item, or two with PA_PATH_TCGEN05_PAIRS
-  p.s.chunk_span = path == PA_PATH_TCGEN05_PAIRS ? 2 * p.s.chunk_qt : p.s.chunk_qt;
+  p.s.chunk_span = p.s.chunk_qt;
   switch (a.dtype) {
     case PA_BF16: return run_typed<__nv_bfloat16>(a, p, use_mma);
     case PA_F16: return run_typed<__half>(a, p, use_mma);
@@ -557,22 +527,43 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
 // Scratch for pa_decode_static: a fixed array in the library's device image,
 // for callers that cannot allocate (see include/pa.h).  Host code may not use
 // the symbol itself as a device address; static_workspace() looks the address
-// up once per device with that device current.
+// up, with the device current, once per (device, context): after a
+// cudaDeviceReset the primary context is new and the module may load
+// elsewhere, so a new context gets a new lookup.
 static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 
 pa_status static_workspace(void** ptr) {
   static std::mutex mu;
-  static std::map<int, void*> addr;
+  static std::map<std::pair<int, CUcontext>, void*> addr;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  CUcontext ctx = nullptr;
+  const CtxGetCurrentFn get = ctx_get_current_fn();
+  if (!get || get(&ctx) != CUDA_SUCCESS) ctx = nullptr;  // keyed on the device alone
   std::lock_guard<std::mutex> lk(mu);
-  auto it = addr.find(dev);
+  const auto key = std::make_pair(dev, ctx);
+  auto it = addr.find(key);
   if (it == addr.end()) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
-    it = addr.emplace(dev, p).first;
+    it = addr.emplace(key, p).first;
   }
   *ptr = it->second;
   return PA_OK;
@@ -623,8 +614,8 @@ pa_status pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, 
   if (!valid_dtype(dtype)) return fail(PA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks < 0)
     return fail(PA_ERR_INVALID_ARG, "bad sizes");
-  if (head_dim != 64 && head_dim != 128)
-    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", head_dim);
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128, 256)", head_dim);
   if (!supported_block_size(block_size))
     return fail(PA_ERR_UNSUPPORTED, "block_size %d (supported: 8, 16, 32)", block_size);
   if (num_tokens == 0) return PA_OK;
@@ -931,6 +922,26 @@ const char* pa_status_string(pa_status status) {
 }
 
 const char* pa_last_error_message(void) { return g_msg.c_str(); }
+
+pa_status pa_debug_lost_load(int kernel) {
+  if (kernel < 0 || kernel > 2) return fail(PA_ERR_INVALID_ARG, "kernel %d (0, 1 or 2)", kernel);
+  // about one millisecond at the top SM clock while the hook is on
+  const long long limit = kernel ? 2000000LL : pa::kWaitLimitCycles;
+  cudaError_t e = cudaMemcpyToSymbol(pa::g_wait_limit_cycles, &limit, sizeof(limit));
+  if (e != cudaSuccess) return cuda_fail(e, "set wait limit");
+  e = cudaMemcpyToSymbol(pa::g_debug_lost_load, &kernel, sizeof(kernel));
+  if (e != cudaSuccess) return cuda_fail(e, "set lost-load hook");
+  return PA_OK;
+}
+
+int pa_binary_version(void) {
+  cudaFuncAttributes at{};
+  if (cudaFuncGetAttributes(&at, pa::reshape_and_cache_kernel) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return at.binaryVersion;
+}
 
 int pa_version(void) { return 100; }
 

@@ -45,8 +45,9 @@ struct MetaSlot {
 // KV8: the cache holds FP8 e4m3 codes and a stage holds the 1-byte K and V
 // tiles (16 rows x D bytes).  At head_dim 128 they are 128 B-swizzled and the
 // consumers build their MMA operands straight from them (see fp8_direct
-// below); at head_dim 64 they are unswizzled and each consumer warp first
-// converts its tile into a 16-bit staging tile laid out like a 16-bit stage.
+// below); at head_dim 64 and 256 they are unswizzled and each consumer warp
+// first converts its tile into a 16-bit staging tile laid out like a 16-bit
+// stage.
 template <int D, int NCW, int STAGES, bool KV8 = false>
 struct MmaLayout {
   static constexpr bool kStaging = KV8 && D != 128;
@@ -76,6 +77,12 @@ struct MmaLayout {
   static constexpr int kSmem = kBytes + 1024;  // slack to align the base to 1024 B
   static constexpr int kThreads = (NCW + 2) * 32;
   static_assert(kOffQ % 1024 == 0 && kQSlotBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  // Inside one unit, consumer warp w takes the tiles j = w, w + NCW, ... and
+  // tile j uses stage (n0 + j) % STAGES: with STAGES a multiple of NCW every
+  // refill of a stage within a unit goes to the warp that drained it, so no
+  // warp can wait on a stage's phase while another warp still holds the
+  // previous one (across units the consumers meet at the epilogue barrier).
+  static_assert(STAGES % NCW == 0, "a stage must stay with one consumer warp inside a unit");
   // two CTAs per SM up to head_dim 128; one at 256
   static_assert(D > 128 || kSmem <= 116 * 1024, "two CTAs per SM");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
@@ -125,11 +132,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 // One FP8 tile (16 rows x D codes, row-major, as TMA lands it) -> the 16-bit
-// (f16) tile layout of a 128 B-swizzled stage.  Lane l converts 16-byte
-// groups l, l + 32, ...; every e4m3 value is exact in f16.
+// (f16) tile layout of a 128 B-swizzled stage, [8-row group][64-dim half][8
+// rows][128 B] (kv_off).  Lane l converts 16-byte groups l, l + 32, ...;
+// every e4m3 value is exact in f16.
 template <int D>
 __device__ __forceinline__ void convert_fp8_tile(uint32_t src, uint32_t dst, int lane) {
   constexpr int kGroups = D / 16;  // 16-code groups per row
+  constexpr int kGroupBytes = D / 64 * 1024;  // one 8-row group of all halves
 #pragma unroll
   for (int c = lane; c < kBlock * kGroups; c += 32) {
     const int r = c / kGroups, g = c % kGroups;
@@ -148,12 +157,12 @@ __device__ __forceinline__ void convert_fp8_tile(uint32_t src, uint32_t dst, int
       hv[2 * i + 1] = static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16);
     }
     // codes 16g .. 16g+15 = dims of half g/4, 16-byte chunks 2(g%4) and 2(g%4)+1
-    const uint32_t base = dst + (g >> 2) * (kBlock * 128);
+    const uint32_t base = dst + (r >> 3) * kGroupBytes + (g >> 2) * 1024;
     const int ch = (g & 3) * 2;
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + swz(r, ch)), "r"(hv[0]),
-                 "r"(hv[1]), "r"(hv[2]), "r"(hv[3])
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + swz(r & 7, ch)),
+                 "r"(hv[0]), "r"(hv[1]), "r"(hv[2]), "r"(hv[3])
                  : "memory");
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + swz(r, ch + 1)),
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + swz(r & 7, ch + 1)),
                  "r"(hv[4]), "r"(hv[5]), "r"(hv[6]), "r"(hv[7])
                  : "memory");
   }
@@ -291,6 +300,8 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
     prefetch_tensormap(&tm_q);
     const uint32_t q_bytes = static_cast<uint32_t>(L::kHalves * 128 * s.gs * s.qpt);
     int n = 0, issued = 0;
+    // test hook: every CTA leaves its first tile unissued (see g_debug_lost_load)
+    const int lost = g_debug_lost_load == 1 ? 0 : -1;
     bool ok = true;
     for (int j = 0; ok; ++j) {
       const int ms = j % kMetaSlots;
@@ -315,6 +326,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
         if (!(ok = mbar_wait(empty_bar(st), ((n / STAGES) & 1) ^ 1, kWhereWaitEmpty, abort_flag)))
           break;
         ++issued;
+        if (n == lost) continue;
         const uint32_t kdst = sbase + st * L::kStageBytes;
         const uint32_t vdst = kdst + L::kKVTileBytes;
         if constexpr (KV8) {
@@ -358,6 +370,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       volatile int drain_flag = 0;
       for (int st = 0; st < STAGES && st < issued; ++st) {
         const int last = issued - 1 - ((issued - 1 - st) % STAGES);
+        if (last == lost) continue;  // nothing was issued for it
         if (!mbar_wait(full_bar(st), (last / STAGES) & 1, kWhereWaitFull, &drain_flag)) break;
       }
     }

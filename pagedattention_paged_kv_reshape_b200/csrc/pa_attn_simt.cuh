@@ -9,8 +9,10 @@
 // per tile row in the log2 domain; the epilogue merges the four warps.
 //
 // Lane layout for one block: for scores, lane = 2 * token + half, each lane
-// dots half of head_dim and a shuffle joins the halves; for P.V, lane owns
-// head dims lane, lane + 32, ...
+// dots half of head_dim (loaded 32 elements at a time, so head_dim 256 needs
+// no more registers than 64) and a shuffle joins the halves; for P.V, lane
+// owns head dims lane, lane + 32, ...  The query tile and the merge buffer
+// live in dynamic shared memory (simt_smem_bytes).
 //
 // KV8: the cache holds FP8 e4m3 codes with one fp32 scale per KV head for K
 // and for V; codes are decoded to fp32 as they are loaded, the K scale folds
@@ -21,10 +23,11 @@
 
 namespace pa {
 
-template <typename T, int D>
-__device__ __forceinline__ void load_half_row(const T* __restrict__ src, float (&dst)[D / 2]) {
-  constexpr int kBytes = D / 2 * sizeof(T);
-  static_assert(kBytes % 16 == 0, "row half must be 16-byte vectors");
+// N consecutive elements of a cache row, converted to fp32.
+template <typename T, int N>
+__device__ __forceinline__ void load_row_piece(const T* __restrict__ src, float (&dst)[N]) {
+  constexpr int kBytes = N * sizeof(T);
+  static_assert(kBytes % 16 == 0, "row pieces must be 16-byte vectors");
   const uint4* p = reinterpret_cast<const uint4*>(src);
 #pragma unroll
   for (int c = 0; c < kBytes / 16; ++c) {
@@ -44,13 +47,13 @@ __device__ __forceinline__ void load_half_row(const T* __restrict__ src, float (
   }
 }
 
-template <int D>
-__device__ __forceinline__ void load_half_row(const uint8_t* __restrict__ src,
-                                              float (&dst)[D / 2]) {
-  static_assert(D / 2 % 16 == 0, "row half must be 16-byte vectors");
+template <int N>
+__device__ __forceinline__ void load_row_piece(const uint8_t* __restrict__ src,
+                                               float (&dst)[N]) {
+  static_assert(N % 16 == 0, "row pieces must be 16-byte vectors");
   const uint4* p = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-  for (int c = 0; c < D / 2 / 16; ++c) {
+  for (int c = 0; c < N / 16; ++c) {
     const uint4 w = __ldg(p + c);
     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -69,6 +72,13 @@ __device__ __forceinline__ float fp8_to_f32(uint8_t code) {
   return __half2float(*reinterpret_cast<const __half*>(&h));
 }
 
+// Dynamic shared memory of attn_simt_kernel<.., D, ..>: the query tile
+// [kRows][D] and the four warps' merge buffer [4][kRows][D + 8], fp32.
+template <int D>
+constexpr int simt_smem_bytes() {
+  return (kRows * D + 4 * kRows * (D + 8)) * 4;
+}
+
 template <typename T, int D, bool KV8 = false>
 __global__ void __launch_bounds__(128, 1)
     attn_simt_kernel(Shape s, T* __restrict__ out, const T* __restrict__ q,
@@ -79,11 +89,13 @@ __global__ void __launch_bounds__(128, 1)
                      const float* __restrict__ k_scale, const float* __restrict__ v_scale) {
   constexpr int NW = 4;
   constexpr int HALF = D / 2;
+  constexpr int PIECE = 32;  // K elements a lane holds at a time
   constexpr int PER = D / 32;
-  __shared__ __align__(16) float q_s[kRows][D];
+  extern __shared__ __align__(16) float simt_smem[];
+  auto q_s = reinterpret_cast<float (*)[D]>(simt_smem);                        // [kRows][D]
+  auto co = reinterpret_cast<float (*)[kRows][D + 8]>(simt_smem + kRows * D);  // [NW][kRows][D+8]
   __shared__ float cm[NW * kRows];
   __shared__ float cl[NW * kRows];
-  __shared__ __align__(16) float co[NW][kRows][D + 8];
   __shared__ Unit u_s;
 
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the prep kernel's results
@@ -144,18 +156,31 @@ __global__ void __launch_bounds__(128, 1)
                                    s.num_blocks, u.row)
                          : y0;
       auto row_of = [&](int t) { return static_cast<size_t>(t < 8 ? y0 + t : y1 + t - 8); };
-      float kr[HALF];
-      if constexpr (KV8)
-        load_half_row<D>(k_cache + row_of(tok) * D + half * HALF, kr);
-      else
-        load_half_row<T, D>(k_cache + row_of(tok) * D + half * HALF, kr);
+      // this lane's half of the dot products, one 32-element piece of the key
+      // row at a time (each sum in the order of the head dims)
+      float dot[kRows];
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) dot[r] = 0.f;
+#pragma unroll
+      for (int pc = 0; pc < HALF / PIECE; ++pc) {
+        float kr[PIECE];
+        const size_t at = row_of(tok) * D + half * HALF + pc * PIECE;
+        if constexpr (KV8)
+          load_row_piece<PIECE>(k_cache + at, kr);
+        else
+          load_row_piece<T, PIECE>(k_cache + at, kr);
+#pragma unroll
+        for (int r = 0; r < kRows; ++r)
+          if (r < nrows)
+#pragma unroll
+            for (int e = 0; e < PIECE; ++e)
+              dot[r] = fmaf(q_s[r][half * HALF + pc * PIECE + e], kr[e], dot[r]);
+      }
       const int kidx = blk_start + tok;
 #pragma unroll
       for (int r = 0; r < kRows; ++r) {
         if (r < nrows) {
-          float sc = 0.f;
-#pragma unroll
-          for (int e = 0; e < HALF; ++e) sc = fmaf(q_s[r][half * HALF + e], kr[e], sc);
+          float sc = dot[r];
           sc += __shfl_xor_sync(0xffffffffu, sc, 1);
           const int lim = u.lim0 + r / s.gs;
           const float x = kidx < lim ? sc * sl : -INFINITY;

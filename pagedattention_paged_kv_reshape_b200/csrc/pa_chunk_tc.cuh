@@ -203,6 +203,11 @@ __global__ void __launch_bounds__(320, 1)
       return it;
     };
     bool ok = true;
+    // The last Q, K and V loads issued (a CTA that gives up waits for them
+    // before it exits), and the test hook: every CTA leaves its first K tile
+    // unissued (see g_debug_lost_load).
+    int q_last = -1, k_last = -1, v_last = -1;
+    const int lost = g_debug_lost_load == 2 ? 0 : -1;
     // make item k current: publish its metadata and load its Q
     auto publish = [&](int k, const TcItem& it) -> bool {
       const int qb = k % QS;
@@ -219,7 +224,9 @@ __global__ void __launch_bounds__(320, 1)
                         it.token0);
         }
       }
-      return __shfl_sync(0xffffffffu, r, 0);
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r) q_last = k;
+      return r;
     };
     // V of a tile reuses the block ids its K looked up; at most two tiles
     // wait for their V (the older one is issued right after a new K).
@@ -241,6 +248,7 @@ __global__ void __launch_bounds__(320, 1)
       if (r && lane < p.nb)
         tma_load_4d(v_smem(vs) + lane * (box_rows / 8) * L::kGroupBytes, &tm_v, vfull(vs), 0, 0,
                     0, p.y >> 3);
+      if (r) v_last = p.gt;
       return r;
     };
     int2 ent1 = entry_of(1);
@@ -268,15 +276,16 @@ __global__ void __launch_bounds__(320, 1)
         bool r = true;
         if (lane == 0) {
           r = mbar_wait(kempty(ks), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-          if (r)
+          if (r && gt != lost)
             mbar_arrive_expect_tx(kfull(ks),
                                   static_cast<uint32_t>(nb * L::kHalves * box_rows * 128));
         }
         ok = __shfl_sync(0xffffffffu, r, 0);
         if (!ok) break;
-        if (lane < nb)
+        if (lane < nb && gt != lost)
           tma_load_4d(k_smem(ks) + lane * (box_rows / 8) * L::kGroupBytes, &tm_k, kfull(ks), 0, 0,
                       0, y >> 3);
+        k_last = gt;
         // queue this tile's V; issue the previous tile's
         if (npend == 0) {
           va = Pending{y, nb, gt};
@@ -296,7 +305,18 @@ __global__ void __launch_bounds__(320, 1)
         ok = publish(k, it);
       }
     }
-    if (ok && npend == 1) issue_v(va);  // the last tile's V
+    if (ok && npend == 1) ok = issue_v(va);  // the last tile's V
+    if (!ok && lane == 0) {
+      // A wait gave up: let the copies already issued land before the CTA
+      // exits (each wait bounded again, independently of the abort flag).
+      volatile int own_flag = 0;
+      for (int i = max(0, q_last - QS + 1); i <= q_last; ++i)
+        mbar_wait(qfull(i % QS), (i / QS) & 1, kWhereWaitQ, &own_flag);
+      for (int i = max(0, k_last - KS + 1); i <= k_last; ++i)
+        if (i != lost) mbar_wait(kfull(i % KS), (i / KS) & 1, kWhereWaitFull, &own_flag);
+      for (int i = max(0, v_last - VS + 1); i <= v_last; ++i)
+        mbar_wait(vfull(i % VS), (i / VS) & 1, kWhereWaitFull, &own_flag);
+    }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issue
     // The CTA's tiles form one sequence gt = 0, 1, 2, ... across its items.

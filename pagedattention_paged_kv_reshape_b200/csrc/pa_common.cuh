@@ -111,18 +111,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // this means a lost arrival, never slow memory.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
+// The limit every bounded wait uses (SM cycles).  kWaitLimitCycles unless a
+// test shortened it with pa_debug_lost_load.
+__device__ long long g_wait_limit_cycles = kWaitLimitCycles;
+
+// Test hook, 0 in normal operation (pa_debug_lost_load): 1 makes the load
+// warp of every CTA of attn_mma_kernel, 2 that of chunk_tc_kernel, leave its
+// first K/V tile unissued (no copy and no arrival on its barrier), so the
+// warp that waits for that tile runs into the wait limit.
+__device__ int g_debug_lost_load = 0;
+
 // Wait for the phase with the given parity to complete.  Returns false, after
 // recording PA_ERR_TIMEOUT and raising the CTA's abort flag, if it did not
-// complete within kWaitLimitCycles; returns false at once if another warp of
-// the CTA already raised the flag.  Every wait in these kernels goes through
-// here, so no CTA can wait without bound.
+// complete within g_wait_limit_cycles; returns false at once if another warp
+// of the CTA already raised the flag.  Every wait in these kernels goes
+// through here, so no CTA can wait without bound.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int where,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const long long limit = g_wait_limit_cycles;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       report_error(PA_ERR_TIMEOUT, where, bar, parity);
       *abort_flag = 1;
       return false;

@@ -1,9 +1,9 @@
 """Test plumbing: run the CUDA path and the oracle on the same seeded batch.
 
 The oracle only ever sees host copies of the generator's tensors (never a
-value the CUDA path produced).  For full-size batches the oracle runs on a
-compact copy of a few sampled requests: their blocks are copied out of the
-pool (an exact byte copy) and their block ids renumbered; nothing else moves.
+value the CUDA path produced).  Full-size batches go to ``oracle_full``: the
+batch's tensors are copied once into shared host memory and the plain oracle
+runs on every (request, KV head) sub-problem on all host cores.
 """
 
 from __future__ import annotations
@@ -117,61 +117,6 @@ def oracle_step(b: PagedBatch, varlen: bool | None = None, seqs=None):
     return out, kc, vc
 
 
-def compact(b: PagedBatch, rows) -> dict:
-    """Host copy of requests ``rows`` of a (large) batch with renumbered blocks."""
-    rows = list(rows)
-    tables = b.host_tables[rows]
-    lens = b.host_seq_lens[rows]
-    used = sorted({int(tables[i, j]) for i in range(len(rows))
-                   for j in range(-(-int(lens[i]) // b.block_size))})
-    remap = {old: new for new, old in enumerate(used)}
-    idx = torch.tensor(used, dtype=torch.long, device=b.k_cache.device)
-    kc = host(b.k_cache.index_select(0, idx)) if used else host(b.k_cache[:0])
-    vc = host(b.v_cache.index_select(0, idx)) if used else host(b.v_cache[:0])
-    new_tables = np.zeros_like(tables)
-    for i in range(len(rows)):
-        for j in range(-(-int(lens[i]) // b.block_size)):
-            new_tables[i, j] = remap[int(tables[i, j])]
-    tok = np.concatenate([np.arange(b.host_qsl[r], b.host_qsl[r + 1]) for r in rows]) \
-        if rows else np.zeros(0, np.int64)
-    qsl = np.zeros(len(rows) + 1, np.int32)
-    qsl[1:] = np.cumsum([b.host_qsl[r + 1] - b.host_qsl[r] for r in rows])
-    slots = b.host_slots[tok]
-    new_slots = np.array([remap[int(s) // b.block_size] * b.block_size + int(s) % b.block_size
-                          for s in slots], dtype=np.int32)
-    ti = torch.from_numpy(tok.astype(np.int64)).to(b.q.device)
-    return dict(tokens=tok, tables=new_tables, lens=lens, qsl=qsl, slots=new_slots, kc=kc, vc=vc,
-                q=host(b.q.index_select(0, ti)), k_new=host(b.k_new.index_select(0, ti)),
-                v_new=host(b.v_new.index_select(0, ti)))
-
-
-def oracle_rows(b: PagedBatch, rows, varlen: bool | None = None):
-    """Oracle output (float64) for the query tokens of requests ``rows``."""
-    varlen = (not b.is_decode) if varlen is None else varlen
-    c = compact(b, rows)
-    bs = b.block_size
-    if b.fp8:
-        ks, vs = host(b.k_scale), host(b.v_scale)
-        kc, vc = O.reshape_and_cache_fp8(c["kc"], c["vc"], c["k_new"], c["v_new"], c["slots"],
-                                         ks, vs, b.dtype, block_size=bs)
-        if varlen:
-            out = O.paged_varlen_fp8(c["q"], kc, vc, ks, vs, c["tables"], c["qsl"], c["lens"],
-                                     b.scale, b.dtype, block_size=bs)
-        else:
-            out = O.paged_decode_fp8(c["q"], kc, vc, ks, vs, c["tables"], c["lens"], b.scale,
-                                     b.dtype, block_size=bs)
-        return c["tokens"], out
-    kc, vc = O.reshape_and_cache(c["kc"], c["vc"], c["k_new"], c["v_new"], c["slots"],
-                                 block_size=bs)
-    if varlen:
-        out = O.paged_varlen(c["q"], kc, vc, c["tables"], c["qsl"], c["lens"], b.scale, b.dtype,
-                             block_size=bs)
-    else:
-        out = O.paged_decode(c["q"], kc, vc, c["tables"], c["lens"], b.scale, b.dtype,
-                             block_size=bs)
-    return c["tokens"], out
-
-
 def assert_close(gpu_out: torch.Tensor, ref: np.ndarray, dtype: str, what: str = ""):
     got = f64(gpu_out)
     assert got.shape == ref.shape, (got.shape, ref.shape)
@@ -181,3 +126,41 @@ def assert_close(gpu_out: torch.Tensor, ref: np.ndarray, dtype: str, what: str =
     assert err.max() <= max_tol, f"{what}: max abs err {err.max():.3e} > {max_tol}"
     assert err.mean() <= mean_tol, f"{what}: mean abs err {err.mean():.3e} > {mean_tol}"
     return float(err.max()), float(err.mean())
+
+
+# ---------------------------------------------------------------------------
+# the oracle on every row of a (full-size) batch, on all host cores
+# ---------------------------------------------------------------------------
+
+_NP_OF = {torch.bfloat16: np.int16, torch.float16: np.float16, torch.float32: np.float32,
+          torch.uint8: np.uint8}
+
+
+def _fill_shared(pool, name: str, t: torch.Tensor) -> None:
+    """Copy tensor ``t`` into the pool's shared array ``name`` (bf16 as its
+    16-bit patterns, the oracle's encoding)."""
+    npdt = _NP_OF[t.dtype]
+    arr = pool.array(name, tuple(t.shape), np.uint16 if t.dtype == torch.bfloat16 else npdt)
+    view = arr.view(npdt) if t.dtype == torch.bfloat16 else arr
+    src = t.view(torch.int16) if t.dtype == torch.bfloat16 else t
+    torch.from_numpy(view).copy_(src)
+
+
+def oracle_full(b: PagedBatch, varlen: bool | None = None, workers: int | None = None):
+    """Oracle output (float64, ``[total_q, Hq, D]``) for every query row of
+    ``b``: the batch's input tensors go to shared host memory once and
+    ``oracle.parallel`` solves its (request, KV head) sub-problems on all host
+    cores with the plain oracle functions."""
+    from oracle.parallel import OraclePool
+
+    varlen = (not b.is_decode) if varlen is None else varlen
+    with OraclePool(workers) as pool:
+        for name in ("k_cache", "v_cache", "q", "k_new", "v_new"):
+            _fill_shared(pool, name, getattr(b, name))
+        pool.start(tables=b.host_tables, seq_lens=b.host_seq_lens, qsl=b.host_qsl,
+                   slots=b.host_slots, num_q_heads=b.num_q_heads,
+                   num_kv_heads=b.num_kv_heads, block_size=b.block_size, dtype=b.dtype,
+                   scale=b.scale, varlen=varlen, fp8=b.fp8,
+                   k_scale=None if not b.fp8 else host(b.k_scale),
+                   v_scale=None if not b.fp8 else host(b.v_scale))
+        return pool.solve_batch()

@@ -3,8 +3,8 @@
 Bars: cache writes bit-exact; attention within max-abs 1e-2 / mean-abs 1e-3
 for bf16 and f16 inputs (fp32 accumulation) and 1e-5 for fp32 inputs.
 Small cases span several 16-token blocks and 512-token partitions with ragged
-tails; full-size configurations are checked on sampled requests plus
-properties that hold at any size.  Every call goes through the C ABI.
+tails; the full-size workloads are checked on every row in
+test_gpu_full_size.py.  Every call goes through the C ABI.
 """
 
 import math
@@ -17,7 +17,7 @@ import oracle as O
 import pagedattention_paged_kv_reshape_b200 as pa
 from pagedattention_paged_kv_reshape_b200 import workload as W
 from tests._helpers import (assert_close, f64, gpu_attention, gpu_cache_write, gpu_step, host,
-                            oracle_rows, oracle_step)
+                            oracle_step)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -156,16 +156,16 @@ VARLEN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["auto", "mma", "simt", "pairs"])
+@pytest.mark.parametrize("path", ["auto", "mma", "simt"])
 @pytest.mark.parametrize("case", range(len(VARLEN_CASES)))
 def test_varlen_matches_oracle(case, path):
     rows, hq, hkv, d, dtype = VARLEN_CASES[case]
     if path == "simt":
         pa.pa_set_path(pa.Path.SIMT)
-    elif path in ("mma", "pairs"):
+    elif path == "mma":
         if dtype == "f32":
             pytest.skip("tensor-core paths need 16-bit inputs")
-        pa.pa_set_path(pa.Path.MMA if path == "mma" else pa.Path.TCGEN05_PAIRS)
+        pa.pa_set_path(pa.Path.MMA)
     b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
                       head_dim=d, dtype=dtype, seed=100 + case, device=DEV, pool_factor=1.2)
     out, _, _ = gpu_step(b, varlen=True)
@@ -202,16 +202,16 @@ BLOCK_SIZE_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["auto", "mma", "simt", "pairs"])
+@pytest.mark.parametrize("path", ["auto", "mma", "simt"])
 @pytest.mark.parametrize("case", range(len(BLOCK_SIZE_CASES)))
 def test_block_sizes_match_oracle(case, path):
     rows, hq, hkv, d, dtype, bs = BLOCK_SIZE_CASES[case]
     if path == "simt":
         pa.pa_set_path(pa.Path.SIMT)
-    elif path in ("mma", "pairs"):
+    elif path == "mma":
         if dtype == "f32":
             pytest.skip("tensor-core paths need 16-bit inputs")
-        pa.pa_set_path(pa.Path.MMA if path == "mma" else pa.Path.TCGEN05_PAIRS)
+        pa.pa_set_path(pa.Path.MMA)
     b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
                       head_dim=d, dtype=dtype, seed=300 + case, device=DEV, pool_factor=1.2,
                       block_size=bs)
@@ -230,34 +230,28 @@ def test_block_sizes_match_oracle(case, path):
 
 
 HEAD_DIM_256_CASES = [
-    # head_dim 256 runs on the bf16/f16 tensor-core decode kernel (chunk rows too)
+    # head_dim 256: the tensor-core decode/varlen kernel for 16-bit types (chunk
+    # rows too), the CUDA-core kernel for fp32 and when it is forced
     ([(700, 37), (1, 1), (2000, 1), (600, 160), (9, 9)], 16, 2, "bf16"),    # group 8
     ([(1300, 1), (33, 1), (4096, 1)], 8, 8, "f16"),                          # MHA, split-K
     ([(520, 20), (17, 17), (1025, 1)], 32, 8, "bf16"),                      # group 4
+    ([(700, 1), (40, 9), (1537, 1)], 8, 2, "f32"),                           # fp32
 ]
 
 
+@pytest.mark.parametrize("path", ["auto", "simt"])
 @pytest.mark.parametrize("case", range(len(HEAD_DIM_256_CASES)))
-def test_head_dim_256_matches_oracle(case):
+def test_head_dim_256_matches_oracle(case, path):
     rows, hq, hkv, dtype = HEAD_DIM_256_CASES[case]
+    if path == "simt":
+        pa.pa_set_path(pa.Path.SIMT)
     b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=hq, num_kv_heads=hkv,
                       head_dim=256, dtype=dtype, seed=700 + case, device=DEV, pool_factor=1.2)
     varlen = any(q_ != 1 for _, q_ in rows)
     out, kc, vc = gpu_step(b, varlen=varlen)
     ref, okc, _ = oracle_step(b, varlen=varlen)
     assert np.array_equal(host(kc).view(np.uint8), okc.view(np.uint8))
-    assert_close(out, ref, dtype, f"head_dim 256 case {case}")
-
-
-def test_head_dim_256_refuses_cuda_core_paths():
-    b = decode_batch([100, 40], 8, 2, 256, "bf16", seed=71)
-    kc, vc = gpu_cache_write(b)
-    ws = pa.alloc_workspace(pa.pa_decode_workspace_size(2, 8, 2, 256, 100), DEV)
-    pa.pa_set_path(pa.Path.SIMT)
-    with pytest.raises(pa.PaError) as e:
-        pa.pa_decode(torch.empty_like(b.q), b.q, kc, vc, b.block_tables, b.seq_lens, 100,
-                     b.scale, ws)
-    assert e.value.status == pa.Status.UNSUPPORTED
+    assert_close(out, ref, dtype, f"head_dim 256 case {case} ({path})")
 
 
 # Batches whose longest row has 16 or more 512-key partitions take the wide
@@ -303,10 +297,6 @@ def test_chunk_kernel_agrees_with_decode_kernel_tiles():
     mma = gpu_attention(b, kc, vc, varlen=True)
     assert_close(tc, f64(mma), "bf16", "tcgen05 vs mma tiles")
     assert torch.equal(tc[-1], mma[-1])   # the decode row takes the same kernel on both
-    pa.pa_set_path(pa.Path.TCGEN05_PAIRS)  # two query tiles per chunk item
-    pairs = gpu_attention(b, kc, vc, varlen=True)
-    assert_close(pairs, f64(mma), "bf16", "tcgen05 pairs vs mma tiles")
-    assert torch.equal(pairs[-1], mma[-1])
 
 
 def test_varlen_decode_rows_equal_decode():
@@ -315,35 +305,6 @@ def test_varlen_decode_rows_equal_decode():
     dec = gpu_attention(b, kc, vc, varlen=False)
     var = gpu_attention(b, kc, vc, varlen=True)
     assert torch.equal(dec, var)
-
-
-# ---------------------------------------------------------------------------
-# full-size configurations: sampled requests + any-size properties
-# ---------------------------------------------------------------------------
-
-def sample_rows(b, k=6, seed=0):
-    lens = b.host_seq_lens
-    rng = np.random.default_rng(seed)
-    pick = {int(np.argmin(lens)), int(np.argmax(lens)), b.num_seqs - 1}
-    pick |= set(rng.choice(b.num_seqs, size=min(k, b.num_seqs), replace=False).tolist())
-    return sorted(pick)
-
-
-@pytest.mark.parametrize("name", ["mha_bs64", "gqa_bs256", "long_32k", "mixed_2048"])
-def test_full_config_sampled(name):
-    b = W.make_config(name, seed=0, device=DEV)
-    out, kc, vc = gpu_step(b)
-    assert torch.all(torch.isfinite(out)), "every output row is written and finite"
-    # the cache write landed exactly: written rows equal the new rows, bit for bit
-    slots = b.slot_mapping.long()
-    blk, off = slots // 16, slots % 16
-    assert torch.equal(kc[blk, :, off, :].view(torch.int16), b.k_new.view(torch.int16))
-    assert torch.equal(vc[blk, :, off, :].view(torch.int16), b.v_new.view(torch.int16))
-    rows = sample_rows(b)
-    tokens, ref = oracle_rows(b, rows)
-    assert_close(out[torch.from_numpy(tokens).to(DEV)], ref, b.dtype, name)
-    del kc, vc, out, b
-    torch.cuda.empty_cache()
 
 
 # ---------------------------------------------------------------------------

@@ -88,4 +88,4 @@ def test_reference_arm_rank0_prints_the_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"] == "mha_bs64"
+    assert d["config"]["workload"] == "mixed_2048"

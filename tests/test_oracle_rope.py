@@ -92,8 +92,26 @@ def pin_cache_write():
     np.testing.assert_allclose(qr[1], OR.rotate(q[1].astype(np.float64), table[41], R, True))
 
 
+def pin_table_values():
+    """The angle table of RoFormer: pair i of a rot_dim-dim rotation turns by
+    p * base^(-2i/rot_dim) at position p.  Values fixed by the mathematics:
+    row 0 is (cos 0, sin 0) = (1, 0); pair 0 has frequency 1, so row 1 holds
+    (cos 1, sin 1) = (0.5403023058681398, 0.8414709848078965); with rot_dim 4
+    and base 10000 pair 1 has frequency 10000^(-1/2) = 0.01, so at position
+    100 it too is turned by exactly one radian; and cos^2 + sin^2 = 1."""
+    t = OR.rope_table(128, 4)
+    assert t.shape == (128, 4)
+    assert np.array_equal(t[0], [1.0, 1.0, 0.0, 0.0])
+    assert t[1, 0] == pytest.approx(0.5403023058681398, abs=1e-15)
+    assert t[1, 2] == pytest.approx(0.8414709848078965, abs=1e-15)
+    assert t[100, 1] == pytest.approx(0.5403023058681398, abs=1e-13)
+    assert t[100, 3] == pytest.approx(0.8414709848078965, abs=1e-13)
+    big = OR.rope_table(300, 64)
+    np.testing.assert_allclose(big[:, :32] ** 2 + big[:, 32:] ** 2, 1.0, atol=1e-14)
+
+
 ALL_PINS = [pin_identity_and_norm, pin_known_angle, pin_relative_position, pin_layouts_agree,
-            pin_cache_write]
+            pin_cache_write, pin_table_values]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -123,9 +141,17 @@ def _mut_no_rot_dim(x64, row, rot_dim, neox):
     return _orig_rotate(x64, full, d, neox)
 
 
-@pytest.mark.parametrize("name", ["sign", "cross", "position", "rot_dim"])
+def _mut_table(max_position, rot_dim, base=10000.0):
+    inv = base ** (-np.arange(0, rot_dim // 2, dtype=np.float64) / rot_dim)  # exponent halved
+    ang = np.arange(max_position, dtype=np.float64)[:, None] * inv[None, :]
+    return np.concatenate([np.cos(ang), np.sin(ang)], axis=1)
+
+
+@pytest.mark.parametrize("name", ["sign", "cross", "position", "rot_dim", "table"])
 def test_pins_catch_planted_mistake(name, monkeypatch):
-    if name == "sign":
+    if name == "table":
+        monkeypatch.setattr(OR, "rope_table", _mut_table)
+    elif name == "sign":
         monkeypatch.setattr(OR, "rotate", _mut_sign)
     elif name == "cross":
         monkeypatch.setattr(OR, "rotate", _mut_cross)
