@@ -17,6 +17,7 @@
 #include "pa_attn_simt.cuh"
 #include "pa_blocks.cuh"
 #include "pa_chunk_tc.cuh"
+#include "pa_chunk_tc2.cuh"
 #include "pa_reduce.cuh"
 
 #include "pa_reshape.cuh"
@@ -380,8 +381,8 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
 
 template <typename T, int D>
 pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
-  using L = pa::TcLayout<D>;
-  auto kern = pa::chunk_tc_kernel<T, D>;
+  using L = pa::Tc2Layout<D>;
+  auto kern = pa::chunk_tc2_kernel<T, D>;
   int occ = 0;
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "chunk kernel set-up");
@@ -516,7 +517,7 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
                      ? p.chunk_qt
                      : 0;
   p.s.chunk_cap = static_cast<int>(p.chunk_cap);
-  p.s.chunk_span = p.s.chunk_qt;
+  p.s.chunk_span = 2 * p.s.chunk_qt;  // a chunk item holds two query tiles
   switch (a.dtype) {
     case PA_BF16: return run_typed<__nv_bfloat16>(a, p, use_mma);
     case PA_F16: return run_typed<__half>(a, p, use_mma);
