@@ -110,7 +110,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-    INTERVAL_MS = 50
+    INTERVAL_MS = 20
 
     def __init__(self, uuid: str):
         self.uuid = uuid.lower().replace("gpu-", "")
@@ -313,11 +313,20 @@ def timed_loop(torch, fn, n: int, warmup: int = 3) -> float:
     return s.elapsed_time(e) / n
 
 
+# Idle time before each timed loop.  Under a sustained full-bandwidth load the
+# B200 reaches its power cap within about 50 ms and slows by a few percent
+# (the largest batch's back-to-back calls went from 1.96 to 2.2 ms over 0.7 s);
+# a short rest before every loop gives each the same starting point, so the
+# attention call and the whole step are timed under the same conditions.
+REST_S = 1.0
+
+
 def measure_workload(torch, pa, b, steps: int, warmup: int, sampler=None):
     """(step ms, attention-call ms, cache-write ms): K steps (cache write +
     attention) between two events after W warm-up steps, then the attention
-    call alone and the cache write alone, each in its own loop of K calls.
-    Every input is larger than the L2 except the cache write's few MB."""
+    call alone and the cache write alone, each in its own loop of K calls,
+    each loop after REST_S of idle time.  Every input is larger than the L2
+    except the cache write's few MB."""
     out = torch.empty_like(b.q)
     ws = workspace_for(pa, b)
 
@@ -335,12 +344,15 @@ def measure_workload(torch, pa, b, steps: int, warmup: int, sampler=None):
         step()
     pa.pa_get_device_error()
     torch.cuda.synchronize()
+    time.sleep(REST_S)
     if sampler:
         sampler.mark("timed_start")
     step_ms = timed_loop(torch, step, steps, warmup=0)
     if sampler:
         sampler.mark("timed_end")
-    attn_ms = timed_loop(torch, attend, steps)
+    time.sleep(REST_S)
+    attn_ms = timed_loop(torch, attend, steps, warmup=1)
+    time.sleep(REST_S)
     write_ms = timed_loop(torch, write, steps)
     pa.pa_get_device_error()
     return step_ms, attn_ms, write_ms
@@ -552,6 +564,7 @@ def run_ours(args):
         dist.all_reduce(attn_t, op=dist.ReduceOp.MAX)
     attn_ms = attn_t.item()
 
+    time.sleep(REST_S)
     e2e_ms, h2d, d2h = time_e2e(torch, pa, b, args.e2e_steps)
     e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
