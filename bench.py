@@ -62,6 +62,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="CPU-seconds of oracle work in the cpu_baseline sample")
+    ap.add_argument("--requests", type=int, default=0,
+                    help="keep only the first N decode requests of the workload (its chunk rows "
+                         "stay): a smaller case of the same recipe, e.g. for profiler captures")
+    ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
@@ -76,8 +80,8 @@ def measured_peaks():
 
 
 # Sources the attention kernels are compiled from (traffic records are keyed to them).
-ATTENTION_SOURCES = ("pa_common.cuh", "pa_sched.cuh", "pa_attn_mma.cuh", "pa_chunk_tc.cuh",
-                     "pa_tcgen05.cuh", "pa_reduce.cuh")
+ATTENTION_SOURCES = ("pa_common.cuh", "pa_sched.cuh", "pa_attn_mma.cuh",
+                     "pa_chunk_tc2.cuh", "pa_tcgen05.cuh", "pa_reduce.cuh", "pa_api.cu")
 
 
 def kernel_source_hash() -> str:
@@ -519,6 +523,19 @@ def per_config_entry(A, b, step_ms, attn_ms, write_ms, peak, tensor_peak) -> dic
     return ent
 
 
+def make_batch(W, workload: str, seed: int, device, requests: int = 0):
+    """The named workload, or (requests > 0) a smaller case of its recipe: its
+    first `requests` decode requests plus all its chunk rows."""
+    if requests <= 0:
+        return W.make_config(workload, seed=seed, device=device)
+    spec = dict(W.CONFIGS[workload])
+    reqs = spec.pop("requests")(seed)
+    spec.pop("kind")
+    spec.pop("about")
+    keep = [r for r in reqs if r.q_len <= 1][:requests] + [r for r in reqs if r.q_len > 1]
+    return W.build_batch(keep, seed=seed, device=device, name=f"{workload}[:{requests}]", **spec)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -545,7 +562,7 @@ def run_ours(args):
 
     dev = torch.device("cuda", local)
     peak, tensor_peak, peak_kind = measured_peaks()
-    b = W.make_config(args.workload, seed=args.seed + rank, device=dev)
+    b = make_batch(W, args.workload, args.seed + rank, dev, args.requests)
     acc = A.attention_bytes(b)
     step_bytes = acc["total"] + A.reshape_bytes(b)
 
@@ -565,7 +582,8 @@ def run_ours(args):
     attn_ms = attn_t.item()
 
     time.sleep(REST_S)
-    e2e_ms, h2d, d2h = time_e2e(torch, pa, b, args.e2e_steps)
+    e2e_ms, h2d, d2h = (float("nan"), 0, 0) if args.no_e2e else time_e2e(torch, pa, b,
+                                                                       args.e2e_steps)
     e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(e2e, op=dist.ReduceOp.MAX)
@@ -587,7 +605,9 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": b.dtype,
         "data": "synthetic (seeded N(0,1) q/k/v, shuffled block pool, NaN-poisoned padding)",
-        "config": {"workload": args.workload, "about": W.CONFIGS[args.workload]["about"],
+        "config": {"workload": args.workload if args.requests <= 0 else
+                   f"{args.workload} (first {args.requests} decode requests)",
+                   "about": W.CONFIGS[args.workload]["about"],
                    "num_seqs": b.num_seqs, "total_q": b.total_q,
                    "kv_tokens": int(b.host_seq_lens.sum()),
                    "pool_bytes": 2 * b.k_cache.numel() * b.k_cache.element_size(),
@@ -601,7 +621,7 @@ def run_ours(args):
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": recorded_traffic(args.workload),
                      "kernel": ("one pa_varlen call (schedule_kernel + attn_mma_kernel + "
-                                "chunk_tc_kernel + reduce_kernel)" if not b.is_decode else
+                                "chunk_tc2_kernel + reduce_kernel)" if not b.is_decode else
                                 "one pa_decode call (schedule_kernel + attn_mma_kernel "
                                 "[+ reduce_kernel])"),
                      "timing": f"CUDA events on the launching stream around a loop of "

@@ -16,7 +16,6 @@
 #include "pa_attn_mma.cuh"
 #include "pa_attn_simt.cuh"
 #include "pa_blocks.cuh"
-#include "pa_chunk_tc.cuh"
 #include "pa_chunk_tc2.cuh"
 #include "pa_reduce.cuh"
 

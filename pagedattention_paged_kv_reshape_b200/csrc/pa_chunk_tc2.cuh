@@ -16,19 +16,19 @@
 //   O_B [384,384+D).  P is written over the first 64 columns of its S
 //   (16-bit pairs); the P.V MMA reads it from there as its A operand, and
 //   the next S of that tile is issued after that P.V, in order.
-// * warp 8 loads the K and V tiles of the CTA's items (one 4-D box of all
+// * warp 0 loads the K and V tiles of the CTA's items (one 4-D box of all
 //   halves per 16 keys, or per 8-token block) into a K ring and a V ring; V
-//   trails K by one tile.  Warp 10 loads Q_A and Q_B (one 3-D TMA box per
+//   trails K by one tile.  Warp 2 loads Q_A and Q_B (one 3-D TMA box per
 //   64-dim half) of each item as soon as the last S of the previous item that
 //   read them has completed, so the K/V stream never waits for Q.
-// * warp 9 issues the MMAs in the order S_A(t+1), P.V_B(t), S_B(t+1),
-//   P.V_A(t+1), ...: while softmax A works on S_A the tensor core runs
-//   P.V_B and S_B, and the other way round.
-// * warps 0-3 (tile A) and 4-7 (tile B): one thread per tile row (TMEM lane)
+// * one thread of warp 1 issues the MMAs in the order P.V_A(t), S_A(t+1),
+//   P.V_B(t), S_B(t+1), ...: while softmax A works on S_A the tensor core
+//   runs P.V_B and S_B, and the other way round.
+// * warps 4-7 (tile A) and 8-11 (tile B): one thread per tile row (TMEM lane)
 //   reads the row's 128 scores, takes the masked maximum (key <= position),
-//   writes P rounded to the input type, and keeps the row sum of the rounded
-//   P.  The reference maximum that P is taken against is raised only when the
-//   row maximum grows past it by more than 2^8; only then is the row's O
+//   writes P rounded to the input type, and keeps the row sum of P.  The
+//   reference maximum that P is taken against is raised only when the row
+//   maximum grows past it by more than 2^8; only then is the row's O
 //   rescaled in TMEM, after the previous P.V of that tile has completed.  At
 //   the end of the item the thread reads its O row once, divides by the sum
 //   and stores it.
@@ -48,9 +48,14 @@
 
 #include <type_traits>
 
-#include "pa_chunk_tc.cuh"
+#include "pa_sched.cuh"
+#include "pa_tcgen05.cuh"
 
 namespace pa {
+
+constexpr int kTcRows = 128;       // query-tile rows = TMEM lanes
+constexpr int kTcKeys = 128;       // keys per K/V tile = 8 blocks of 16
+constexpr float kTcRescale = 8.f;  // raise the reference maximum past this (log2 units)
 
 // Half of the softmax exponentials on the FMA pipe (exp2_poly2) instead of
 // the special-function unit.

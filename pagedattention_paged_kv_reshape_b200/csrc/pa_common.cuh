@@ -116,7 +116,7 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 __device__ long long g_wait_limit_cycles = kWaitLimitCycles;
 
 // Test hook, 0 in normal operation (pa_debug_lost_load): 1 makes the load
-// warp of every CTA of attn_mma_kernel, 2 that of chunk_tc_kernel, leave its
+// warp of every CTA of attn_mma_kernel, 2 that of chunk_tc2_kernel, leave its
 // first K/V tile unissued (no copy and no arrival on its barrier), so the
 // warp that waits for that tile runs into the wait limit.
 __device__ int g_debug_lost_load = 0;

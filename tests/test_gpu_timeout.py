@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("kernel", [1, 2], ids=["attn_mma_kernel", "chunk_tc_kernel"])
+@pytest.mark.parametrize("kernel", [1, 2], ids=["attn_mma_kernel", "chunk_tc2_kernel"])
 def test_lost_load_times_out_and_next_call_is_clean(kernel):
     if kernel == 1:   # decode rows: the TMA + mma.sync attention kernel
         b = W.build_batch([W.Request(L) for L in (700, 40, 1500)], num_q_heads=32,
