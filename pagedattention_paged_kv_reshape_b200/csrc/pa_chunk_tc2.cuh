@@ -57,9 +57,9 @@ constexpr int kTcRows = 128;       // query-tile rows = TMEM lanes
 constexpr int kTcKeys = 128;       // keys per K/V tile = 8 blocks of 16
 constexpr float kTcRescale = 8.f;  // raise the reference maximum past this (log2 units)
 
-// Half of the softmax exponentials on the FMA pipe (exp2_poly2) instead of
-// the special-function unit.
-constexpr bool kPolyExp = false;
+// Pairs of softmax exponentials, of every 8, computed on the FMA pipe
+// (exp2_poly2) instead of the special-function unit.
+constexpr int kPolyPairs = 0;
 
 template <int D>
 struct Tc2Layout {
@@ -95,6 +95,15 @@ struct Tc2Layout {
   // warps 0: K/V loads, 1: MMA issue, 2: Q loads, 3: idle, 4-7: softmax of
   // tile A, 8-11: softmax of tile B
   static constexpr int kThreads = 384;
+  // Registers per thread after the split (setmaxnreg): the 128 threads of
+  // warps 0-3 give up what the 256 softmax threads take.  Launched with 168
+  // (65,536 / 384, rounded down to 8): 128 x 80 + 256 x 208 = 63,488 of the
+  // 64,512 the block holds.
+  static constexpr int kRegsLaunch = 168;
+  static constexpr int kRegsIssue = 80;
+  static constexpr int kRegsSoftmax = 208;
+  static_assert(128 * kRegsIssue + 256 * kRegsSoftmax <= kThreads * kRegsLaunch,
+                "register split within the block's allocation");
   static constexpr uint32_t kTmemCols = 512;
   static_assert(D == 64 || D == 128, "two O accumulators of D columns next to two S");
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffBar % 1024 == 0, "1 KB alignment");
@@ -206,381 +215,410 @@ __global__ void __launch_bounds__(384, 1)
     return tc2_item(s, w, qsl, seq_lens, count, static_cast<int>(blockIdx.x) + k * gridDim.x, qt);
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------- K / V loads
-    const int box_rows = min(s.block_size, kBlock);  // rows of one K/V TMA box
-    bool ok = true;
-    // The last K and V loads issued, for the drain of a CTA that gives up, and
-    // the test hook: every CTA leaves its first K tile unissued (see
-    // g_debug_lost_load).
-    int k_last = -1, v_last = -1;
-    const int lost = g_debug_lost_load == 2 ? 0 : -1;
-    struct Pending {
-      int y, nb, gt;
-    };
-    Pending va{0, 0, 0}, vb{0, 0, 0};
-    int npend = 0;
-    auto issue_v = [&](const Pending& p) -> bool {
-      const int vs = p.gt % VS;
-      bool r = true;
-      if (lane == 0) {
-        r = mbar_wait(vempty(vs), ((p.gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-        if (r)
-          mbar_arrive_expect_tx(vfull(vs),
-                                static_cast<uint32_t>(p.nb * L::kHalves * box_rows * 128));
-      }
-      r = __shfl_sync(0xffffffffu, r, 0);
-      if (r && lane < p.nb)
-        tma_load_4d(v_smem(vs) + lane * (box_rows / 8) * L::kGroupBytes, &tm_v, vfull(vs), 0, 0,
-                    0, p.y >> 3);
-      if (r) v_last = p.gt;
-      return r;
-    };
-    Tc2Item it{};
-    if (my_items > 0) it = item_of(0);
-    Tc2Item nxt = it;
-    if (my_items > 1) nxt = item_of(1);
-    int g = 0;  // K/V tiles of earlier items
-    for (int k = 0; k < my_items && ok; ++k) {
-      for (int t = 0; t < it.nkt && ok; ++t) {
-        const int gt = g + t, ks = gt % KS;
-        // one lane per TMA box of the tile (box = 16 rows, or 8 rows with
-        // 8-token blocks): its cache row, then its K boxes
-        const int key0 = t * kTcKeys;
-        const int nb = min(kTcKeys / box_rows, ceil_div(it.kv_end - key0, box_rows));
-        int y = 0;
-        if (lane < nb)
-          y = key_row(block_tables + static_cast<size_t>(it.row) * s.table_stride,
-                      key0 + lane * box_rows, s.block_size, s.num_kv_heads, it.kvh, s.num_blocks,
-                      it.row);
+  if (warp < 4) {
+    // load, MMA-issue and Q warps: they need few registers, and the softmax
+    // warpgroups take the rest (a row of scores, P and their sums)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(L::kRegsIssue));
+    if (warp == 0) {
+      // ------------------------------------------------------- K / V loads
+      const int box_rows = min(s.block_size, kBlock);  // rows of one K/V TMA box
+      bool ok = true;
+      // The last K and V loads issued, for the drain of a CTA that gives up, and
+      // the test hook: every CTA leaves its first K tile unissued (see
+      // g_debug_lost_load).
+      int k_last = -1, v_last = -1;
+      const int lost = g_debug_lost_load == 2 ? 0 : -1;
+      struct Pending {
+        int y, nb, gt;
+      };
+      Pending va{0, 0, 0}, vb{0, 0, 0};
+      int npend = 0;
+      auto issue_v = [&](const Pending& p) -> bool {
+        const int vs = p.gt % VS;
         bool r = true;
         if (lane == 0) {
-          r = mbar_wait(kempty(ks), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
-          if (r && gt != lost)
-            mbar_arrive_expect_tx(kfull(ks),
-                                  static_cast<uint32_t>(nb * L::kHalves * box_rows * 128));
+          r = mbar_wait(vempty(vs), ((p.gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+          if (r)
+            mbar_arrive_expect_tx(vfull(vs),
+                                  static_cast<uint32_t>(p.nb * L::kHalves * box_rows * 128));
         }
-        ok = __shfl_sync(0xffffffffu, r, 0);
-        if (!ok) break;
-        if (lane < nb && gt != lost)
-          tma_load_4d(k_smem(ks) + lane * (box_rows / 8) * L::kGroupBytes, &tm_k, kfull(ks), 0, 0,
-                      0, y >> 3);
-        k_last = gt;
-        // queue this tile's V; issue the previous tile's
-        if (npend == 0) {
-          va = Pending{y, nb, gt};
-          npend = 1;
-        } else {
-          vb = Pending{y, nb, gt};
-          ok = issue_v(va);
-          va = vb;
+        r = __shfl_sync(0xffffffffu, r, 0);
+        if (r && lane < p.nb)
+          tma_load_4d(v_smem(vs) + lane * (box_rows / 8) * L::kGroupBytes, &tm_v, vfull(vs), 0, 0,
+                      0, p.y >> 3);
+        if (r) v_last = p.gt;
+        return r;
+      };
+      Tc2Item it{};
+      if (my_items > 0) it = item_of(0);
+      Tc2Item nxt = it;
+      if (my_items > 1) nxt = item_of(1);
+      int g = 0;  // K/V tiles of earlier items
+      for (int k = 0; k < my_items && ok; ++k) {
+        for (int t = 0; t < it.nkt && ok; ++t) {
+          const int gt = g + t, ks = gt % KS;
+          // one lane per TMA box of the tile (box = 16 rows, or 8 rows with
+          // 8-token blocks): its cache row, then its K boxes
+          const int key0 = t * kTcKeys;
+          const int nb = min(kTcKeys / box_rows, ceil_div(it.kv_end - key0, box_rows));
+          int y = 0;
+          if (lane < nb)
+            y = key_row(block_tables + static_cast<size_t>(it.row) * s.table_stride,
+                        key0 + lane * box_rows, s.block_size, s.num_kv_heads, it.kvh, s.num_blocks,
+                        it.row);
+          bool r = true;
+          if (lane == 0) {
+            r = mbar_wait(kempty(ks), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+            if (r && gt != lost)
+              mbar_arrive_expect_tx(kfull(ks),
+                                    static_cast<uint32_t>(nb * L::kHalves * box_rows * 128));
+          }
+          ok = __shfl_sync(0xffffffffu, r, 0);
+          if (!ok) break;
+          if (lane < nb && gt != lost)
+            tma_load_4d(k_smem(ks) + lane * (box_rows / 8) * L::kGroupBytes, &tm_k, kfull(ks), 0, 0,
+                        0, y >> 3);
+          k_last = gt;
+          // queue this tile's V; issue the previous tile's
+          if (npend == 0) {
+            va = Pending{y, nb, gt};
+            npend = 1;
+          } else {
+            vb = Pending{y, nb, gt};
+            ok = issue_v(va);
+            va = vb;
+          }
+        }
+        g += it.nkt;
+        it = nxt;
+        if (k + 2 < my_items) nxt = item_of(k + 2);
+      }
+      if (ok && npend == 1) ok = issue_v(va);  // the last tile's V
+      if (!ok && lane == 0) {
+        // A wait gave up: let the copies already issued land before the CTA
+        // exits (each wait bounded again, independently of the abort flag).
+        volatile int own_flag = 0;
+        for (int i = max(0, k_last - KS + 1); i <= k_last; ++i)
+          if (i != lost) mbar_wait(kfull(i % KS), (i / KS) & 1, kWhereWaitFull, &own_flag);
+        for (int i = max(0, v_last - VS + 1); i <= v_last; ++i)
+          mbar_wait(vfull(i % VS), (i / VS) & 1, kWhereWaitFull, &own_flag);
+      }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------ Q loads
+      // Item k's metadata goes to its slot, then its Q_A and Q_B tiles come in
+      // as soon as the last S of item k - 1 that read each buffer has completed.
+      if (lane == 0) {
+        int q_last = -1;
+        bool ok = true;
+        Tc2Item nxt{};
+        if (my_items > 0) nxt = item_of(0);
+        for (int k = 0; k < my_items && ok; ++k) {
+          const Tc2Item it = nxt;
+          if (k + 1 < my_items) nxt = item_of(k + 1);
+          *item_slot(k) = it;
+  #pragma unroll
+          for (int x = 0; x < 2 && ok; ++x) {
+            ok = mbar_wait(qfree(x), (k & 1) ^ 1, kWhereWaitQ, abort_flag);
+            if (!ok) break;
+            mbar_arrive_expect_tx(qfull(x), static_cast<uint32_t>(L::kTileBytes));
+  #pragma unroll
+            for (int h = 0; h < L::kHalves; ++h)
+              tma_load_3d(q_smem(x) + h * L::kHalfBytes, &tm_q, qfull(x), h * 64, it.head0,
+                          it.token0 + x * qt);
+          }
+          if (ok) q_last = k;
+        }
+        if (!ok && q_last >= 0) {
+          // a wait gave up: let the Q copies already issued land
+          volatile int own_flag = 0;
+          mbar_wait(qfull(0), q_last & 1, kWhereWaitQ, &own_flag);
+          mbar_wait(qfull(1), q_last & 1, kWhereWaitQ, &own_flag);
         }
       }
-      g += it.nkt;
-      it = nxt;
-      if (k + 2 < my_items) nxt = item_of(k + 2);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issue
+      // One thread.  Two cursors walk the CTA's (item, key tile) sequence, the S
+      // cursor one tile ahead of the P.V cursor.  Per step: P.V_A(cp), S_A(cs),
+      // P.V_B(cp), S_B(cs).  S_x(cs) overwrites the columns P.V_x(cp) reads P
+      // from; it is issued after that P.V, and the tensor core executes them in
+      // order.  The step's V tile (and its padding rows) and K tile are waited
+      // for before its first P: they arrive well ahead of it, and once a P is
+      // written only the issue of its MMAs stands between it and the tensor
+      // core.  (The other lanes go straight to the teardown barrier: this warp
+      // shares its SM sub-partition with two softmax warps, and every
+      // instruction it saves shortens the tensor core's idle gaps.)
+      if (lane == 0) {
+        struct Cursor {
+          int k, t, nkt, nkt_a, kv_end_a, kv_end;
+          int ks, kph, vs, vph;  // K and V ring stage of the tile, and its phase parity
+        };
+        auto load_item = [&](Cursor& c, bool wait_q) -> bool {
+          if (c.k >= my_items) return true;
+          if (wait_q && !mbar_wait(qfull(0), c.k & 1, kWhereWaitQ, abort_flag)) return false;
+          const Tc2Item* it = item_slot(c.k);
+          c.nkt = it->nkt;
+          c.nkt_a = it->nkt_a;
+          c.kv_end_a = it->kv_end_a;
+          c.kv_end = it->kv_end;
+          return true;
+        };
+        auto advance = [&](Cursor& c) -> bool {  // true when it moved on to the next item
+          if (++c.ks == KS) {
+            c.ks = 0;
+            c.kph ^= 1;
+          }
+          if (++c.vs == VS) {
+            c.vs = 0;
+            c.vph ^= 1;
+          }
+          if (++c.t < c.nkt) return false;
+          c.t = 0;
+          ++c.k;
+          return true;
+        };
+        // S_x of the S cursor's tile (its K tile, and for x = 1 its Q_B, waited for)
+        auto issue_s = [&](const Cursor& c, int x) {
+          // (no tcgen05 fence here: the softmax threads' last reads of S_x were
+          // ordered before this thread's tcgen05 operations by the fence after
+          // its wait on their P, earlier in this thread's program order)
+          const uint64_t qd = smem_desc_sw128(q_smem(x), 16, 1024);
+          const uint64_t kd = smem_desc_sw128(k_smem(c.ks), 16, L::kGroupBytes);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // descriptor start addresses advance in 16-byte units
+            const uint64_t qoff = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
+            const uint64_t koff = ((kk >> 2) * 1024 + (kk & 3) * 32) >> 4;
+            umma_ss(t_s(x), qd + qoff, kd + koff, kIdescS, kk > 0);
+          }
+          umma_commit(sfull(x));
+          if (c.t == (x == 0 ? c.nkt_a : c.nkt) - 1) umma_commit(qfree(x));
+          if (x == 1) umma_commit(kempty(c.ks));  // both tiles' S of this K tile issued
+        };
+        // P.V_x of the P.V cursor's tile, once P_x is written (its V tile waited for)
+        auto issue_pv = [&](const Cursor& c, int x, int nx) -> bool {
+          if (!mbar_wait(pfull(x), nx & 1, kWhereWaitMma, abort_flag)) return false;
+          tc_fence_after();
+          const int valid = min(kTcKeys, (x == 0 ? c.kv_end_a : c.kv_end) - c.t * kTcKeys);
+          const int steps = (valid + 15) >> 4;  // 16-key MMA steps holding visible keys
+          const uint64_t vd = smem_desc_sw128(v_smem(c.vs), 1024, L::kGroupBytes);
+          const uint32_t acc0 = c.t > 0 ? 1u : 0u;  // the item's first tile starts O afresh
+  #pragma unroll
+          for (int kk = 0; kk < kTcKeys / 16; ++kk)
+            umma_ts(t_o(x), t_s(x) + kk * 8, vd + ((kk * 2 * L::kGroupBytes) >> 4), kIdescPV,
+                    kk > 0 ? 1u : acc0, kk < steps);
+          umma_commit(pdone(x));
+          if (x == 1) umma_commit(vempty(c.vs));  // both tiles' P.V of this V tile issued
+          return true;
+        };
+        // The step's V tile has landed; for the item's last tile, zero the rows
+        // of its last 16-key step past the item's last key (padding slots, or
+        // rows no box covered) before any P.V reads them.
+        auto v_ready = [&](const Cursor& c) -> bool {
+          if (!mbar_wait(vfull(c.vs), c.vph, kWhereWaitFull, abort_flag)) return false;
+          if (c.t == c.nkt - 1) {
+            const int key0 = c.t * kTcKeys;
+            const int last = min(kTcKeys, c.kv_end - key0);
+            const int pad1 = min(kTcKeys, (last + 15) & ~15);
+            for (int row = last; row < pad1; ++row) {
+              uint8_t* dst = smem + L::kOffV + c.vs * L::kTileBytes + (row >> 3) * L::kGroupBytes +
+                             (row & 7) * 128;
+  #pragma unroll
+              for (int h = 0; h < L::kHalves; ++h)
+  #pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                  *reinterpret_cast<uint4*>(dst + h * 1024 + ch * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
+          return true;
+        };
+        Cursor cs{}, cp{};
+        int na = 0, nb = 0;  // P.V issued so far for tile A and tile B
+        bool ok = my_items > 0 && load_item(cs, true);
+        if (ok) {  // S of the first tile
+          ok = mbar_wait(kfull(cs.ks), cs.kph, kWhereWaitFull, abort_flag) &&
+               mbar_wait(qfull(1), 0, kWhereWaitQ, abort_flag);
+          if (ok) {
+            issue_s(cs, 0);
+            issue_s(cs, 1);
+          }
+        }
+        if (ok && advance(cs)) ok = load_item(cs, true);
+        if (ok) ok = load_item(cp, false);  // the S cursor has waited for item 0's Q
+        while (ok && cp.k < my_items) {
+          const bool has_a = cp.t < cp.nkt_a;
+          const bool s_next = cs.k < my_items;
+          ok = v_ready(cp) &&
+               (!s_next || mbar_wait(kfull(cs.ks), cs.kph, kWhereWaitFull, abort_flag));
+          if (ok && has_a) ok = issue_pv(cp, 0, na);
+          if (!ok) break;
+          na += has_a;
+          if (s_next && cs.t < cs.nkt_a) issue_s(cs, 0);
+          ok = issue_pv(cp, 1, nb);
+          if (!ok) break;
+          ++nb;
+          if (s_next) {  // tile B's Q of a new item
+            if (cs.t == 0) ok = mbar_wait(qfull(1), cs.k & 1, kWhereWaitQ, abort_flag);
+            if (!ok) break;
+            issue_s(cs, 1);
+          }
+          if (advance(cs)) ok = load_item(cs, true);
+          if (ok && advance(cp)) ok = load_item(cp, false);  // the S cursor is past it already
+        }
+        // no MMA of this CTA may still run when TMEM is freed
+        umma_commit(drain);
+        volatile int own_flag = 0;
+        mbar_wait(drain, 0, kWhereWaitMma, &own_flag);
+      }
     }
-    if (ok && npend == 1) ok = issue_v(va);  // the last tile's V
-    if (!ok && lane == 0) {
-      // A wait gave up: let the copies already issued land before the CTA
-      // exits (each wait bounded again, independently of the abort flag).
-      volatile int own_flag = 0;
-      for (int i = max(0, k_last - KS + 1); i <= k_last; ++i)
-        if (i != lost) mbar_wait(kfull(i % KS), (i / KS) & 1, kWhereWaitFull, &own_flag);
-      for (int i = max(0, v_last - VS + 1); i <= v_last; ++i)
-        mbar_wait(vfull(i % VS), (i / VS) & 1, kWhereWaitFull, &own_flag);
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ Q loads
-    // Item k's metadata goes to its slot, then its Q_A and Q_B tiles come in
-    // as soon as the last S of item k - 1 that read each buffer has completed.
-    if (lane == 0) {
-      int q_last = -1;
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(L::kRegsSoftmax));
+    {
+      // ------------------------------------------------------- softmax warps
+      const int x = (warp - 4) >> 2;                        // 0: tile A, 1: tile B
+      const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const int r = (warp & 3) * 32 + lane;                 // tile row = TMEM lane
+      const int i = r / s.gs, gi = r % s.gs;
+      // Scores enter as x = s * |scale| after a sign flip of s for a negative
+      // scale, so that the row maximum is always a max.  Masked keys hold
+      // -inf, which the exponent turns into 0; a zero scale is taken as
+      // 2^-100 so that -inf * scale stays -inf (every visible x is then 0 to
+      // within fp32, as with the zero scale).
+      const bool neg = scale_log2 < 0.f;
+      const float sc = fmaxf(fabsf(scale_log2), 7.8886091e-31f);
+      int nx = 0;  // tiles of this query tile processed so far (P written)
       bool ok = true;
       Tc2Item nxt{};
       if (my_items > 0) nxt = item_of(0);
       for (int k = 0; k < my_items && ok; ++k) {
+        // (the metadata comes from the chunk list itself: waiting on the Q
+        // barrier for it could observe a phase two items ahead)
         const Tc2Item it = nxt;
         if (k + 1 < my_items) nxt = item_of(k + 1);
-        *item_slot(k) = it;
-#pragma unroll
-        for (int x = 0; x < 2 && ok; ++x) {
-          ok = mbar_wait(qfree(x), (k & 1) ^ 1, kWhereWaitQ, abort_flag);
+        const int nq = x == 0 ? it.nqa : it.nqb;
+        const int ntiles = x == 0 ? it.nkt_a : it.nkt;
+        const bool valid = i < nq && gi < it.rows;
+        const int lim = it.pos0 + x * qt + i + 1;  // keys visible to this row
+        float m = -INFINITY;                       // reference maximum (log2 units)
+        float l = 0.f;                             // sum of the rounded P
+        for (int t = 0; t < ntiles && ok; ++t) {
+          ok = __all_sync(0xffffffffu, mbar_wait(sfull(x), nx & 1, kWhereWaitMma, abort_flag));
           if (!ok) break;
-          mbar_arrive_expect_tx(qfull(x), static_cast<uint32_t>(L::kTileBytes));
-#pragma unroll
-          for (int h = 0; h < L::kHalves; ++h)
-            tma_load_3d(q_smem(x) + h * L::kHalfBytes, &tm_q, qfull(x), h * 64, it.head0,
-                        it.token0 + x * qt);
-        }
-        if (ok) q_last = k;
-      }
-      if (!ok && q_last >= 0) {
-        // a wait gave up: let the Q copies already issued land
-        volatile int own_flag = 0;
-        mbar_wait(qfull(0), q_last & 1, kWhereWaitQ, &own_flag);
-        mbar_wait(qfull(1), q_last & 1, kWhereWaitQ, &own_flag);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issue
-    // One thread.  Two cursors walk the CTA's (item, key tile) sequence, the S
-    // cursor one tile ahead of the P.V cursor.  Per step: P.V_A(cp), S_A(cs),
-    // P.V_B(cp), S_B(cs).  S_x(cs) overwrites the columns P.V_x(cp) reads P
-    // from; it is issued after that P.V, and the tensor core executes them in
-    // order.  (The other lanes go straight to the teardown barrier: this warp
-    // shares its SM sub-partition with two softmax warps, and every
-    // instruction it saves shortens the tensor core's idle gaps.)
-    if (lane == 0) {
-      struct Cursor {
-        int k, t, gt, nkt, nkt_a, kv_end_a, kv_end;
-      };
-      auto load_item = [&](Cursor& c, bool wait_q) -> bool {
-        if (c.k >= my_items) return true;
-        if (wait_q && !mbar_wait(qfull(0), c.k & 1, kWhereWaitQ, abort_flag)) return false;
-        const Tc2Item* it = item_slot(c.k);
-        c.nkt = it->nkt;
-        c.nkt_a = it->nkt_a;
-        c.kv_end_a = it->kv_end_a;
-        c.kv_end = it->kv_end;
-        return true;
-      };
-      auto advance = [&](Cursor& c) -> bool {  // true when it moved on to the next item
-        ++c.gt;
-        if (++c.t < c.nkt) return false;
-        c.t = 0;
-        ++c.k;
-        return true;
-      };
-      // S_x of the S cursor's tile (x = 0: tile A, 1: tile B)
-      auto issue_s = [&](const Cursor& c, int x) -> bool {
-        if (c.k >= my_items) return true;
-        if (x == 0 && c.t >= c.nkt_a) return true;  // no key of this tile is visible to A
-        const int ks = c.gt % KS;
-        if ((x == 0 || c.t >= c.nkt_a) &&
-            !mbar_wait(kfull(ks), (c.gt / KS) & 1, kWhereWaitFull, abort_flag))
-          return false;
-        if (x == 1 && c.t == 0 && !mbar_wait(qfull(1), c.k & 1, kWhereWaitQ, abort_flag))
-          return false;  // tile B's Q of this item
-        // (no tcgen05 fence here: the softmax threads' last reads of S_x were
-        // ordered before this thread's tcgen05 operations by the fence after
-        // its wait on their P, earlier in this thread's program order)
-        const uint64_t qd = smem_desc_sw128(q_smem(x), 16, 1024);
-        const uint64_t kd = smem_desc_sw128(k_smem(ks), 16, L::kGroupBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // descriptor start addresses advance in 16-byte units
-          const uint64_t qoff = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
-          const uint64_t koff = ((kk >> 2) * 1024 + (kk & 3) * 32) >> 4;
-          umma_ss(t_s(x), qd + qoff, kd + koff, kIdescS, kk > 0);
-        }
-        umma_commit(sfull(x));
-        if (c.t == (x == 0 ? c.nkt_a : c.nkt) - 1) umma_commit(qfree(x));
-        if (x == 1) umma_commit(kempty(ks));  // both tiles' S of this K tile issued
-        return true;
-      };
-      // P.V_x of the P.V cursor's tile
-      auto issue_pv = [&](const Cursor& c, int x, int nx) -> bool {
-        if (x == 0 && c.t >= c.nkt_a) return true;
-        const int vs = c.gt % VS;
-        if (!mbar_wait(pfull(x), nx & 1, kWhereWaitMma, abort_flag)) return false;
-        const bool first_use = x == 0 || c.t >= c.nkt_a;  // the first P.V on this V tile
-        if (first_use && !mbar_wait(vfull(vs), (c.gt / VS) & 1, kWhereWaitFull, abort_flag))
-          return false;
-        const int key0 = c.t * kTcKeys;
-        const int valid = min(kTcKeys, (x == 0 ? c.kv_end_a : c.kv_end) - key0);
-        const int steps = (valid + 15) >> 4;  // 16-key MMA steps holding visible keys
-        if (first_use && c.t == c.nkt - 1) {
-          // the item's last V tile: zero the rows of its last 16-key step past
-          // the item's last key (padding slots, or rows no box covered)
-          const int last = min(kTcKeys, c.kv_end - key0);
-          const int pad1 = min(kTcKeys, (last + 15) & ~15);
-          for (int row = last; row < pad1; ++row) {
-            uint8_t* dst = smem + L::kOffV + vs * L::kTileBytes + (row >> 3) * L::kGroupBytes +
-                           (row & 7) * 128;
-#pragma unroll
-            for (int h = 0; h < L::kHalves; ++h)
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(dst + h * 1024 + ch * 16) = make_uint4(0, 0, 0, 0);
+          tc_fence_after();
+          uint32_t ra[64], rb[64];
+          tmem_ld64_issue(t_s(x) + lane_base, ra);
+          tmem_ld64_issue(t_s(x) + lane_base + 64, rb);
+          tmem_ld_wait(ra);
+          reg_tie(rb);
+          float v[128];
+  #pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            v[j] = __uint_as_float(ra[j]);
+            v[64 + j] = __uint_as_float(rb[j]);
           }
-          fence_proxy_async_smem();
-        }
-        tc_fence_after();
-        const uint64_t vd = smem_desc_sw128(v_smem(vs), 1024, L::kGroupBytes);
-        const uint32_t acc0 = c.t > 0 ? 1u : 0u;  // the item's first tile starts O afresh
-        // unrolled: this thread shares its SM sub-partition with softmax warps,
-        // and a loop of a few instructions per MMA costs more than the MMA
-#pragma unroll
-        for (int kk = 0; kk < kTcKeys / 16; ++kk)
-          if (kk < steps)
-            umma_ts(t_o(x), t_s(x) + kk * 8, vd + ((kk * 2 * L::kGroupBytes) >> 4), kIdescPV,
-                    kk > 0 ? 1u : acc0);
-        umma_commit(pdone(x));
-        if (x == 1) umma_commit(vempty(vs));  // both tiles' P.V of this V tile issued
-        return true;
-      };
-      Cursor cs{0, 0, 0, 0, 0, 0, 0}, cp{0, 0, 0, 0, 0, 0, 0};
-      int na = 0, nb = 0;  // P.V issued so far for tile A and tile B
-      bool ok = my_items > 0 && load_item(cs, true);
-      if (ok) ok = issue_s(cs, 0) && issue_s(cs, 1);
-      if (ok && advance(cs)) ok = load_item(cs, true);
-      if (ok) ok = load_item(cp, false);  // the S cursor has waited for item 0's Q
-      while (ok && cp.k < my_items) {
-        const bool has_a = cp.t < cp.nkt_a;
-        ok = issue_pv(cp, 0, na) && issue_s(cs, 0) && issue_pv(cp, 1, nb) && issue_s(cs, 1);
-        na += has_a;
-        ++nb;
-        if (ok && advance(cs)) ok = load_item(cs, true);
-        if (ok && advance(cp)) ok = load_item(cp, false);  // the S cursor is past it already
-      }
-      // no MMA of this CTA may still run when TMEM is freed
-      umma_commit(drain);
-      volatile int own_flag = 0;
-      mbar_wait(drain, 0, kWhereWaitMma, &own_flag);
-    }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------- softmax warps
-    const int x = (warp - 4) >> 2;                        // 0: tile A, 1: tile B
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int r = (warp & 3) * 32 + lane;                 // tile row = TMEM lane
-    const int i = r / s.gs, gi = r % s.gs;
-    // Scores enter as x = s * |scale| after a sign flip of s for a negative
-    // scale, so that the row maximum is always a max.
-    const bool neg = scale_log2 < 0.f;
-    const float sc = fabsf(scale_log2);
-    int nx = 0;  // tiles of this query tile processed so far (P written)
-    bool ok = true;
-    Tc2Item nxt{};
-    if (my_items > 0) nxt = item_of(0);
-    for (int k = 0; k < my_items && ok; ++k) {
-      // (the metadata comes from the chunk list itself: waiting on the Q
-      // barrier for it could observe a phase two items ahead)
-      const Tc2Item it = nxt;
-      if (k + 1 < my_items) nxt = item_of(k + 1);
-      const int nq = x == 0 ? it.nqa : it.nqb;
-      const int ntiles = x == 0 ? it.nkt_a : it.nkt;
-      const bool valid = i < nq && gi < it.rows;
-      const int lim = it.pos0 + x * qt + i + 1;  // keys visible to this row
-      float m = -INFINITY;                       // reference maximum (log2 units)
-      float l = 0.f;                             // sum of the rounded P
-      for (int t = 0; t < ntiles && ok; ++t) {
-        ok = __all_sync(0xffffffffu, mbar_wait(sfull(x), nx & 1, kWhereWaitMma, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t ra[64], rb[64];
-        tmem_ld64_issue(t_s(x) + lane_base, ra);
-        tmem_ld64_issue(t_s(x) + lane_base + 64, rb);
-        tmem_ld_wait(ra);
-        reg_tie(rb);
-        float v[128];
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          v[j] = __uint_as_float(ra[j]);
-          v[64 + j] = __uint_as_float(rb[j]);
-        }
-        if (neg) {
-#pragma unroll
-          for (int j = 0; j < 128; ++j) v[j] = -v[j];
-        }
-        const int nvis = lim - t * kTcKeys;  // keys of this tile this row may see
-        if (nvis < kTcKeys) {
-#pragma unroll
-          for (int j = 0; j < 128; ++j) v[j] = j < nvis ? v[j] : -INFINITY;
-        }
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int j = 0; j < 128; j += 2) m4[(j >> 1) & 3] = fmax3(m4[(j >> 1) & 3], v[j], v[j + 1]);
-        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
-        // raise the reference maximum only when the row maximum has grown by
-        // more than 2^kTcRescale (always on the first visible keys)
-        const bool raise = mx > m + kTcRescale;
-        float alpha = 1.f;
-        if (raise) {
-          alpha = ex2_approx(m - mx);  // 0 when m = -inf
-          m = mx;
-        }
-        l *= alpha;
-        // P = 2^(v * sc - m), rounded to the input type, over the first 64
-        // columns of S (the scores are all in registers by now).  Half of the
-        // exponentials go to the special-function unit, half to the FMA pipe
-        // (exp2_poly2): at head_dim 128 a row's exponentials on the special-
-        // function unit alone take as long as the tensor core's QK^T and P.V
-        // for that row.  The row sum adds the weights before their rounding
-        // to the input type (the rounding is unbiased; its effect on the
-        // normalised output is of order 2^-9 / sqrt(keys)).
-        const float nm = m == -INFINITY ? 0.f : -m;
-        const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(nm, nm);
-        float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float2 a =
-                ffma2(make_float2(v[64 * hh + 2 * j], v[64 * hh + 2 * j + 1]), sc2, nm2);
-            float2 e = (kPolyExp && (j & 1)) ? exp2_poly2(a)
-                                             : make_float2(ex2_approx(a.x), ex2_approx(a.y));
-            if (nvis < kTcKeys) {  // masked keys: 0 (their -inf times a zero scale is NaN)
-              e.x = 64 * hh + 2 * j < nvis ? e.x : 0.f;
-              e.y = 64 * hh + 2 * j + 1 < nvis ? e.y : 0.f;
+          if (neg) {
+  #pragma unroll
+            for (int j = 0; j < 128; ++j) v[j] = -v[j];
+          }
+          const int nvis = lim - t * kTcKeys;  // keys of this tile this row may see
+          if (nvis < kTcKeys) {
+  #pragma unroll
+            for (int j = 0; j < 128; ++j) v[j] = j < nvis ? v[j] : -INFINITY;
+          }
+          // (eight independent chains: the maximum is on the critical path)
+          float m8[8];
+  #pragma unroll
+          for (int c = 0; c < 8; ++c) m8[c] = fmaxf(v[2 * c], v[2 * c + 1]);
+  #pragma unroll
+          for (int j = 16; j < 128; j += 2) m8[(j >> 1) & 7] = fmax3(m8[(j >> 1) & 7], v[j], v[j + 1]);
+          const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                                 fmaxf(m8[6], m8[7])) * sc;
+          // raise the reference maximum only when the row maximum has grown by
+          // more than 2^kTcRescale (always on the first visible keys)
+          const bool raise = mx > m + kTcRescale;
+          float alpha = 1.f;
+          if (raise) {
+            alpha = ex2_approx(m - mx);  // 0 when m = -inf
+            m = mx;
+          }
+          l *= alpha;
+          // P = 2^(v * sc - m), rounded to the input type, over the first 64
+          // columns of S (the scores are all in registers by now).  The
+          // exponentials run on the special-function unit, except kPolyPairs of
+          // every 8 pairs, which take exp2_poly2 on the FMA pipe.  The row sum
+          // adds the weights before their rounding to the input type (the
+          // rounding is unbiased; its effect on the normalised output is of
+          // order 2^-9 / sqrt(keys)).
+          const float nm = m == -INFINITY ? 0.f : -m;
+          const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(nm, nm);
+          float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+  #pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t pk[32];
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float2 a =
+                  ffma2(make_float2(v[64 * hh + 2 * j], v[64 * hh + 2 * j + 1]), sc2, nm2);
+              float2 e = (j & 7) < kPolyPairs ? exp2_poly2(a)
+                                              : make_float2(ex2_approx(a.x), ex2_approx(a.y));
+              pk[j] = pack2<T>(e.x, e.y);
+              ps[j & 3] = fadd2(ps[j & 3], e);
             }
-            pk[j] = pack2<T>(e.x, e.y);
-            ps[j & 1] = fadd2(ps[j & 1], e);
+            tmem_st32(t_s(x) + lane_base + hh * 32, pk);
           }
-          tmem_st32(t_s(x) + lane_base + hh * 32, pk);
-        }
-        if (t > 0 && __any_sync(0xffffffffu, raise)) {
-          // O holds P.V of tiles 0 .. t-1: once the last of them is done,
-          // bring the row to the new reference point (before P.V of tile t,
-          // which waits for this thread's arrival below)
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(pdone(x), (nx - 1) & 1, kWhereWaitMma, abort_flag));
-          if (!ok) break;
-          tc_fence_after();
-          uint32_t ro[64];
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 64) {
-            tmem_ld64_issue(t_o(x) + lane_base + c0, ro);
-            tmem_ld_wait(ro);
-#pragma unroll
-            for (int j = 0; j < 64; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
-            tmem_st64(t_o(x) + lane_base + c0, ro);
+          if (t > 0 && __any_sync(0xffffffffu, raise)) {
+            // O holds P.V of tiles 0 .. t-1: once the last of them is done,
+            // bring the row to the new reference point (before P.V of tile t,
+            // which waits for this thread's arrival below)
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(pdone(x), (nx - 1) & 1, kWhereWaitMma, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t ro[64];
+  #pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 64) {
+              tmem_ld64_issue(t_o(x) + lane_base + c0, ro);
+              tmem_ld_wait(ro);
+  #pragma unroll
+              for (int j = 0; j < 64; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
+              tmem_st64(t_o(x) + lane_base + c0, ro);
+            }
           }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(pfull(x));
+          l += ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) + ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
+          ++nx;
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(pfull(x));
-        l += (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y);
-        ++nx;
-      }
-      if (ok && ntiles > 0) {
-        // the item's last P.V of this tile done: O is final
-        ok = __all_sync(0xffffffffu, mbar_wait(pdone(x), (nx - 1) & 1, kWhereWaitMma,
-                                               abort_flag));
-        if (ok) {
-          tc_fence_after();
-          const float inv = l > 0.f ? 1.f / l : 0.f;
-          uint32_t ro[64];
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 64) {
-            tmem_ld64_issue(t_o(x) + lane_base + c0, ro);
-            tmem_ld_wait(ro);
-            if (valid) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                float a[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(ro[q * 8 + e]);
-                store_row8<T, D>(s, out, it.token0 + x * qt + i, it.head0 + gi, c0 / 8 + q, a,
-                                 inv);
+        if (ok && ntiles > 0) {
+          // the item's last P.V of this tile done: O is final
+          ok = __all_sync(0xffffffffu, mbar_wait(pdone(x), (nx - 1) & 1, kWhereWaitMma,
+                                                 abort_flag));
+          if (ok) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            uint32_t ro[64];
+  #pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 64) {
+              tmem_ld64_issue(t_o(x) + lane_base + c0, ro);
+              tmem_ld_wait(ro);
+              if (valid) {
+  #pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  float a[8];
+  #pragma unroll
+                  for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(ro[q * 8 + e]);
+                  store_row8<T, D>(s, out, it.token0 + x * qt + i, it.head0 + gi, c0 / 8 + q, a,
+                                   inv);
+                }
               }
             }
+            // the next item's first P.V overwrites O: the reads above complete
+            // before this thread's next arrival on pfull
+            tc_fence_before();
           }
-          // the next item's first P.V overwrites O: the reads above complete
-          // before this thread's next arrival on pfull
-          tc_fence_before();
         }
       }
     }

@@ -77,14 +77,17 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
 
 // D[tmem] (+)= A[tmem] * B[smem]: A (M x K, K-major) is read from tensor
 // memory, row i in lane i, two 16-bit elements per 32-bit column (the lower K
-// index in the low half).
+// index in the low half).  Issued only when `issue` is nonzero: a predicated
+// instruction, not a branch (a branch around each MMA roughly doubles the
+// issue time of a group of them).
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
+                                        uint32_t idesc, uint32_t accumulate, uint32_t issue = 1) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(issue)
       : "memory");
 }
 
@@ -285,27 +288,28 @@ constexpr float kExp2C1 = 0.6932609677314758f;
 constexpr float kExp2C2 = 0.2426111251115799f;
 constexpr float kExp2C3 = 0.0551716685295105f;
 
-// 2^x for two values on the FMA and integer pipes, leaving the special-
-// function unit to the other half of a row's exponentials.  Range reduction
-// in the manner of Cody and Waite: x = j + f with j the nearest integer
-// (adding 1.5 * 2^23 leaves round(x) in the low mantissa bits), f in
-// [-1/2, 1/2]; 2^f from the cubic above; 2^j added to the exponent field.
-// x is clamped below at -126 (the result is then a weight of order 2^-126,
-// not 0; callers zero masked entries themselves).  Valid for x < 127.
+// 2^x for two values on the FMA pipe, leaving the special-function unit to
+// the other exponentials of a row.  Range reduction in the manner of Cody and
+// Waite: x = j + f with j the nearest integer (adding 1.5 * 2^23 leaves
+// round(x) in the low mantissa bits of t), f in [-1/2, 1/2]; 2^f from the
+// cubic above; 2^j added to the exponent field as t's bits times 2^23 (the
+// bits of 1.5 * 2^23 vanish in that product modulo 2^32).  x is clamped below
+// at -125, where 2^f's exponent field (126 or 127) plus j stays positive: the
+// result is then a weight of order 2^-125, not 0 (callers zero masked
+// entries themselves).  Valid for x < 127.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
   const float2 shift = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
   const float2 t = fadd2(x, shift);
-  const float2 j = fsub2(t, shift);
-  const float2 f = fsub2(x, j);
+  const float2 f = fsub2(x, fsub2(t, shift));
   float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
   p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
   p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
-  const unsigned jx = static_cast<unsigned>(__float_as_int(t.x) - 0x4B400000);
-  const unsigned jy = static_cast<unsigned>(__float_as_int(t.y) - 0x4B400000);
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (jx << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (jy << 23)));
+  uint32_t rx, ry;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(p.x)));
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(p.y)));
+  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 // max(a, b, c) in one instruction.
