@@ -316,17 +316,26 @@ __global__ void __launch_bounds__(384, 1)
           const Tc2Item it = nxt;
           if (k + 1 < my_items) nxt = item_of(k + 1);
           *item_slot(k) = it;
-  #pragma unroll
+#pragma unroll
           for (int x = 0; x < 2 && ok; ++x) {
             ok = mbar_wait(qfree(x), (k & 1) ^ 1, kWhereWaitQ, abort_flag);
             if (!ok) break;
             mbar_arrive_expect_tx(qfull(x), static_cast<uint32_t>(L::kTileBytes));
-  #pragma unroll
+#pragma unroll
             for (int h = 0; h < L::kHalves; ++h)
               tma_load_3d(q_smem(x) + h * L::kHalfBytes, &tm_q, qfull(x), h * 64, it.head0,
                           it.token0 + x * qt);
           }
           if (ok) q_last = k;
+          // the next item's Q tiles into L2 now, so that their loads, which
+          // wait for this item's last S, take an L2 hit
+          if (ok && k + 1 < my_items) {
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+              for (int h = 0; h < L::kHalves; ++h)
+                tma_prefetch_3d(&tm_q, h * 64, nxt.head0, nxt.token0 + x * qt);
+          }
         }
         if (!ok && q_last >= 0) {
           // a wait gave up: let the Q copies already issued land
@@ -383,7 +392,7 @@ __global__ void __launch_bounds__(384, 1)
           // its wait on their P, earlier in this thread's program order)
           const uint64_t qd = smem_desc_sw128(q_smem(x), 16, 1024);
           const uint64_t kd = smem_desc_sw128(k_smem(c.ks), 16, L::kGroupBytes);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             // descriptor start addresses advance in 16-byte units
             const uint64_t qoff = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
@@ -396,13 +405,14 @@ __global__ void __launch_bounds__(384, 1)
         };
         // P.V_x of the P.V cursor's tile, once P_x is written (its V tile waited for)
         auto issue_pv = [&](const Cursor& c, int x, int nx) -> bool {
-          if (!mbar_wait(pfull(x), nx & 1, kWhereWaitMma, abort_flag)) return false;
-          tc_fence_after();
+          // operands first: only the MMAs themselves wait for P
           const int valid = min(kTcKeys, (x == 0 ? c.kv_end_a : c.kv_end) - c.t * kTcKeys);
           const int steps = (valid + 15) >> 4;  // 16-key MMA steps holding visible keys
           const uint64_t vd = smem_desc_sw128(v_smem(c.vs), 1024, L::kGroupBytes);
           const uint32_t acc0 = c.t > 0 ? 1u : 0u;  // the item's first tile starts O afresh
-  #pragma unroll
+          if (!mbar_wait(pfull(x), nx & 1, kWhereWaitMma, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
           for (int kk = 0; kk < kTcKeys / 16; ++kk)
             umma_ts(t_o(x), t_s(x) + kk * 8, vd + ((kk * 2 * L::kGroupBytes) >> 4), kIdescPV,
                     kk > 0 ? 1u : acc0, kk < steps);
@@ -422,9 +432,9 @@ __global__ void __launch_bounds__(384, 1)
             for (int row = last; row < pad1; ++row) {
               uint8_t* dst = smem + L::kOffV + c.vs * L::kTileBytes + (row >> 3) * L::kGroupBytes +
                              (row & 7) * 128;
-  #pragma unroll
+#pragma unroll
               for (int h = 0; h < L::kHalves; ++h)
-  #pragma unroll
+#pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
                   *reinterpret_cast<uint4*>(dst + h * 1024 + ch * 16) = make_uint4(0, 0, 0, 0);
             }
@@ -485,6 +495,7 @@ __global__ void __launch_bounds__(384, 1)
       // 2^-100 so that -inf * scale stays -inf (every visible x is then 0 to
       // within fp32, as with the zero scale).
       const bool neg = scale_log2 < 0.f;
+      const bool out32 = (reinterpret_cast<uintptr_t>(out) & 31) == 0;
       const float sc = fmaxf(fabsf(scale_log2), 7.8886091e-31f);
       int nx = 0;  // tiles of this query tile processed so far (P written)
       bool ok = true;
@@ -511,25 +522,25 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld_wait(ra);
           reg_tie(rb);
           float v[128];
-  #pragma unroll
+#pragma unroll
           for (int j = 0; j < 64; ++j) {
             v[j] = __uint_as_float(ra[j]);
             v[64 + j] = __uint_as_float(rb[j]);
           }
           if (neg) {
-  #pragma unroll
+#pragma unroll
             for (int j = 0; j < 128; ++j) v[j] = -v[j];
           }
           const int nvis = lim - t * kTcKeys;  // keys of this tile this row may see
           if (nvis < kTcKeys) {
-  #pragma unroll
+#pragma unroll
             for (int j = 0; j < 128; ++j) v[j] = j < nvis ? v[j] : -INFINITY;
           }
           // (eight independent chains: the maximum is on the critical path)
           float m8[8];
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < 8; ++c) m8[c] = fmaxf(v[2 * c], v[2 * c + 1]);
-  #pragma unroll
+#pragma unroll
           for (int j = 16; j < 128; j += 2) m8[(j >> 1) & 7] = fmax3(m8[(j >> 1) & 7], v[j], v[j + 1]);
           const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
                                  fmaxf(m8[6], m8[7])) * sc;
@@ -553,10 +564,10 @@ __global__ void __launch_bounds__(384, 1)
           const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(nm, nm);
           float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
-  #pragma unroll
+#pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t pk[32];
-  #pragma unroll
+#pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float2 a =
                   ffma2(make_float2(v[64 * hh + 2 * j], v[64 * hh + 2 * j + 1]), sc2, nm2);
@@ -576,11 +587,11 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) break;
             tc_fence_after();
             uint32_t ro[64];
-  #pragma unroll
+#pragma unroll
             for (int c0 = 0; c0 < D; c0 += 64) {
               tmem_ld64_issue(t_o(x) + lane_base + c0, ro);
               tmem_ld_wait(ro);
-  #pragma unroll
+#pragma unroll
               for (int j = 0; j < 64; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
               tmem_st64(t_o(x) + lane_base + c0, ro);
             }
@@ -599,19 +610,36 @@ __global__ void __launch_bounds__(384, 1)
           if (ok) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
+            T* orow = out + (static_cast<size_t>(it.token0 + x * qt + i) * s.num_q_heads +
+                             it.head0 + gi) * D;
             uint32_t ro[64];
-  #pragma unroll
+#pragma unroll
             for (int c0 = 0; c0 < D; c0 += 64) {
               tmem_ld64_issue(t_o(x) + lane_base + c0, ro);
               tmem_ld_wait(ro);
               if (valid) {
-  #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  float a[8];
-  #pragma unroll
-                  for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(ro[q * 8 + e]);
-                  store_row8<T, D>(s, out, it.token0 + x * qt + i, it.head0 + gi, c0 / 8 + q, a,
-                                   inv);
+                // each lane writes its own row: whole 32-byte sectors where the
+                // output is 32-byte aligned (rows are 128 or 256 bytes)
+                if (out32) {
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                      w[e] = pack2<T>(__uint_as_float(ro[q * 16 + 2 * e]) * inv,
+                                      __uint_as_float(ro[q * 16 + 2 * e + 1]) * inv);
+                    st_global_v8(orow + c0 + q * 16, w);
+                  }
+                } else {
+#pragma unroll
+                  for (int q = 0; q < 8; ++q) {
+                    uint4 w;
+                    w.x = pack2<T>(__uint_as_float(ro[q * 8]) * inv, __uint_as_float(ro[q * 8 + 1]) * inv);
+                    w.y = pack2<T>(__uint_as_float(ro[q * 8 + 2]) * inv, __uint_as_float(ro[q * 8 + 3]) * inv);
+                    w.z = pack2<T>(__uint_as_float(ro[q * 8 + 4]) * inv, __uint_as_float(ro[q * 8 + 5]) * inv);
+                    w.w = pack2<T>(__uint_as_float(ro[q * 8 + 6]) * inv, __uint_as_float(ro[q * 8 + 7]) * inv);
+                    *reinterpret_cast<uint4*>(orow + c0 + q * 8) = w;
+                  }
                 }
               }
             }
