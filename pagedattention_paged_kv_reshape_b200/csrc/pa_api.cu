@@ -346,13 +346,18 @@ pa_status launch_simt(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   return PA_OK;
 }
 
-template <typename T, int D, bool KV8>
+template <typename T, int D, bool KV8, bool NARROW = false>
 pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
+  // tiles of at most 8 rows on an FP8 cache at head_dim 128: the transposed
+  // P.V form of the kernel
+  if constexpr (KV8 && D == 128 && !NARROW) {
+    if (p.s.gs * p.s.qpt <= 8) return launch_mma<T, D, KV8, true>(a, p, w);
+  }
   // FP8 stages are half as large: at head_dim 128 twice as many keep the same
   // bytes in flight; at 64 the per-warp f16 staging tiles take that room
   constexpr int kS = KV8 && D == 128 ? 2 * kStages : kStages;
   using L = pa::MmaLayout<D, kNcw, kS, KV8>;
-  auto kern = pa::attn_mma_kernel<T, D, kNcw, kS, KV8>;
+  auto kern = pa::attn_mma_kernel<T, D, kNcw, kS, KV8, NARROW>;
   int occ = 0;
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "mma kernel set-up");

@@ -32,6 +32,7 @@
 namespace pa {
 
 constexpr int kMetaSlots = 4;
+constexpr float kLazyRaise = 8.f;  // see the online softmax of attn_mma_kernel (log2 units)
 
 // One scheduler-ring slot: a decoded unit and, for each 16-key tile of its
 // partition, the cache row of the tile's first key (y0) and, with 8-token
@@ -168,7 +169,7 @@ __device__ __forceinline__ void convert_fp8_tile(uint32_t src, uint32_t dst, int
   }
 }
 
-template <typename T, int D, int NCW, int STAGES, bool KV8 = false>
+template <typename T, int D, int NCW, int STAGES, bool KV8 = false, bool NARROW = false>
 __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
@@ -189,8 +190,17 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
   // reads the 16 bytes of dims 16g .. 16g+15 of each of its four keys.  The
   // epilogue writes every accumulator to its own head dim.
   constexpr bool fp8_direct = KV8 && !L::kStaging;
+  // NARROW (FP8 direct, tiles of at most 8 rows: decode with a group of up to
+  // 8 heads): P.V is taken transposed, O^T = V^T P^T, as D/16 m16n8k16 MMAs
+  // whose 8 columns are the tile's rows -- half the MMAs and half the
+  // accumulators of the 16-row form, whose rows 8-15 would be padding.  P^T
+  // is the B operand straight from the QK^T accumulators of rows 0-7.  Row i
+  // of m-tile mt is head dim 16 (i % 8) + 2 mt + i / 8, so that lane group g
+  // again reads the 16 bytes of dims 16g .. 16g+15 of its four keys.
+  static_assert(!NARROW || fp8_direct, "the transposed P.V is built on the FP8 direct operands");
   constexpr int KSTEPS = D / 16;  // k-steps of QK^T, also n-tile pairs of PV
   constexpr int NT = D / 8;       // PV n-tiles of 8 dims
+  constexpr int NO = NARROW ? D / 16 : NT;  // accumulator tiles of O (or of O^T)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -444,14 +454,18 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
           qa[kk][e] = pack2<__half>(f.x, f.y);
         }
     }
+    if constexpr (NARROW) {  // rows 8-15 are padding: a zero operand, no registers
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) qa[kk][1] = qa[kk][3] = 0u;
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(qempty_bar(qs));
     ++k;
 
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float o[NT][4];
+    float o[NO][4];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    for (int t = 0; t < NO; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
     // FP8: the K scale of this KV head folds into the softmax scale
     const float sl = KV8 ? scale_log2 * __ldg(k_scale + u.kvh) : scale_log2;
     const int lim0 = u.lim0 + r0 / s.gs;
@@ -490,24 +504,28 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       const int blk_start = u.kv_begin + j * kBlock;
 
       // ---- S = Q K^T over this block's 16 tokens
-      float sacc[2][4];
+      // (two partial sums per n-tile, over even and odd k-steps: four
+      // independent MMA chains instead of two halve the latency of this phase)
+      float sacc[2][4], sodd[2][4];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) sacc[t][0] = sacc[t][1] = sacc[t][2] = sacc[t][3] = 0.f;
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[t][e] = sodd[t][e] = 0.f;
       if constexpr (fp8_direct) {
         const int g = lane >> 2, q4 = lane & 3;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        for (int G = 0; G < D / 64; ++G) {
+          uint32_t w[2][4];  // keys g and 8+g, dims 64G + 16 q4 .. +15
 #pragma unroll
-          for (int G = 0; G < D / 64; ++G) {
-            uint32_t w[4];  // key nt*8+g, dims 64G + 16 q4 .. +15
-            lds128(kb + swz(nt * 8 + g, 4 * G + q4), w);
+          for (int nt = 0; nt < 2; ++nt) lds128(kb + swz(nt * 8 + g, 4 * G + q4), w[nt]);
 #pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4) {
+          for (int s4 = 0; s4 < 4; ++s4)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
               uint32_t b0, b1;
-              fp8x4_to_f16x2x2(w[s4], b0, b1);
-              mma_16816<MT>(sacc[nt], qa[4 * G + s4], b0, b1);
+              fp8x4_to_f16x2x2(w[nt][s4], b0, b1);
+              mma_16816<MT>((s4 & 1) ? sodd[nt] : sacc[nt], qa[4 * G + s4], b0, b1);
             }
-          }
         }
       } else {
         const int mi = lane >> 3;
@@ -517,10 +535,14 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
           uint32_t b0, b1, b2, b3;
           const int ch = (kk & 3) * 2 + (mi & 1);
           ldsm_x4(kb + kv_off(tk, kk >> 2, ch, L::kGroupBytes), b0, b1, b2, b3);
-          mma_16816<MT>(sacc[0], qa[kk], b0, b1);
-          mma_16816<MT>(sacc[1], qa[kk], b2, b3);
+          mma_16816<MT>((kk & 1) ? sodd[0] : sacc[0], qa[kk], b0, b1);
+          mma_16816<MT>((kk & 1) ? sodd[1] : sacc[1], qa[kk], b2, b3);
         }
       }
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[t][e] += sodd[t][e];
       float x[2][4];
 #pragma unroll
       for (int t = 0; t < 2; ++t)
@@ -535,36 +557,65 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
             if (key >= (e < 2 ? lim0 : lim1)) x[t][e] = -INFINITY;
           }
       }
-      // ---- online softmax (rows r0 and r1 of this thread)
-      float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-      float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-      const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float a0 = exp2f(m0 - mu0), a1 = exp2f(m1 - mu1);
+      // ---- online softmax (rows r0 and r1 of this thread), against a
+      // reference maximum per row that is raised only when a score of the row
+      // passes it by more than 2^8 (so P <= 256, exact enough in the 16-bit
+      // operand type); until then no shuffle, no rescale.  (In NARROW rows
+      // 8-15 are padding and take no part.)
+      const float lx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+      const float lx1 =
+          NARROW ? -INFINITY : fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+      if (__any_sync(0xffffffffu, lx0 > m0 + kLazyRaise || lx1 > m1 + kLazyRaise)) {
+        float mx0 = lx0, mx1 = lx1;
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        // factor from the old reference to the new: 1 for rows that keep it,
+        // 0 for rows that had none (m = -inf)
+        const float a0 = ex2_approx(m0 - (mn0 == -INFINITY ? 0.f : mn0));
+        const float a1 = ex2_approx(m1 - (mn1 == -INFINITY ? 0.f : mn1));
+        l0 *= a0;
+        l1 *= a1;
+        if constexpr (NARROW) {  // this lane's O^T columns are rows 2 quad, 2 quad + 1
+          const float c0 = __shfl_sync(0xffffffffu, a0, (2 * quad) << 2);
+          const float c1 = __shfl_sync(0xffffffffu, a0, (2 * quad + 1) << 2);
+#pragma unroll
+          for (int t = 0; t < NO; ++t) {
+            o[t][0] *= c0;
+            o[t][1] *= c1;
+            o[t][2] *= c0;
+            o[t][3] *= c1;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            o[t][0] *= a0;
+            o[t][1] *= a0;
+            o[t][2] *= a1;
+            o[t][3] *= a1;
+          }
+        }
+        m0 = mn0;
+        m1 = mn1;
+      }
+      const float mu0 = m0 == -INFINITY ? 0.f : m0;
+      const float mu1 = m1 == -INFINITY ? 0.f : m1;
       uint32_t pa[4];
-      pa[0] = pack2<MT>(exp2f(x[0][0] - mu0), exp2f(x[0][1] - mu0));
-      pa[1] = pack2<MT>(exp2f(x[0][2] - mu1), exp2f(x[0][3] - mu1));
-      pa[2] = pack2<MT>(exp2f(x[1][0] - mu0), exp2f(x[1][1] - mu0));
-      pa[3] = pack2<MT>(exp2f(x[1][2] - mu1), exp2f(x[1][3] - mu1));
+      pa[0] = pack2<MT>(ex2_approx(x[0][0] - mu0), ex2_approx(x[0][1] - mu0));
+      pa[2] = pack2<MT>(ex2_approx(x[1][0] - mu0), ex2_approx(x[1][1] - mu0));
+      if constexpr (NARROW) {  // rows 8-15 are padding
+        pa[1] = pa[3] = 0u;
+      } else {
+        pa[1] = pack2<MT>(ex2_approx(x[0][2] - mu1), ex2_approx(x[0][3] - mu1));
+        pa[3] = pack2<MT>(ex2_approx(x[1][2] - mu1), ex2_approx(x[1][3] - mu1));
+      }
       // the normaliser sums the same rounded weights the P.V product uses
       const float2 p00 = unpack2<MT>(pa[0]), p01 = unpack2<MT>(pa[1]);
       const float2 p10 = unpack2<MT>(pa[2]), p11 = unpack2<MT>(pa[3]);
-      l0 = l0 * a0 + ((p00.x + p00.y) + (p10.x + p10.y));
-      l1 = l1 * a1 + ((p01.x + p01.y) + (p11.x + p11.y));
-      m0 = mn0;
-      m1 = mn1;
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        o[t][0] *= a0;
-        o[t][1] *= a0;
-        o[t][2] *= a1;
-        o[t][3] *= a1;
-      }
+      l0 += (p00.x + p00.y) + (p10.x + p10.y);
+      l1 += (p01.x + p01.y) + (p11.x + p11.y);
       // ---- O += P V ; V rows at or past the unit's last visible key are
       // zeroed (padding may hold anything, and 0 * NaN is NaN)
       uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
@@ -573,7 +624,30 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
         vm0 = (t0 < nv ? 0x0000ffffu : 0u) | (t0 + 1 < nv ? 0xffff0000u : 0u);
         vm1 = (t0 + 8 < nv ? 0x0000ffffu : 0u) | (t0 + 9 < nv ? 0xffff0000u : 0u);
       }
-      if constexpr (fp8_direct) {  // V from the bytes loaded above
+      if constexpr (NARROW) {  // O^T += V^T P^T, V^T from the bytes loaded above
+        auto pvn = [&](bool masked) {
+#pragma unroll
+          for (int mt = 0; mt < NO; ++mt) {
+            // bytes 2(mt%2), +1 of word mt/2: dims 16g + 2mt (rows g) and
+            // 16g + 2mt + 1 (rows g + 8) of keys 2q4, 2q4+1 and 2q4+8, 2q4+9
+            const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+            uint32_t av[4];
+            fp8x4_to_f16x2x2(prmt(va[mt >> 1], vb1[mt >> 1], sel), av[0], av[1]);
+            fp8x4_to_f16x2x2(prmt(vc[mt >> 1], vd[mt >> 1], sel), av[2], av[3]);
+            if (masked) {
+              av[0] &= vm0;
+              av[1] &= vm0;
+              av[2] &= vm1;
+              av[3] &= vm1;
+            }
+            mma_16816<MT>(o[mt], av, pa[0], pa[2]);
+          }
+        };
+        if (blk_start + kBlock > u.kv_end)  // padding rows: only the last tile has them
+          pvn(true);
+        else
+          pvn(false);
+      } else if constexpr (fp8_direct) {  // V from the bytes loaded above
         auto pv8 = [&](bool masked) {
 #pragma unroll
           for (int jw = 0; jw < 4; ++jw) {
@@ -631,7 +705,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
     if constexpr (KV8) {  // the V scale of this KV head
       const float vsc = __ldg(v_scale + u.kvh);
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
+      for (int t = 0; t < NO; ++t)
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[t][e] *= vsc;
     }
@@ -646,7 +720,17 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       cm[warp * kRows + r1] = m1;
       cl[warp * kRows + r1] = l1;
     }
-    if constexpr (fp8_direct) {
+    if constexpr (NARROW) {
+      // m-tile mt holds dims 16g + 2mt (c0, c1) and 16g + 2mt + 1 (c2, c3) of
+      // rows 2 quad (c0, c2) and 2 quad + 1 (c1, c3)
+#pragma unroll
+      for (int rs = 0; rs < 2; ++rs)
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          *reinterpret_cast<float4*>(&co[warp][2 * quad + rs][16 * r0 + 4 * c4]) =
+              make_float4(o[2 * c4][rs], o[2 * c4][2 + rs], o[2 * c4 + 1][rs],
+                          o[2 * c4 + 1][2 + rs]);
+    } else if constexpr (fp8_direct) {
       // n-tile t, columns 2q, 2q+1 hold head dims 32q + t and 32q + 16 + t: this
       // lane has dims 32q .. 32q+31 of rows r0 and r1, stored as eight float4
       // chunks per row in the swizzled layout (conflict-free; plain offsets put
@@ -670,7 +754,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       }
     }
     if (!consumers_sync()) return;
-    epilogue<T, D, NCW, fp8_direct>(s, u, cm, cl, co, out, w, tid, NCW * 32);
+    epilogue<T, D, NCW, fp8_direct && !NARROW>(s, u, cm, cl, co, out, w, tid, NCW * 32);
     if (!consumers_sync()) return;
   }
 }
