@@ -43,7 +43,8 @@ sys.path.insert(0, ROOT)
 METRIC = ("paged-attn decode KV-read GB/s (% of B200 HBM peak); decode tokens/s per config")
 HEADLINE = "mixed_2048"
 PER_CONFIG = ("mha_bs64", "gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512",
-              "gqa_bs256_b8", "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256")
+              "gqa_bs256_b8", "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256",
+              "prefill_16x512_d256")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 

@@ -333,6 +333,10 @@ CONFIGS = {
                            head_dim=128, dtype="bf16", pool_factor=1.0, kind="varlen",
                            about="16 causal prefill chunks of 512 tokens on 1536 cached tokens, "
                                  "32/8 heads, head_dim 128, bf16 (tensor-core chunk kernel)"),
+    "prefill_16x512_d256": dict(requests=prefill_requests, num_q_heads=16, num_kv_heads=4,
+                                head_dim=256, dtype="bf16", pool_factor=1.0, kind="varlen",
+                                about="prefill_16x512's chunks with head_dim 256, 16/4 heads "
+                                      "(the same KV bytes per token and FLOPs per query token)"),
 }
 
 

@@ -29,7 +29,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 FULL_SIZE = ["mha_bs64", "gqa_bs256", "long_32k", "mixed_2048", "prefill_16x512",
-             "gqa_bs256_b8", "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256"]
+             "gqa_bs256_b8", "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256",
+             "prefill_16x512_d256"]
 
 
 def check_cache_write(b, kc, vc):

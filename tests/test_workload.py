@@ -88,6 +88,12 @@ def test_prefill_and_variants():
     base = [x.seq_len for x in reqs("gqa_bs256")]
     for name in ("gqa_bs256_b8", "gqa_bs256_b32", "gqa_bs256_fp8", "gqa_bs256_d256"):
         assert [x.seq_len for x in reqs(name)] == base
+    # prefill at head_dim 256: prefill_16x512's rows, the same KV bytes per token
+    p = W.CONFIGS["prefill_16x512_d256"]
+    q = W.CONFIGS["prefill_16x512"]
+    assert p["head_dim"] == 256 and p["kind"] == "varlen"
+    assert p["num_kv_heads"] * p["head_dim"] == q["num_kv_heads"] * q["head_dim"]
+    assert [(x.seq_len, x.q_len) for x in reqs("prefill_16x512_d256")] == [(2048, 512)] * 16
 
 
 @pytest.mark.parametrize("name", ["mha_bs64", "gqa_bs256", "mixed_2048"])
