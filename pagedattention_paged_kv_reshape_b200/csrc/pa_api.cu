@@ -16,6 +16,7 @@
 #include "pa_attn_mma.cuh"
 #include "pa_attn_simt.cuh"
 #include "pa_blocks.cuh"
+#include "pa_chunk_tc1.cuh"
 #include "pa_chunk_tc2.cuh"
 #include "pa_reduce.cuh"
 
@@ -383,10 +384,12 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   return PA_OK;
 }
 
+// The tcgen05 chunk kernel: two query tiles per item up to head_dim 128,
+// one per item (64-key tiles) at 256.
 template <typename T, int D>
 pa_status launch_chunk(const AttnArgs& a, const Plan& p, const pa::Work& w) {
-  using L = pa::Tc2Layout<D>;
-  auto kern = pa::chunk_tc2_kernel<T, D>;
+  using L = typename std::conditional<D == 256, pa::Tc1Layout<256>, pa::Tc2Layout<D>>::type;
+  auto kern = D == 256 ? pa::chunk_tc1_kernel<T, 256> : pa::chunk_tc2_kernel<T, D == 256 ? 128 : D>;
   int occ = 0;
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "chunk kernel set-up");
@@ -446,7 +449,9 @@ pa_status run_typed(const AttnArgs& a, const Plan& p, bool use_mma) {
   if (st != PA_OK) return st;
   if constexpr (sizeof(T) == 2) {
     if (p.s.chunk_qt > 0) {
-      st = a.head_dim == 128 ? launch_chunk<T, 128>(a, p, w) : launch_chunk<T, 64>(a, p, w);
+      st = a.head_dim == 128   ? launch_chunk<T, 128>(a, p, w)
+           : a.head_dim == 256 ? launch_chunk<T, 256>(a, p, w)
+                               : launch_chunk<T, 64>(a, p, w);
       if (st != PA_OK) return st;
     }
   }
@@ -515,13 +520,14 @@ pa_status run_attention(const AttnArgs& a, bool varlen) {
   const bool use_mma = sixteen && path != PA_PATH_SIMT;
   // Prefill-chunk rows (q_len >= one 128-row tile) go to the tcgen05 kernel
   // unless a family without it was forced.
-  p.s.chunk_qt = (use_mma && !a.kv8() && a.head_dim != 256 && path != PA_PATH_MMA &&
+  p.s.chunk_qt = (use_mma && !a.kv8() && path != PA_PATH_MMA &&
                   p.chunk_qt > 0 &&
                   a.max_query_len >= p.chunk_qt)
                      ? p.chunk_qt
                      : 0;
   p.s.chunk_cap = static_cast<int>(p.chunk_cap);
-  p.s.chunk_span = 2 * p.s.chunk_qt;  // a chunk item holds two query tiles
+  // a chunk item holds two query tiles (one at head_dim 256)
+  p.s.chunk_span = a.head_dim == 256 ? p.s.chunk_qt : 2 * p.s.chunk_qt;
   switch (a.dtype) {
     case PA_BF16: return run_typed<__nv_bfloat16>(a, p, use_mma);
     case PA_F16: return run_typed<__half>(a, p, use_mma);

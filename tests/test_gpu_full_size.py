@@ -76,7 +76,8 @@ def test_full_size_every_row_matches_oracle(name):
 
 
 @pytest.mark.parametrize("name,repeats", [("gqa_bs256", 200), ("gqa_bs256_fp8", 200),
-                                          ("mixed_2048", 40), ("prefill_16x512", 100)])
+                                          ("mixed_2048", 40), ("prefill_16x512", 100),
+                                          ("prefill_16x512_d256", 40)])
 def test_repeated_full_size_calls_are_bitwise_identical(name, repeats):
     """The same call repeated back to back on one stream and one workspace
     (each call's kernels overlap the previous call's tail through

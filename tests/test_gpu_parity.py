@@ -173,8 +173,9 @@ def test_varlen_matches_oracle(case, path):
     assert_close(out, ref, dtype, f"varlen case {case} ({path})")
 
 
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("scale", [1.0, -0.3, 0.0])
-def test_varlen_other_scales(scale):
+def test_varlen_other_scales(scale, d):
     """Scales other than 1/sqrt(head_dim).  With 1.0 the scores of N(0,1) data
     have a standard deviation of about 11, so a row's running maximum climbs by
     many powers of two across the context and the chunk kernel has to move the
@@ -184,11 +185,11 @@ def test_varlen_other_scales(scale):
     about 5) still round to within the 1e-2 bound."""
     rows = [(1500, 300), (700, 129), (40, 1), (900, 1)]
     b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=32, num_kv_heads=8,
-                      head_dim=128, dtype="f16", seed=55, device=DEV, pool_factor=1.2)
+                      head_dim=d, dtype="f16", seed=55, device=DEV, pool_factor=1.2)
     b.scale = scale
     out, _, _ = gpu_step(b, varlen=True)
     ref, _, _ = oracle_step(b, varlen=True)
-    assert_close(out, ref, "f16", f"varlen scale {scale}")
+    assert_close(out, ref, "f16", f"varlen scale {scale} head_dim {d}")
 
 
 BLOCK_SIZE_CASES = [
@@ -230,12 +231,17 @@ def test_block_sizes_match_oracle(case, path):
 
 
 HEAD_DIM_256_CASES = [
-    # head_dim 256: the tensor-core decode/varlen kernel for 16-bit types (chunk
-    # rows too), the CUDA-core kernel for fp32 and when it is forced
+    # head_dim 256: the tensor-core decode/varlen kernel for 16-bit types, the
+    # one-tile tcgen05 chunk kernel for rows of >= 128/gs new tokens, the
+    # CUDA-core kernel for fp32 and when it is forced
     ([(700, 37), (1, 1), (2000, 1), (600, 160), (9, 9)], 16, 2, "bf16"),    # group 8
     ([(1300, 1), (33, 1), (4096, 1)], 8, 8, "f16"),                          # MHA, split-K
     ([(520, 20), (17, 17), (1025, 1)], 32, 8, "bf16"),                      # group 4
     ([(700, 1), (40, 9), (1537, 1)], 8, 2, "f32"),                           # fp32
+    # chunk rows of several 64-key tiles with ragged last query tiles
+    ([(900, 300), (5, 1), (2100, 777), (64, 64)], 32, 8, "bf16"),          # group 4
+    ([(640, 200), (130, 130), (3000, 1)], 4, 4, "f16"),                     # MHA: 128-token tiles
+    ([(1000, 64), (700, 300), (8, 8)], 16, 1, "bf16"),                      # group 16: 8-token tiles
 ]
 
 
@@ -285,11 +291,25 @@ def test_wide_split_k_reduce_matches_oracle(case):
     assert_close(out, ref, dtype, f"wide reduce case {case} ({path})")
 
 
-def test_chunk_kernel_agrees_with_decode_kernel_tiles():
+@pytest.mark.parametrize("bs", [8, 32])
+def test_head_dim_256_chunk_block_sizes(bs):
+    """The head_dim-256 chunk kernel's K/V boxes for 8-token blocks (one box
+    per block) and 32-token blocks (two boxes per block)."""
+    rows = [(1300, 300), (700, 37), (33, 1), (200, 129)]
+    b = W.build_batch([W.Request(s, q) for s, q in rows], num_q_heads=16, num_kv_heads=4,
+                      head_dim=256, dtype="bf16", seed=1200 + bs, device=DEV, pool_factor=1.2,
+                      block_size=bs)
+    out, _, _ = gpu_step(b, varlen=True)
+    ref, _, _ = oracle_step(b, varlen=True)
+    assert_close(out, ref, "bf16", f"head_dim 256 chunk, block_size {bs}")
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_chunk_kernel_agrees_with_decode_kernel_tiles(d):
     """The tcgen05 chunk tiles and the decode kernel's 16-row tiles compute the
     same rows; both are within tolerance of each other as well as the oracle."""
     b = W.build_batch([W.Request(s, q) for s, q in [(1536 + 512, 512), (800, 1)]],
-                      num_q_heads=32, num_kv_heads=8, head_dim=128, dtype="bf16", seed=7,
+                      num_q_heads=32, num_kv_heads=8, head_dim=d, dtype="bf16", seed=7,
                       device=DEV, pool_factor=1.1)
     kc, vc = gpu_cache_write(b)
     tc = gpu_attention(b, kc, vc, varlen=True)
