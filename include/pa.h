@@ -52,10 +52,10 @@
  *   block_idx]).  Entries past ceil(len/block_size) are never read.
  * - Grouped-query attention: query head h reads KV head
  *   h / (num_q_heads / num_kv_heads).  num_q_heads % num_kv_heads == 0.
- * - head_dim is 64 or 128, or 256 for bf16/f16 attention over a 16-bit cache
- *   (the tensor-core decode kernel; no FP8 cache, no PA_PATH_SIMT).  dtype:
- *   PA_F32, PA_BF16 or PA_F16; q, k, v, the caches and out all have that dtype.  Arithmetic is fp32 with one
- *   round-to-nearest-even conversion of the output.
+ * - head_dim is 64, 128 or 256, for every dtype, cache type and block size.
+ *   dtype: PA_F32, PA_BF16 or PA_F16; q, k, v, the caches and out all have
+ *   that dtype (an FP8 cache holds e4m3 codes instead).  Arithmetic is fp32
+ *   with one round-to-nearest-even conversion of the output.
  * - Errors: a status other than PA_OK returned by a call means nothing was
  *   launched (argument checks are done on the host before any launch) or a
  *   launch failed (PA_ERR_CUDA).  Checks that need device data (a block id
