@@ -126,6 +126,14 @@ __device__ __forceinline__ void lds128(uint32_t addr, uint32_t (&w)[4]) {
                : "memory");
 }
 
+// The 8x8 16-bit matrix whose row t / 4, columns 2 (t % 4) and + 1 lane t
+// holds, transposed: lane t receives row t / 4 of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -503,119 +511,175 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       }
       const int blk_start = u.kv_begin + j * kBlock;
 
-      // ---- S = Q K^T over this block's 16 tokens
-      // (two partial sums per n-tile, over even and odd k-steps: four
-      // independent MMA chains instead of two halve the latency of this phase)
-      float sacc[2][4], sodd[2][4];
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sacc[t][e] = sodd[t][e] = 0.f;
-      if constexpr (fp8_direct) {
+      uint32_t pa[4];  // P as the A operand of P.V; NARROW: P^T's B fragments in pa[0], pa[2]
+      if constexpr (NARROW) {
+        // ---- S^T = K Q^T over this block's 16 keys: keys g and g + 8 (the
+        // rows) of tile rows 2 quad and 2 quad + 1 (the columns) -- one MMA
+        // per k-step instead of two, as rows 8-15 of the tile are padding.
+        // Its A fragments are the K codes the 16-row form takes as B, its B
+        // fragments Q's rows g.  Even and odd k-steps in two chains.
         const int g = lane >> 2, q4 = lane & 3;
+        float st[2][4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st[0][e] = st[1][e] = 0.f;
 #pragma unroll
         for (int G = 0; G < D / 64; ++G) {
-          uint32_t w[2][4];  // keys g and 8+g, dims 64G + 16 q4 .. +15
+          uint32_t w[2][4];  // keys g and 8 + g, dims 64G + 16 q4 .. +15
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) lds128(kb + swz(nt * 8 + g, 4 * G + q4), w[nt]);
 #pragma unroll
-          for (int s4 = 0; s4 < 4; ++s4)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              uint32_t b0, b1;
-              fp8x4_to_f16x2x2(w[nt][s4], b0, b1);
-              mma_16816<MT>((s4 & 1) ? sodd[nt] : sacc[nt], qa[4 * G + s4], b0, b1);
-            }
+          for (int s4 = 0; s4 < 4; ++s4) {
+            uint32_t ka[4];
+            fp8x4_to_f16x2x2(w[0][s4], ka[0], ka[2]);
+            fp8x4_to_f16x2x2(w[1][s4], ka[1], ka[3]);
+            mma_16816<MT>(st[s4 & 1], ka, qa[4 * G + s4][0], qa[4 * G + s4][2]);
+          }
         }
+        // y[e]: key g + 8 (e / 2), tile row 2 quad + e % 2; m0, l0 and m1, l1
+        // belong to rows 2 quad and 2 quad + 1 here
+        float y[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) y[e] = (st[0][e] + st[1][e]) * sl;
+        if (blk_start + kBlock > u.lim0) {  // some key of this block is past some row's limit
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = blk_start + g + 8 * (e >> 1);
+            if (key >= u.lim0 + (2 * quad + (e & 1)) / s.gs) y[e] = -INFINITY;
+          }
+        }
+        // the same lazy reference maximum as the 16-row form below; a row's
+        // keys are spread over the eight lanes of its quad position
+        const float lx0 = fmaxf(y[0], y[2]), lx1 = fmaxf(y[1], y[3]);
+        if (__any_sync(0xffffffffu, lx0 > m0 + kLazyRaise || lx1 > m1 + kLazyRaise)) {
+          float mx0 = lx0, mx1 = lx1;
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+          }
+          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+          const float a0 = ex2_approx(m0 - (mn0 == -INFINITY ? 0.f : mn0));
+          const float a1 = ex2_approx(m1 - (mn1 == -INFINITY ? 0.f : mn1));
+          l0 *= a0;
+          l1 *= a1;
+#pragma unroll
+          for (int t = 0; t < NO; ++t) {  // O^T columns: rows 2 quad (c0, c2), 2 quad + 1
+            o[t][0] *= a0;
+            o[t][1] *= a1;
+            o[t][2] *= a0;
+            o[t][3] *= a1;
+          }
+          m0 = mn0;
+          m1 = mn1;
+        }
+        const float mu0 = m0 == -INFINITY ? 0.f : m0;
+        const float mu1 = m1 == -INFINITY ? 0.f : m1;
+        const uint32_t plo = pack2<MT>(ex2_approx(y[0] - mu0), ex2_approx(y[1] - mu1));
+        const uint32_t phi = pack2<MT>(ex2_approx(y[2] - mu0), ex2_approx(y[3] - mu1));
+        const float2 flo = unpack2<MT>(plo), fhi = unpack2<MT>(phi);
+        l0 += flo.x + fhi.x;  // this lane's keys; the quad positions are summed at the end
+        l1 += flo.y + fhi.y;
+        // P^T's B fragments (keys 2 quad, 2 quad + 1 and + 8 of tile row g):
+        // the two 8x8 blocks of P^T that plo and phi hold, transposed
+        pa[0] = movmatrix_t(plo);
+        pa[2] = movmatrix_t(phi);
+        pa[1] = pa[3] = 0u;
       } else {
-        const int mi = lane >> 3;
-        const int tk = (lane & 7) + ((mi >> 1) << 3);
-#pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-          uint32_t b0, b1, b2, b3;
-          const int ch = (kk & 3) * 2 + (mi & 1);
-          ldsm_x4(kb + kv_off(tk, kk >> 2, ch, L::kGroupBytes), b0, b1, b2, b3);
-          mma_16816<MT>((kk & 1) ? sodd[0] : sacc[0], qa[kk], b0, b1);
-          mma_16816<MT>((kk & 1) ? sodd[1] : sacc[1], qa[kk], b2, b3);
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sacc[t][e] += sodd[t][e];
-      float x[2][4];
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[t][e] = sacc[t][e] * sl;
-      if (blk_start + kBlock > u.lim0) {  // some key of this block is past some row's limit
+        // ---- S = Q K^T over this block's 16 tokens
+        // (two partial sums per n-tile, over even and odd k-steps: four
+        // independent MMA chains instead of two halve the latency of this phase)
+        float sacc[2][4], sodd[2][4];
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int key = blk_start + t * 8 + 2 * quad + (e & 1);
-            if (key >= (e < 2 ? lim0 : lim1)) x[t][e] = -INFINITY;
-          }
-      }
-      // ---- online softmax (rows r0 and r1 of this thread), against a
-      // reference maximum per row that is raised only when a score of the row
-      // passes it by more than 2^8 (so P <= 256, exact enough in the 16-bit
-      // operand type); until then no shuffle, no rescale.  (In NARROW rows
-      // 8-15 are padding and take no part.)
-      const float lx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-      const float lx1 =
-          NARROW ? -INFINITY : fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-      if (__any_sync(0xffffffffu, lx0 > m0 + kLazyRaise || lx1 > m1 + kLazyRaise)) {
-        float mx0 = lx0, mx1 = lx1;
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        // factor from the old reference to the new: 1 for rows that keep it,
-        // 0 for rows that had none (m = -inf)
-        const float a0 = ex2_approx(m0 - (mn0 == -INFINITY ? 0.f : mn0));
-        const float a1 = ex2_approx(m1 - (mn1 == -INFINITY ? 0.f : mn1));
-        l0 *= a0;
-        l1 *= a1;
-        if constexpr (NARROW) {  // this lane's O^T columns are rows 2 quad, 2 quad + 1
-          const float c0 = __shfl_sync(0xffffffffu, a0, (2 * quad) << 2);
-          const float c1 = __shfl_sync(0xffffffffu, a0, (2 * quad + 1) << 2);
+          for (int e = 0; e < 4; ++e) sacc[t][e] = sodd[t][e] = 0.f;
+        if constexpr (fp8_direct) {
+          const int g = lane >> 2, q4 = lane & 3;
 #pragma unroll
-          for (int t = 0; t < NO; ++t) {
-            o[t][0] *= c0;
-            o[t][1] *= c1;
-            o[t][2] *= c0;
-            o[t][3] *= c1;
+          for (int G = 0; G < D / 64; ++G) {
+            uint32_t w[2][4];  // keys g and 8+g, dims 64G + 16 q4 .. +15
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) lds128(kb + swz(nt * 8 + g, 4 * G + q4), w[nt]);
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4)
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                uint32_t b0, b1;
+                fp8x4_to_f16x2x2(w[nt][s4], b0, b1);
+                mma_16816<MT>((s4 & 1) ? sodd[nt] : sacc[nt], qa[4 * G + s4], b0, b1);
+              }
           }
         } else {
+          const int mi = lane >> 3;
+          const int tk = (lane & 7) + ((mi >> 1) << 3);
 #pragma unroll
-          for (int t = 0; t < NT; ++t) {
+          for (int kk = 0; kk < KSTEPS; ++kk) {
+            uint32_t b0, b1, b2, b3;
+            const int ch = (kk & 3) * 2 + (mi & 1);
+            ldsm_x4(kb + kv_off(tk, kk >> 2, ch, L::kGroupBytes), b0, b1, b2, b3);
+            mma_16816<MT>((kk & 1) ? sodd[0] : sacc[0], qa[kk], b0, b1);
+            mma_16816<MT>((kk & 1) ? sodd[1] : sacc[1], qa[kk], b2, b3);
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[t][e] += sodd[t][e];
+        float x[2][4];
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[t][e] = sacc[t][e] * sl;
+        if (blk_start + kBlock > u.lim0) {  // some key of this block is past some row's limit
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int key = blk_start + t * 8 + 2 * quad + (e & 1);
+              if (key >= (e < 2 ? lim0 : lim1)) x[t][e] = -INFINITY;
+            }
+        }
+        // ---- online softmax (rows r0 and r1 of this thread), against a
+        // reference maximum per row that is raised only when a score of the row
+        // passes it by more than 2^8 (so P <= 256, exact enough in the 16-bit
+        // operand type); until then no shuffle, no rescale.
+        const float lx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+        const float lx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+        if (__any_sync(0xffffffffu, lx0 > m0 + kLazyRaise || lx1 > m1 + kLazyRaise)) {
+          float mx0 = lx0, mx1 = lx1;
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+          // factor from the old reference to the new: 1 for rows that keep it,
+          // 0 for rows that had none (m = -inf)
+          const float a0 = ex2_approx(m0 - (mn0 == -INFINITY ? 0.f : mn0));
+          const float a1 = ex2_approx(m1 - (mn1 == -INFINITY ? 0.f : mn1));
+          l0 *= a0;
+          l1 *= a1;
+#pragma unroll
+          for (int t = 0; t < NO; ++t) {
             o[t][0] *= a0;
             o[t][1] *= a0;
             o[t][2] *= a1;
             o[t][3] *= a1;
           }
+          m0 = mn0;
+          m1 = mn1;
         }
-        m0 = mn0;
-        m1 = mn1;
-      }
-      const float mu0 = m0 == -INFINITY ? 0.f : m0;
-      const float mu1 = m1 == -INFINITY ? 0.f : m1;
-      uint32_t pa[4];
-      pa[0] = pack2<MT>(ex2_approx(x[0][0] - mu0), ex2_approx(x[0][1] - mu0));
-      pa[2] = pack2<MT>(ex2_approx(x[1][0] - mu0), ex2_approx(x[1][1] - mu0));
-      if constexpr (NARROW) {  // rows 8-15 are padding
-        pa[1] = pa[3] = 0u;
-      } else {
+        const float mu0 = m0 == -INFINITY ? 0.f : m0;
+        const float mu1 = m1 == -INFINITY ? 0.f : m1;
+        pa[0] = pack2<MT>(ex2_approx(x[0][0] - mu0), ex2_approx(x[0][1] - mu0));
         pa[1] = pack2<MT>(ex2_approx(x[0][2] - mu1), ex2_approx(x[0][3] - mu1));
+        pa[2] = pack2<MT>(ex2_approx(x[1][0] - mu0), ex2_approx(x[1][1] - mu0));
         pa[3] = pack2<MT>(ex2_approx(x[1][2] - mu1), ex2_approx(x[1][3] - mu1));
+        // the normaliser sums the same rounded weights the P.V product uses
+        const float2 p00 = unpack2<MT>(pa[0]), p01 = unpack2<MT>(pa[1]);
+        const float2 p10 = unpack2<MT>(pa[2]), p11 = unpack2<MT>(pa[3]);
+        l0 += (p00.x + p00.y) + (p10.x + p10.y);
+        l1 += (p01.x + p01.y) + (p11.x + p11.y);
       }
-      // the normaliser sums the same rounded weights the P.V product uses
-      const float2 p00 = unpack2<MT>(pa[0]), p01 = unpack2<MT>(pa[1]);
-      const float2 p10 = unpack2<MT>(pa[2]), p11 = unpack2<MT>(pa[3]);
-      l0 += (p00.x + p00.y) + (p10.x + p10.y);
-      l1 += (p01.x + p01.y) + (p11.x + p11.y);
       // ---- O += P V ; V rows at or past the unit's last visible key are
       // zeroed (padding may hold anything, and 0 * NaN is NaN)
       uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
@@ -710,15 +774,29 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
         for (int e = 0; e < 4; ++e) o[t][e] *= vsc;
     }
     // ---- merge the warps' states
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    if (quad == 0) {
-      cm[warp * kRows + r0] = m0;
-      cl[warp * kRows + r0] = l0;
-      cm[warp * kRows + r1] = m1;
-      cl[warp * kRows + r1] = l1;
+    if constexpr (NARROW) {  // rows 2 quad, 2 quad + 1; keys over the eight lanes g
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      if (lane < 4) {
+        cm[warp * kRows + 2 * quad] = m0;
+        cl[warp * kRows + 2 * quad] = l0;
+        cm[warp * kRows + 2 * quad + 1] = m1;
+        cl[warp * kRows + 2 * quad + 1] = l1;
+      }
+    } else {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      if (quad == 0) {
+        cm[warp * kRows + r0] = m0;
+        cl[warp * kRows + r0] = l0;
+        cm[warp * kRows + r1] = m1;
+        cl[warp * kRows + r1] = l1;
+      }
     }
     if constexpr (NARROW) {
       // m-tile mt holds dims 16g + 2mt (c0, c1) and 16g + 2mt + 1 (c2, c3) of
