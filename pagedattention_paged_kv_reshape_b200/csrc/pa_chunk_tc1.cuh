@@ -175,13 +175,11 @@ __global__ void __launch_bounds__(256, 1)
 
   const int count = __ldcg(&w.sched->chunk_count);
   const int items = count * head_units(s);
-  // the k-th item of this CTA is blockIdx.x + k * gridDim.x
-  const int my_items = static_cast<int>(blockIdx.x) < items
-                           ? (items - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
-                           : 0;
+  // the k-th item of this CTA (chunk_item_index)
+  const int my_items = chunk_items_of_cta(items);
   const int qt = kTcRows / s.gs;  // query tokens per tile
   auto item_of = [&](int k) {
-    return tc1_item(s, w, qsl, seq_lens, count, static_cast<int>(blockIdx.x) + k * gridDim.x, qt);
+    return tc1_item(s, w, qsl, seq_lens, count, chunk_item_index(k), qt);
   };
 
   if (warp == 0) {

@@ -147,6 +147,24 @@ __device__ __forceinline__ Tc2Item tc2_item(const Shape& s, const Work& w,
   return it;
 }
 
+// The k-th item of this CTA: rounds of gridDim.x items, visited in
+// alternating directions (CTA b takes item b of even rounds and item
+// gridDim.x - 1 - b of odd ones), so that a CTA that drew long items in one
+// round draws short ones in the next (causal items grow along a chunk row;
+// on prefill_16x512 the longest CTA has 3% more key tiles than the mean,
+// against 6% for a plain round robin).
+__device__ __forceinline__ int chunk_item_index(int k) {
+  const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  return k * g + ((k & 1) ? g - 1 - b : b);
+}
+
+// How many items chunk_item_index gives this CTA out of `items`.
+__device__ __forceinline__ int chunk_items_of_cta(int items) {
+  const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  const int rounds = items / g, rem = items - rounds * g;
+  return rounds + ((rounds & 1) ? (b >= g - rem) : (b < rem));
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(384, 1)
     chunk_tc2_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -206,13 +224,11 @@ __global__ void __launch_bounds__(384, 1)
 
   const int count = __ldcg(&w.sched->chunk_count);
   const int items = count * head_units(s);
-  // the k-th item of this CTA is blockIdx.x + k * gridDim.x
-  const int my_items = static_cast<int>(blockIdx.x) < items
-                           ? (items - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
-                           : 0;
+  // the k-th item of this CTA (chunk_item_index)
+  const int my_items = chunk_items_of_cta(items);
   const int qt = kTcRows / s.gs;  // query tokens per tile
   auto item_of = [&](int k) {
-    return tc2_item(s, w, qsl, seq_lens, count, static_cast<int>(blockIdx.x) + k * gridDim.x, qt);
+    return tc2_item(s, w, qsl, seq_lens, count, chunk_item_index(k), qt);
   };
 
   if (warp < 4) {
