@@ -355,9 +355,10 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
     if (p.s.gs * p.s.qpt <= 8) return launch_mma<T, D, KV8, true>(a, p, w);
   }
   // FP8 stages are half as large: at head_dim 128 twice as many keep the same
-  // bytes in flight; at 64 the per-warp f16 staging tiles take that room
-  constexpr int kS = KV8 && D == 128 ? 2 * kStages : kStages;
-  using L = pa::MmaLayout<D, kNcw, kS, KV8>;
+  // bytes in flight; at 64 the per-warp f16 staging tiles take that room.  The
+  // NARROW form runs three CTAs per SM with 8 stages each.
+  constexpr int kS = NARROW ? 8 : (KV8 && D == 128 ? 2 * kStages : kStages);
+  using L = pa::MmaLayout<D, kNcw, kS, KV8, NARROW>;
   auto kern = pa::attn_mma_kernel<T, D, kNcw, kS, KV8, NARROW>;
   int occ = 0;
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);

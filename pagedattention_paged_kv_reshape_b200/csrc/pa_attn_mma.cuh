@@ -49,7 +49,7 @@ struct MetaSlot {
 // below); at head_dim 64 and 256 they are unswizzled and each consumer warp
 // first converts its tile into a 16-bit staging tile laid out like a 16-bit
 // stage.
-template <int D, int NCW, int STAGES, bool KV8 = false>
+template <int D, int NCW, int STAGES, bool KV8 = false, bool NARROW = false>
 struct MmaLayout {
   static constexpr bool kStaging = KV8 && D != 128;
   static constexpr int kHalves = D / 64;             // 64 16-bit elements = one 128 B swizzle row
@@ -63,10 +63,11 @@ struct MmaLayout {
   static constexpr int kQSlots = 2;
   static constexpr int kOffQ = STAGES * kStageBytes;
   static constexpr int kOffCo = kOffQ + kQSlots * kQSlotBytes;
-  static constexpr int kCoBytes = NCW * kRows * (D + 8) * 4;
+  static constexpr int kCoRows = NARROW ? 8 : kRows;  // tile rows the merge buffer holds
+  static constexpr int kCoBytes = NCW * kCoRows * (D + 8) * 4;
   static constexpr int kOffCm = kOffCo + kCoBytes;
-  static constexpr int kOffCl = kOffCm + NCW * kRows * 4;
-  static constexpr int kOffBar = kOffCl + NCW * kRows * 4;
+  static constexpr int kOffCl = kOffCm + NCW * kCoRows * 4;
+  static constexpr int kOffBar = kOffCl + NCW * kCoRows * 4;
   // full[S], empty[S], qfull[2], qempty[2], meta_full[M], meta_empty[M], consumers
   static constexpr int kNumBars = 2 * STAGES + 2 * kQSlots + 2 * kMetaSlots + 1;
   static constexpr int kOffDesc = kOffBar + kNumBars * 8;
@@ -84,8 +85,9 @@ struct MmaLayout {
   // warp can wait on a stage's phase while another warp still holds the
   // previous one (across units the consumers meet at the epilogue barrier).
   static_assert(STAGES % NCW == 0, "a stage must stay with one consumer warp inside a unit");
-  // two CTAs per SM up to head_dim 128; one at 256
+  // two CTAs per SM up to head_dim 128 (three in the NARROW form); one at 256
   static_assert(D > 128 || kSmem <= 116 * 1024, "two CTAs per SM");
+  static_assert(!NARROW || kSmem <= 75 * 1024, "three CTAs per SM");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -178,14 +180,14 @@ __device__ __forceinline__ void convert_fp8_tile(uint32_t src, uint32_t dst, int
 }
 
 template <typename T, int D, int NCW, int STAGES, bool KV8 = false, bool NARROW = false>
-__global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
+__global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 3 : (D > 128 ? 1 : 2))
     attn_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, Shape s, T* __restrict__ out,
                     const int* __restrict__ block_tables, const int* __restrict__ qsl,
                     const int* __restrict__ seq_lens, Work w, float scale_log2,
                     const float* __restrict__ k_scale, const float* __restrict__ v_scale) {
-  using L = MmaLayout<D, NCW, STAGES, KV8>;
+  using L = MmaLayout<D, NCW, STAGES, KV8, NARROW>;
   // operand type of the MMAs: the input type, or f16 for an FP8 cache (every
   // e4m3 value is exact in f16; q and P are converted to it)
   using MT = typename std::conditional<KV8, __half, T>::type;
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffFlags);
   float* cm = reinterpret_cast<float*>(smem + L::kOffCm);
   float* cl = reinterpret_cast<float*>(smem + L::kOffCl);
-  auto co = reinterpret_cast<float(*)[kRows][D + 8]>(smem + L::kOffCo);
+  auto co = reinterpret_cast<float(*)[L::kCoRows][D + 8]>(smem + L::kOffCo);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
@@ -781,10 +783,10 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
         l1 += __shfl_xor_sync(0xffffffffu, l1, off);
       }
       if (lane < 4) {
-        cm[warp * kRows + 2 * quad] = m0;
-        cl[warp * kRows + 2 * quad] = l0;
-        cm[warp * kRows + 2 * quad + 1] = m1;
-        cl[warp * kRows + 2 * quad + 1] = l1;
+        cm[warp * L::kCoRows + 2 * quad] = m0;
+        cl[warp * L::kCoRows + 2 * quad] = l0;
+        cm[warp * L::kCoRows + 2 * quad + 1] = m1;
+        cl[warp * L::kCoRows + 2 * quad + 1] = l1;
       }
     } else {
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -832,7 +834,8 @@ __global__ void __launch_bounds__((NCW + 2) * 32, D > 128 ? 1 : 2)
       }
     }
     if (!consumers_sync()) return;
-    epilogue<T, D, NCW, fp8_direct && !NARROW>(s, u, cm, cl, co, out, w, tid, NCW * 32);
+    epilogue<T, D, NCW, fp8_direct && !NARROW, L::kCoRows>(s, u, cm, cl, co, out, w, tid,
+                                                           NCW * 32);
     if (!consumers_sync()) return;
   }
 }

@@ -364,14 +364,14 @@ __device__ __forceinline__ int co_swizzled(int ch) {
   return 4 * ((ch & ~7) | ((ch & 7) ^ x));
 }
 
-template <typename T, int D, int NW, bool kSwizzledCo = false>
+template <typename T, int D, int NW, bool kSwizzledCo = false, int CR = kRows>
 __device__ __forceinline__ void epilogue(const Shape& s, const Unit& u, const float* cm,
-                                         const float* cl, const float (*co)[kRows][D + 8],
+                                         const float* cl, const float (*co)[CR][D + 8],
                                          T* __restrict__ out, const Work& w, int tid,
                                          int nthreads) {
   static_assert(!kSwizzledCo || D <= 128, "the swizzle covers four runs of 32 dims");
   constexpr int kChunks = D / 8;
-  for (int task = tid; task < kRows * kChunks; task += nthreads) {
+  for (int task = tid; task < CR * kChunks; task += nthreads) {
     const int r = task / kChunks, c = task % kChunks;
     const int i = r / s.gs, g = r % s.gs;
     if (i >= u.nq || g >= u.rows) continue;
@@ -379,15 +379,15 @@ __device__ __forceinline__ void epilogue(const Shape& s, const Unit& u, const fl
     if (u.p >= parts) continue;  // no key of this partition is visible to the row
     float mx = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < NW; ++q) mx = fmaxf(mx, cm[q * kRows + r]);
+    for (int q = 0; q < NW; ++q) mx = fmaxf(mx, cm[q * CR + r]);
     float L = 0.f;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
     for (int q = 0; q < NW; ++q) {
-      const float f = exp2f(cm[q * kRows + r] - mx);
-      L += f * cl[q * kRows + r];
+      const float f = exp2f(cm[q * CR + r] - mx);
+      L += f * cl[q * CR + r];
       const int oa = kSwizzledCo ? co_swizzled(2 * c) : c * 8;
       const int ob = kSwizzledCo ? co_swizzled(2 * c + 1) : c * 8 + 4;
       const float4 a = *reinterpret_cast<const float4*>(&co[q][r][oa]);
