@@ -500,9 +500,8 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 3 : (D > 128 ? 1 : 2)
       }
       // FP8 direct: this lane's V bytes come into registers as soon as the
       // stage lands (keys 2q4, 2q4+1, 2q4+8, 2q4+9; head dims 16g .. 16g+15).
-      // (Reading them late, after the softmax, gave sporadically wrong units,
-      // and so did releasing the stage right after Q K^T; the stage is
-      // released at the end of the tile, as on the 16-bit path.)
+      // In the NARROW form the stage is then released right after QK^T, its
+      // last reader; the 16-row form releases it at the end of the tile.
       uint32_t va[4], vb1[4], vc[4], vd[4];
       if constexpr (fp8_direct) {
         const int g = lane >> 2, q4 = lane & 3;
@@ -521,9 +520,9 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 3 : (D > 128 ? 1 : 2)
         // Its A fragments are the K codes the 16-row form takes as B, its B
         // fragments Q's rows g.  Even and odd k-steps in two chains.
         const int g = lane >> 2, q4 = lane & 3;
-        float st[2][4];
+        float sk[2][4];  // even / odd k-steps
 #pragma unroll
-        for (int e = 0; e < 4; ++e) st[0][e] = st[1][e] = 0.f;
+        for (int e = 0; e < 4; ++e) sk[0][e] = sk[1][e] = 0.f;
 #pragma unroll
         for (int G = 0; G < D / 64; ++G) {
           uint32_t w[2][4];  // keys g and 8 + g, dims 64G + 16 q4 .. +15
@@ -534,14 +533,14 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 3 : (D > 128 ? 1 : 2)
             uint32_t ka[4];
             fp8x4_to_f16x2x2(w[0][s4], ka[0], ka[2]);
             fp8x4_to_f16x2x2(w[1][s4], ka[1], ka[3]);
-            mma_16816<MT>(st[s4 & 1], ka, qa[4 * G + s4][0], qa[4 * G + s4][2]);
+            mma_16816<MT>(sk[s4 & 1], ka, qa[4 * G + s4][0], qa[4 * G + s4][2]);
           }
         }
         // y[e]: key g + 8 (e / 2), tile row 2 quad + e % 2; m0, l0 and m1, l1
         // belong to rows 2 quad and 2 quad + 1 here
         float y[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) y[e] = (st[0][e] + st[1][e]) * sl;
+        for (int e = 0; e < 4; ++e) y[e] = (sk[0][e] + sk[1][e]) * sl;
         if (blk_start + kBlock > u.lim0) {  // some key of this block is past some row's limit
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -586,6 +585,11 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 3 : (D > 128 ? 1 : 2)
         pa[0] = movmatrix_t(plo);
         pa[2] = movmatrix_t(phi);
         pa[1] = pa[3] = 0u;
+        // every read of this stage is done: V is in registers and the K codes
+        // fed the MMAs above (each of which waited for its loads), so the
+        // stage goes back to the TMA warp now rather than after P.V
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(st));
       } else {
         // ---- S = Q K^T over this block's 16 tokens
         // (two partial sums per n-tile, over even and odd k-steps: four
@@ -764,7 +768,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 3 : (D > 128 ? 1 : 2)
           pv16(false);
       }
       __syncwarp();  // (FP8 through staging: every lane is done with the staging tiles)
-      if (!L::kStaging && lane == 0) mbar_arrive(empty_bar(st));
+      if (!L::kStaging && !NARROW && lane == 0) mbar_arrive(empty_bar(st));
     }
     n += nblk;
 
