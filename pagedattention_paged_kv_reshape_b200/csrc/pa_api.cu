@@ -356,10 +356,12 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   }
   // FP8 stages are half as large: at head_dim 128 twice as many keep the same
   // bytes in flight; at 64 the per-warp f16 staging tiles take that room.  The
-  // NARROW form runs three CTAs per SM with 8 stages each.
-  constexpr int kS = NARROW ? 8 : (KV8 && D == 128 ? 2 * kStages : kStages);
-  using L = pa::MmaLayout<D, kNcw, kS, KV8, NARROW>;
-  auto kern = pa::attn_mma_kernel<T, D, kNcw, kS, KV8, NARROW>;
+  // NARROW form runs four CTAs per SM of three consumer warps and 6 stages:
+  // its throughput follows the number of CTAs (each with its own TMA thread).
+  constexpr int kN = NARROW ? 3 : kNcw;
+  constexpr int kS = NARROW ? 6 : (KV8 && D == 128 ? 2 * kStages : kStages);
+  using L = pa::MmaLayout<D, kN, kS, KV8, NARROW>;
+  auto kern = pa::attn_mma_kernel<T, D, kN, kS, KV8, NARROW>;
   int occ = 0;
   cudaError_t e = prepare(kern, L::kThreads, L::kSmem, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "mma kernel set-up");

@@ -85,9 +85,9 @@ struct MmaLayout {
   // warp can wait on a stage's phase while another warp still holds the
   // previous one (across units the consumers meet at the epilogue barrier).
   static_assert(STAGES % NCW == 0, "a stage must stay with one consumer warp inside a unit");
-  // two CTAs per SM up to head_dim 128 (three in the NARROW form); one at 256
+  // two CTAs per SM up to head_dim 128 (four in the NARROW form); one at 256
   static_assert(D > 128 || kSmem <= 116 * 1024, "two CTAs per SM");
-  static_assert(!NARROW || kSmem <= 75 * 1024, "three CTAs per SM");
+  static_assert(!NARROW || kSmem <= 56 * 1024, "four CTAs per SM");
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -180,7 +180,7 @@ __device__ __forceinline__ void convert_fp8_tile(uint32_t src, uint32_t dst, int
 }
 
 template <typename T, int D, int NCW, int STAGES, bool KV8 = false, bool NARROW = false>
-__global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 3 : (D > 128 ? 1 : 2))
+__global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 4 : (D > 128 ? 1 : 2))
     attn_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, Shape s, T* __restrict__ out,
