@@ -57,9 +57,6 @@ constexpr int kTcRows = 128;       // query-tile rows = TMEM lanes
 constexpr int kTcKeys = 128;       // keys per K/V tile = 8 blocks of 16
 constexpr float kTcRescale = 8.f;  // raise the reference maximum past this (log2 units)
 
-// Pairs of softmax exponentials, of every 8, computed on the FMA pipe
-// (exp2_poly2) instead of the special-function unit.
-constexpr int kPolyPairs = 0;
 
 template <int D>
 struct Tc2Layout {
@@ -570,10 +567,8 @@ __global__ void __launch_bounds__(384, 1)
           }
           l *= alpha;
           // P = 2^(v * sc - m), rounded to the input type, over the first 64
-          // columns of S (the scores are all in registers by now).  The
-          // exponentials run on the special-function unit, except kPolyPairs of
-          // every 8 pairs, which take exp2_poly2 on the FMA pipe.  The row sum
-          // adds the weights before their rounding to the input type (the
+          // columns of S (the scores are all in registers by now).  The row
+          // sum adds the weights before their rounding to the input type (the
           // rounding is unbiased; its effect on the normalised output is of
           // order 2^-9 / sqrt(keys)).
           const float nm = m == -INFINITY ? 0.f : -m;
@@ -587,8 +582,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int j = 0; j < 32; ++j) {
               const float2 a =
                   ffma2(make_float2(v[64 * hh + 2 * j], v[64 * hh + 2 * j + 1]), sc2, nm2);
-              float2 e = (j & 7) < kPolyPairs ? exp2_poly2(a)
-                                              : make_float2(ex2_approx(a.x), ex2_approx(a.y));
+              const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
               pk[j] = pack2<T>(e.x, e.y);
               ps[j & 3] = fadd2(ps[j & 3], e);
             }

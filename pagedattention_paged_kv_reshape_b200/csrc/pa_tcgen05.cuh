@@ -262,62 +262,11 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return r;
 }
 
-// d = a - b on two lanes at once (one sub.rn.f32x2).
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-  uint64_t d;
-  asm("{\n\t.reg .b64 ra, rb;\n\t"
-      "mov.b64 ra, {%1, %2};\n\t"
-      "mov.b64 rb, {%3, %4};\n\t"
-      "sub.rn.f32x2 %0, ra, rb;\n\t}"
-      : "=l"(d)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-  return r;
-}
-
-// Coefficients of the cubic c0 + c1 f + c2 f^2 + c3 f^3 that approximates 2^f
-// on [-1/2, 1/2] with the smallest largest relative error: a minimax fit,
-// computed as a linear program (minimise t subject to |p(f_i) / 2^f_i - 1| <=
-// t) on 4001 evenly spaced points f_i, then rounded to fp32.  Largest
-// relative error 7.5e-5 (fp32 evaluation included), well under the 2^-9 of
-// the bf16 rounding the weights go through next.  The test of the kernel
-// helpers recomputes the bound from these constants.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
-
-// 2^x for two values on the FMA pipe, leaving the special-function unit to
-// the other exponentials of a row.  Range reduction in the manner of Cody and
-// Waite: x = j + f with j the nearest integer (adding 1.5 * 2^23 leaves
-// round(x) in the low mantissa bits of t), f in [-1/2, 1/2]; 2^f from the
-// cubic above; 2^j added to the exponent field as t's bits times 2^23 (the
-// bits of 1.5 * 2^23 vanish in that product modulo 2^32).  x is clamped below
-// at -125, where 2^f's exponent field (126 or 127) plus j stays positive: the
-// result is then a weight of order 2^-125, not 0 (callers zero masked
-// entries themselves).  Valid for x < 127.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 shift = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
-  const float2 t = fadd2(x, shift);
-  const float2 f = fsub2(x, fsub2(t, shift));
-  float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
-  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
-  uint32_t rx, ry;
-  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(p.x)));
-  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(p.y)));
-  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
-}
-
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-
 
 }  // namespace pa
