@@ -84,6 +84,12 @@ FP8_CASES = [
     ([(1000, 1), (4096, 1), (77, 1)], 32, 4, 128, "f16", 16),
     ([(700, 37), (1, 1), (2000, 1), (600, 160), (9, 9)], 16, 2, 256, "bf16", 16),  # head_dim 256
     ([(1300, 1), (33, 1), (4096, 1)], 8, 8, 256, "f32", 8),
+    # decode at head_dim 128 on both sides of the transposed (<= 8 rows) form:
+    # group 16 (16-row tiles), MHA with 8-token blocks, group 6 with 32-token
+    # blocks, with split-K rows, one-token contexts and ragged last blocks
+    ([(3000, 1), (17, 1), (513, 1), (1, 1)], 16, 1, 128, "bf16", 16),
+    ([(2049, 1), (5, 1), (700, 1)], 8, 8, 128, "f16", 8),
+    ([(1500, 1), (64, 1), (1, 1)], 24, 4, 128, "bf16", 32),
 ]
 
 
