@@ -52,26 +52,28 @@ struct Tc1Layout {
   static constexpr int kQBytes = kHalves * kHalfBytes;     // 64 KB
   static constexpr int kGroupBytes = kHalves * 1024;       // 8 rows of a K or V tile
   static constexpr int kKVBytes = kTc1Keys / 8 * kGroupBytes;  // 32 KB
-  static constexpr int kStages = 2;                        // of K and of V
+  // (a third K stage measured within 1%: the K loads are not what waits)
+  static constexpr int kKStages = 2;                       // a K tile is free once its S ran
+  static constexpr int kVStages = 2;                       // a V tile, once its P.V ran
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kKVBytes;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarQFree = 1;                      // the item's last S done
-  static constexpr int kBarKFull = 2;                      // [2]
-  static constexpr int kBarKEmpty = 4;                     // [2]
-  static constexpr int kBarVFull = 6;                      // [2]
-  static constexpr int kBarVEmpty = 8;                     // [2]
-  static constexpr int kBarSFull = 10;                     // [2] one per S buffer
-  static constexpr int kBarPFull = 12;                     // [2] four warps each
+  static constexpr int kBarKFull = 2;                      // [kKStages]
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;  // [kKStages]
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;  // [2]
+  static constexpr int kBarVEmpty = kBarVFull + 2;         // [2]
+  static constexpr int kBarSFull = kBarVEmpty + 2;         // [2] one per S buffer
+  static constexpr int kBarPFull = kBarSFull + 2;          // [2] four warps each
   // [2] P.V of tiles g with g % 2 = 0, 1.  S runs two tiles ahead of P.V, so
   // when the softmax waits for P.V(g) only P.V(g - 2) is known complete (S(g)
   // followed it): one barrier for every P.V could already show P.V(g - 2)'s
   // phase, of the same parity, while P.V(g - 1) is still running.
-  static constexpr int kBarPDone = 14;
-  static constexpr int kBarDrain = 16;
-  static constexpr int kNumBars = 17;
+  static constexpr int kBarPDone = kBarPFull + 2;
+  static constexpr int kBarDrain = kBarPDone + 2;
+  static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffItems = kOffBar + kNumBars * 8;
   static constexpr int kItemBytes = 64;
   static constexpr int kItemSlots = 8;
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(256, 1)
                      const int* __restrict__ block_tables, const int* __restrict__ qsl,
                      const int* __restrict__ seq_lens, Work w, float scale_log2) {
   using L = Tc1Layout<D>;
-  constexpr int NS = L::kStages;
+  constexpr int KS = L::kKStages, VS = L::kVStages;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescS = instr_desc_f16(kBf16, false, false, kTcRows, kTc1Keys);
   constexpr uint32_t kIdescPV = instr_desc_f16(kBf16, false, true, kTcRows, D);
@@ -196,10 +198,10 @@ __global__ void __launch_bounds__(256, 1)
     Pending va{0, 0, 0};
     bool pend = false;
     auto issue_v = [&](const Pending& p) -> bool {
-      const int vs = p.gt % NS;
+      const int vs = p.gt % VS;
       bool r = true;
       if (lane == 0) {
-        r = mbar_wait(vempty(vs), ((p.gt / NS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+        r = mbar_wait(vempty(vs), ((p.gt / VS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
         if (r)
           mbar_arrive_expect_tx(vfull(vs),
                                 static_cast<uint32_t>(p.nb * L::kHalves * box_rows * 128));
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(256, 1)
     int g = 0;  // K/V tiles of earlier items
     for (int k = 0; k < my_items && ok; ++k) {
       for (int t = 0; t < it.nkt && ok; ++t) {
-        const int gt = g + t, ks = gt % NS;
+        const int gt = g + t, ks = gt % KS;
         // one lane per TMA box of the tile: its cache row, then its K box
         const int key0 = t * kTc1Keys;
         const int nb = min(kTc1Keys / box_rows, ceil_div(it.kv_end - key0, box_rows));
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(256, 1)
                       it.row);
         bool r = true;
         if (lane == 0) {
-          r = mbar_wait(kempty(ks), ((gt / NS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+          r = mbar_wait(kempty(ks), ((gt / KS) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
           if (r && gt != lost)
             mbar_arrive_expect_tx(kfull(ks),
                                   static_cast<uint32_t>(nb * L::kHalves * box_rows * 128));
@@ -254,10 +256,10 @@ __global__ void __launch_bounds__(256, 1)
       // a wait gave up: let the copies already issued land (bounded again,
       // independently of the abort flag)
       volatile int own_flag = 0;
-      for (int i = max(0, k_last - NS + 1); i <= k_last; ++i)
-        if (i != lost) mbar_wait(kfull(i % NS), (i / NS) & 1, kWhereWaitFull, &own_flag);
-      for (int i = max(0, v_last - NS + 1); i <= v_last; ++i)
-        mbar_wait(vfull(i % NS), (i / NS) & 1, kWhereWaitFull, &own_flag);
+      for (int i = max(0, k_last - KS + 1); i <= k_last; ++i)
+        if (i != lost) mbar_wait(kfull(i % KS), (i / KS) & 1, kWhereWaitFull, &own_flag);
+      for (int i = max(0, v_last - VS + 1); i <= v_last; ++i)
+        mbar_wait(vfull(i % VS), (i / VS) & 1, kWhereWaitFull, &own_flag);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ Q loads
@@ -314,8 +316,8 @@ __global__ void __launch_bounds__(256, 1)
         return true;
       };
       auto issue_s = [&](const Cursor& c) -> bool {
-        const int ks = c.g % NS;
-        if (!mbar_wait(kfull(ks), (c.g / NS) & 1, kWhereWaitFull, abort_flag)) return false;
+        const int ks = c.g % KS;
+        if (!mbar_wait(kfull(ks), (c.g / KS) & 1, kWhereWaitFull, abort_flag)) return false;
         const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024);
         const uint64_t kd = smem_desc_sw128(k_smem(ks), 16, L::kGroupBytes);
         const uint32_t ts = t_s(c.g & 1);
@@ -332,14 +334,14 @@ __global__ void __launch_bounds__(256, 1)
         return true;
       };
       auto issue_pv = [&](const Cursor& c) -> bool {
-        const int vs = c.g % NS;
+        const int vs = c.g % VS;
         const int key0 = c.t * kTc1Keys;
         const int valid = min(kTc1Keys, c.kv_end - key0);
         const int steps = (valid + 15) >> 4;  // 16-key MMA steps holding visible keys
         const uint64_t vd = smem_desc_sw128(v_smem(vs), 1024, L::kGroupBytes);
         const uint32_t acc0 = c.t > 0 ? 1u : 0u;  // the item's first tile starts O afresh
         const uint32_t ts = t_s(c.g & 1);
-        if (!mbar_wait(vfull(vs), (c.g / NS) & 1, kWhereWaitFull, abort_flag)) return false;
+        if (!mbar_wait(vfull(vs), (c.g / VS) & 1, kWhereWaitFull, abort_flag)) return false;
         if (c.t == c.nkt - 1) {
           // the item's last V tile: zero the rows of its last 16-key step past
           // the item's last key (padding slots, or rows no box covered)
