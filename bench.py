@@ -440,6 +440,19 @@ def combine_over_ranks(local_ms: float, local_bytes: float, local_tokens: float,
     return max_ms, nb.item() / (max_ms / 1e3) / 1e9, tok.item() / (max_ms / 1e3)
 
 
+def measure_device_copy(torch, dev) -> float:
+    """Context for the peak: torch's device-to-device copy of a 2 GiB buffer
+    (read + write bytes over time), on this machine, in this run."""
+    n = 1 << 31
+    src = torch.empty(n, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    time.sleep(REST_S)
+    ms = timed_loop(torch, lambda: dst.copy_(src), 10)
+    del src, dst
+    torch.cuda.empty_cache()
+    return round(2 * n / (ms * 1e-3) / 1e9, 1)
+
+
 def measure_block_ops(torch, pa, dev, peak) -> dict:
     """Copy-on-write copies inside the device pool and swaps to / from a pinned
     host pool, each on 2048 / 1024 blocks of 8 KV heads x 16 x 128 bf16
@@ -652,7 +665,8 @@ def run_ours(args):
         result["per_config"] = per
         result["block_ops"] = measure_block_ops(torch, pa, dev, peak)
         result["rope_cache_write"] = measure_rope_write(torch, pa, dev, peak)
-        result["peaks"] = {"hbm_gbs": peak, "bf16_tflops": tensor_peak, "kind": peak_kind}
+        result["peaks"] = {"hbm_gbs": peak, "bf16_tflops": tensor_peak, "kind": peak_kind,
+                           "device_copy_gbs": measure_device_copy(torch, dev)}
     result["clocks"] = sampler.stop() if sampler else None
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
