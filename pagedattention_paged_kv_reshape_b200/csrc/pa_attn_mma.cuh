@@ -33,6 +33,7 @@ namespace pa {
 
 constexpr int kMetaSlots = 4;
 constexpr float kLazyRaise = 8.f;  // see the online softmax of attn_mma_kernel (log2 units)
+constexpr int kIssueLanes = 2;     // lanes of the TMA warp that issue K/V loads
 
 // One scheduler-ring slot: a decoded unit and, for each 16-key tile of its
 // partition, the cache row of the tile's first key (y0) and, with 8-token
@@ -314,77 +315,115 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 4 : (D > 128 ? 1 : 2)
 
   if (warp == NCW) {
     // ----------------------------------------------------------------- TMA
-    if (lane != 0) return;
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
-    prefetch_tensormap(&tm_q);
+    // kIssueLanes lanes: lane 0 handles each unit's metadata and query tile,
+    // lane i issues the unit's tiles i, i + kIssueLanes, ...  (The loads of a
+    // tile keep the issuing thread busy for a few hundred cycles; with the
+    // FP8 form's 4 KB stages one thread could not keep up with its consumers.)
+    if (lane >= kIssueLanes) return;
+    constexpr unsigned kIssueMask = (1u << kIssueLanes) - 1u;
+    if (lane == 0) {
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      prefetch_tensormap(&tm_q);
+    }
     const uint32_t q_bytes = static_cast<uint32_t>(L::kHalves * 128 * s.gs * s.qpt);
+    // issued: tiles 0 .. issued-1 all have their loads issued (for the drain)
     int n = 0, issued = 0;
     // test hook: every CTA leaves its first tile unissued (see g_debug_lost_load)
     const int lost = g_debug_lost_load == 1 ? 0 : -1;
     bool ok = true;
     for (int j = 0; ok; ++j) {
       const int ms = j % kMetaSlots;
-      if (!(ok = mbar_wait(mfull_bar(ms), (j / kMetaSlots) & 1, kWhereWaitQ, abort_flag))) break;
+      ok = __all_sync(kIssueMask,
+                      mbar_wait(mfull_bar(ms), (j / kMetaSlots) & 1, kWhereWaitQ, abort_flag));
+      if (!ok) break;
       const Unit un = meta[ms].u;
       const int qs = j & 1;
-      if (!(ok = mbar_wait(qempty_bar(qs), ((j >> 1) & 1) ^ 1, kWhereWaitQ, abort_flag))) break;
-      desc[qs] = un;
+      ok = __all_sync(kIssueMask, mbar_wait(qempty_bar(qs), ((j >> 1) & 1) ^ 1, kWhereWaitQ,
+                                            abort_flag));
+      if (!ok) break;
       if (un.row < 0) {
-        mbar_arrive(qfull_bar(qs));
+        if (lane == 0) {
+          desc[qs] = un;
+          mbar_arrive(qfull_bar(qs));
+        }
         break;
       }
-      mbar_arrive_expect_tx(qfull_bar(qs), q_bytes);
-      const uint32_t qdst = sbase + L::kOffQ + qs * L::kQSlotBytes;
+      if (lane == 0) {
+        desc[qs] = un;
+        mbar_arrive_expect_tx(qfull_bar(qs), q_bytes);
+        const uint32_t qdst = sbase + L::kOffQ + qs * L::kQSlotBytes;
 #pragma unroll
-      for (int h = 0; h < L::kHalves; ++h)
-        tma_load_3d(qdst + h * (kRows * 128), &tm_q, qfull_bar(qs), h * 64, un.head0, un.token0);
+        for (int h = 0; h < L::kHalves; ++h)
+          tma_load_3d(qdst + h * (kRows * 128), &tm_q, qfull_bar(qs), h * 64, un.head0,
+                      un.token0);
+      }
       const int nblk = ceil_div(un.kv_end - un.kv_begin, kBlock);
-      for (int jj = 0; jj < nblk; ++jj, ++n) {
-        const int y = meta[ms].y0[jj];
-        const int st = n % STAGES;
-        if (!(ok = mbar_wait(empty_bar(st), ((n / STAGES) & 1) ^ 1, kWhereWaitEmpty, abort_flag)))
-          break;
-        ++issued;
-        if (n == lost) continue;
-        const uint32_t kdst = sbase + st * L::kStageBytes;
-        const uint32_t vdst = kdst + L::kKVTileBytes;
-        if constexpr (KV8) {
-          // one box of D bytes x 16 rows, or of 8 rows twice with 8-token blocks
-          if (s.block_size >= kBlock) {
-            mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
-            tma_load_2d(kdst, &tm_k, full_bar(st), 0, y);
-            tma_load_2d(vdst, &tm_v, full_bar(st), 0, y);
-          } else {
-            const int y1 = meta[ms].y1[jj];
-            mbar_arrive_expect_tx(full_bar(st), y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
-            tma_load_2d(kdst, &tm_k, full_bar(st), 0, y);
-            tma_load_2d(vdst, &tm_v, full_bar(st), 0, y);
-            if (y1 >= 0) {
-              tma_load_2d(kdst + L::kKVTileBytes / 2, &tm_k, full_bar(st), 0, y1);
-              tma_load_2d(vdst + L::kKVTileBytes / 2, &tm_v, full_bar(st), 0, y1);
+      for (int jj0 = 0; jj0 < nblk; jj0 += kIssueLanes) {
+        const int jj = jj0 + lane;
+        const int nn = n + jj;
+        const int st = nn % STAGES;
+        const bool mine = jj < nblk;
+        bool r = true;
+        if (mine) {
+          const int y = meta[ms].y0[jj];
+          r = mbar_wait(empty_bar(st), ((nn / STAGES) & 1) ^ 1, kWhereWaitEmpty, abort_flag);
+          if (r && nn != lost) {
+            const uint32_t kdst = sbase + st * L::kStageBytes;
+            const uint32_t vdst = kdst + L::kKVTileBytes;
+            if constexpr (KV8) {
+              // one box of D bytes x 16 rows, or of 8 rows twice with 8-token blocks
+              if (s.block_size >= kBlock) {
+                mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
+                tma_load_2d(kdst, &tm_k, full_bar(st), 0, y);
+                tma_load_2d(vdst, &tm_v, full_bar(st), 0, y);
+              } else {
+                const int y1 = meta[ms].y1[jj];
+                mbar_arrive_expect_tx(full_bar(st),
+                                      y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
+                tma_load_2d(kdst, &tm_k, full_bar(st), 0, y);
+                tma_load_2d(vdst, &tm_v, full_bar(st), 0, y);
+                if (y1 >= 0) {
+                  tma_load_2d(kdst + L::kKVTileBytes / 2, &tm_k, full_bar(st), 0, y1);
+                  tma_load_2d(vdst + L::kKVTileBytes / 2, &tm_v, full_bar(st), 0, y1);
+                }
+              }
+            } else if (s.block_size >= kBlock) {
+              // the maps view the cache as (64 dims, 8 rows, half, row group): one
+              // box of 2 row groups is the whole tile
+              mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
+              tma_load_4d(kdst, &tm_k, full_bar(st), 0, 0, 0, y >> 3);
+              tma_load_4d(vdst, &tm_v, full_bar(st), 0, 0, 0, y >> 3);
+            } else {  // 8-token blocks: one row group per block, the second if present
+              const int y1 = meta[ms].y1[jj];
+              mbar_arrive_expect_tx(full_bar(st), y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
+              tma_load_4d(kdst, &tm_k, full_bar(st), 0, 0, 0, y >> 3);
+              tma_load_4d(vdst, &tm_v, full_bar(st), 0, 0, 0, y >> 3);
+              if (y1 >= 0) {
+                tma_load_4d(kdst + L::kGroupBytes, &tm_k, full_bar(st), 0, 0, 0, y1 >> 3);
+                tma_load_4d(vdst + L::kGroupBytes, &tm_v, full_bar(st), 0, 0, 0, y1 >> 3);
+              }
             }
           }
-        } else if (s.block_size >= kBlock) {
-          // the maps view the cache as (64 dims, 8 rows, half, row group): one
-          // box of 2 row groups is the whole tile
-          mbar_arrive_expect_tx(full_bar(st), L::kStageBytes);
-          tma_load_4d(kdst, &tm_k, full_bar(st), 0, 0, 0, y >> 3);
-          tma_load_4d(vdst, &tm_v, full_bar(st), 0, 0, 0, y >> 3);
-        } else {  // 8-token blocks: one row group per block, the second if present
-          const int y1 = meta[ms].y1[jj];
-          mbar_arrive_expect_tx(full_bar(st), y1 >= 0 ? L::kStageBytes : L::kStageBytes / 2);
-          tma_load_4d(kdst, &tm_k, full_bar(st), 0, 0, 0, y >> 3);
-          tma_load_4d(vdst, &tm_v, full_bar(st), 0, 0, 0, y >> 3);
-          if (y1 >= 0) {
-            tma_load_4d(kdst + L::kGroupBytes, &tm_k, full_bar(st), 0, 0, 0, y1 >> 3);
-            tma_load_4d(vdst + L::kGroupBytes, &tm_v, full_bar(st), 0, 0, 0, y1 >> 3);
-          }
         }
+        ok = __all_sync(kIssueMask, r);
+        if (!ok) {
+          // another lane gave up: this lane's tile, if issued, lands before the
+          // CTA leaves (bounded again, independently of the abort flag)
+          if (mine && r && nn != lost) {
+            volatile int own_flag = 0;
+            mbar_wait(full_bar(st), (nn / STAGES) & 1, kWhereWaitFull, &own_flag);
+          }
+          break;
+        }
+        issued = n + min(jj0 + kIssueLanes, nblk);
       }
-      mbar_arrive(mempty_bar(ms));
+      if (!ok) break;
+      n += nblk;
+      __syncwarp(kIssueMask);  // both lanes are done with the slot's block rows
+      if (lane == 0) mbar_arrive(mempty_bar(ms));
     }
-    if (!ok) {
+    if (!ok && lane == 0) {
       // A wait gave up: let the loads already issued land before leaving
       // (each wait bounded again, independently of the CTA's abort flag).
       volatile int drain_flag = 0;
