@@ -356,10 +356,12 @@ pa_status launch_mma(const AttnArgs& a, const Plan& p, const pa::Work& w) {
   }
   // FP8 stages are half as large: at head_dim 128 twice as many keep the same
   // bytes in flight; at 64 the per-warp f16 staging tiles take that room.  The
-  // NARROW form runs four CTAs per SM of three consumer warps and 6 stages:
-  // its throughput follows the number of CTAs (each with its own TMA thread).
+  // NARROW form runs four CTAs per SM of three consumer warps and 9 stages
+  // (three per warp; its 8-row query slots leave the room for them): its
+  // throughput follows the number of CTAs (each with its own TMA thread) and
+  // the tiles each warp has in flight.
   constexpr int kN = NARROW ? 3 : kNcw;
-  constexpr int kS = NARROW ? 6 : (KV8 && D == 128 ? 2 * kStages : kStages);
+  constexpr int kS = NARROW ? 9 : (KV8 && D == 128 ? 2 * kStages : kStages);
   using L = pa::MmaLayout<D, kN, kS, KV8, NARROW>;
   auto kern = pa::attn_mma_kernel<T, D, kN, kS, KV8, NARROW>;
   int occ = 0;

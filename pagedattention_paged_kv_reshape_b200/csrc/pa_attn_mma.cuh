@@ -60,7 +60,9 @@ struct MmaLayout {
   static constexpr int kGroupBytes = kHalves * 8 * 128;
   static constexpr int kKVTileBytes = KV8 ? kBlock * D : kTileBytes;  // ... as loaded
   static constexpr int kStageBytes = 2 * kKVTileBytes;  // K tile then V tile
-  static constexpr int kQSlotBytes = kHalves * kRows * 128;
+  // a query tile of at most 8 rows in the NARROW form, else 16: [half][rows][128 B]
+  static constexpr int kQRows = NARROW ? 8 : kRows;
+  static constexpr int kQSlotBytes = kHalves * kQRows * 128;
   static constexpr int kQSlots = 2;
   static constexpr int kOffQ = STAGES * kStageBytes;
   static constexpr int kOffCo = kOffQ + kQSlots * kQSlotBytes;
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 4 : (D > 128 ? 1 : 2)
         const uint32_t qdst = sbase + L::kOffQ + qs * L::kQSlotBytes;
 #pragma unroll
         for (int h = 0; h < L::kHalves; ++h)
-          tma_load_3d(qdst + h * (kRows * 128), &tm_q, qfull_bar(qs), h * 64, un.head0,
+          tma_load_3d(qdst + h * (L::kQRows * 128), &tm_q, qfull_bar(qs), h * 64, un.head0,
                       un.token0);
       }
       const int nblk = ceil_div(un.kv_end - un.kv_begin, kBlock);
@@ -465,10 +467,15 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 4 : (D > 128 ? 1 : 2)
 #pragma unroll
       for (int G = 0; G < D / 64; ++G) {
         uint32_t a0[4], a1[4], b0[4], b1[4];  // rows g, g+8; dims 16q4 .. +7, +8 .. +15
-        lds128(qb + G * (kRows * 128) + swz(g, 2 * q4), a0);
-        lds128(qb + G * (kRows * 128) + swz(g, 2 * q4 + 1), a1);
-        lds128(qb + G * (kRows * 128) + swz(g + 8, 2 * q4), b0);
-        lds128(qb + G * (kRows * 128) + swz(g + 8, 2 * q4 + 1), b1);
+        lds128(qb + G * (L::kQRows * 128) + swz(g, 2 * q4), a0);
+        lds128(qb + G * (L::kQRows * 128) + swz(g, 2 * q4 + 1), a1);
+        if constexpr (NARROW) {  // the slot holds rows 0-7 only; rows 8-15 are padding
+#pragma unroll
+          for (int e = 0; e < 4; ++e) b0[e] = b1[e] = 0u;
+        } else {
+          lds128(qb + G * (L::kQRows * 128) + swz(g + 8, 2 * q4), b0);
+          lds128(qb + G * (L::kQRows * 128) + swz(g + 8, 2 * q4 + 1), b1);
+        }
 #pragma unroll
         for (int st2 = 0; st2 < 2; ++st2) {
           const uint32_t* ra = st2 ? a1 : a0;
@@ -490,7 +497,7 @@ __global__ void __launch_bounds__((NCW + 2) * 32, NARROW ? 4 : (D > 128 ? 1 : 2)
 #pragma unroll
       for (int kk = 0; kk < KSTEPS; ++kk) {
         const int ch = (kk & 3) * 2 + (mi >> 1);
-        ldsm_x4(qb + (kk >> 2) * (kRows * 128) + swz(r, ch), qa[kk][0], qa[kk][1], qa[kk][2],
+        ldsm_x4(qb + (kk >> 2) * (L::kQRows * 128) + swz(r, ch), qa[kk][0], qa[kk][1], qa[kk][2],
                 qa[kk][3]);
       }
     }
