@@ -81,16 +81,21 @@ struct Tc2Layout {
   static constexpr int kBarPFull = kBarSFull + 2;           // [2] P written (four warps)
   static constexpr int kBarPDone = kBarPFull + 2;           // [2] the P.V that read P done
   static constexpr int kBarDrain = kBarPDone + 2;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kStepSlots = 4;                      // MMA step ring (warp 3 -> warp 1)
+  static constexpr int kBarStepFull = kBarDrain + 1;        // [kStepSlots]
+  static constexpr int kBarStepFree = kBarStepFull + kStepSlots;  // [kStepSlots]
+  static constexpr int kNumBars = kBarStepFree + kStepSlots;
   static constexpr int kOffItems = kOffBar + kNumBars * 8;
   static constexpr int kItemBytes = 64;
   static constexpr int kItemSlots = 8;
-  static constexpr int kOffTmem = kOffItems + kItemSlots * kItemBytes;
+  static constexpr int kOffSteps = kOffItems + kItemSlots * kItemBytes;
+  static constexpr int kStepBytes = 32;
+  static constexpr int kOffTmem = kOffSteps + kStepSlots * kStepBytes;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 12;
   static constexpr int kSmem = kBytes + 1024;               // slack to align the base to 1 KB
-  // warps 0: K/V loads, 1: MMA issue, 2: Q loads, 3: idle, 4-7: softmax of
-  // tile A, 8-11: softmax of tile B
+  // warps 0: K/V loads, 1: MMA issue, 2: Q loads, 3: MMA step preparation,
+  // 4-7: softmax of tile A, 8-11: softmax of tile B
   static constexpr int kThreads = 384;
   // Registers per thread after the split (setmaxnreg): the 128 threads of
   // warps 0-3 give up what the 256 softmax threads take.  Launched with 168
@@ -116,6 +121,18 @@ struct Tc2Item {
   int kv_end;      // ... tile B's (>= kv_end_a): the item's key range
   int nkt_a, nkt;  // 128-key tiles tile A reads, and the item reads
 };
+
+// One step of the MMA issue (P.V of one key tile and S of the next, for both
+// query tiles), as warp 3 prepares it for the issuing thread: the checks that
+// the step's operands have landed are done, and every stage index and count
+// the MMAs need is here.
+struct Tc2Step {
+  int flags;            // kStep* bits
+  int vs, ks;           // V stage of the P.V tile, K stage of the S tile
+  int steps_a, steps_b; // 16-key P.V steps holding keys visible to tile A / B
+};
+constexpr int kStepPvA = 1, kStepPvB = 2, kStepSA = 4, kStepSB = 8, kStepQFreeA = 16,
+              kStepQFreeB = 32, kStepAcc = 64, kStepEnd = 128;
 
 // The item `idx` of the chunk list (idx = entry + count * head unit).  Every
 // warp role computes it itself from the list and the row metadata.
@@ -357,18 +374,16 @@ __global__ void __launch_bounds__(384, 1)
           mbar_wait(qfull(1), q_last & 1, kWhereWaitQ, &own_flag);
         }
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issue
-      // One thread.  Two cursors walk the CTA's (item, key tile) sequence, the S
-      // cursor one tile ahead of the P.V cursor.  Per step: P.V_A(cp), S_A(cs),
-      // P.V_B(cp), S_B(cs).  S_x(cs) overwrites the columns P.V_x(cp) reads P
-      // from; it is issued after that P.V, and the tensor core executes them in
-      // order.  The step's V tile (and its padding rows) and K tile are waited
-      // for before its first P: they arrive well ahead of it, and once a P is
-      // written only the issue of its MMAs stands between it and the tensor
-      // core.  (The other lanes go straight to the teardown barrier: this warp
-      // shares its SM sub-partition with two softmax warps, and every
-      // instruction it saves shortens the tensor core's idle gaps.)
+    } else if (warp == 3) {
+      // ---------------------------------------------------- MMA step preparation
+      // One thread walks the CTA's (item, key tile) sequence with two cursors,
+      // the S cursor one tile ahead of the P.V cursor, waits until each step's
+      // V and K tiles (and a new item's Q tiles) have landed, zeroes the V rows
+      // of an item's last 16-key step past its last key (padding slots, or rows
+      // no box covered; 0 * NaN is NaN), and hands the step to the issuing
+      // thread through a ring of shared-memory slots.  The issuing thread then
+      // only waits for P and issues: the tensor core accepts only a few MMAs
+      // ahead, so bookkeeping in the issuing thread itself would leave it idle.
       if (lane == 0) {
         struct Cursor {
           int k, t, nkt, nkt_a, kv_end_a, kv_end;
@@ -398,44 +413,18 @@ __global__ void __launch_bounds__(384, 1)
           ++c.k;
           return true;
         };
-        // S_x of the S cursor's tile (its K tile, and for x = 1 its Q_B, waited for)
-        auto issue_s = [&](const Cursor& c, int x) {
-          // (no tcgen05 fence here: the softmax threads' last reads of S_x were
-          // ordered before this thread's tcgen05 operations by the fence after
-          // its wait on their P, earlier in this thread's program order)
-          const uint64_t qd = smem_desc_sw128(q_smem(x), 16, 1024);
-          const uint64_t kd = smem_desc_sw128(k_smem(c.ks), 16, L::kGroupBytes);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // descriptor start addresses advance in 16-byte units
-            const uint64_t qoff = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
-            const uint64_t koff = ((kk >> 2) * 1024 + (kk & 3) * 32) >> 4;
-            umma_ss(t_s(x), qd + qoff, kd + koff, kIdescS, kk > 0);
-          }
-          umma_commit(sfull(x));
-          if (c.t == (x == 0 ? c.nkt_a : c.nkt) - 1) umma_commit(qfree(x));
-          if (x == 1) umma_commit(kempty(c.ks));  // both tiles' S of this K tile issued
-        };
-        // P.V_x of the P.V cursor's tile, once P_x is written (its V tile waited for)
-        auto issue_pv = [&](const Cursor& c, int x, int nx) -> bool {
-          // operands first: only the MMAs themselves wait for P
-          const int valid = min(kTcKeys, (x == 0 ? c.kv_end_a : c.kv_end) - c.t * kTcKeys);
-          const int steps = (valid + 15) >> 4;  // 16-key MMA steps holding visible keys
-          const uint64_t vd = smem_desc_sw128(v_smem(c.vs), 1024, L::kGroupBytes);
-          const uint32_t acc0 = c.t > 0 ? 1u : 0u;  // the item's first tile starts O afresh
-          if (!mbar_wait(pfull(x), nx & 1, kWhereWaitMma, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kTcKeys / 16; ++kk)
-            umma_ts(t_o(x), t_s(x) + kk * 8, vd + ((kk * 2 * L::kGroupBytes) >> 4), kIdescPV,
-                    kk > 0 ? 1u : acc0, kk < steps);
-          umma_commit(pdone(x));
-          if (x == 1) umma_commit(vempty(c.vs));  // both tiles' P.V of this V tile issued
+        int j = 0;  // steps handed over
+        auto emit = [&](const Tc2Step& st) -> bool {
+          const int slot = j % L::kStepSlots;
+          if (!mbar_wait(bar(L::kBarStepFree + slot), ((j / L::kStepSlots) & 1) ^ 1,
+                         kWhereWaitMma, abort_flag))
+            return false;
+          *reinterpret_cast<Tc2Step*>(smem + L::kOffSteps + slot * L::kStepBytes) = st;
+          mbar_arrive(bar(L::kBarStepFull + slot));
+          ++j;
           return true;
         };
-        // The step's V tile has landed; for the item's last tile, zero the rows
-        // of its last 16-key step past the item's last key (padding slots, or
-        // rows no box covered) before any P.V reads them.
+        // the P.V tile's V has landed, its padding rows zeroed
         auto v_ready = [&](const Cursor& c) -> bool {
           if (!mbar_wait(vfull(c.vs), c.vph, kWhereWaitFull, abort_flag)) return false;
           if (c.t == c.nkt - 1) {
@@ -455,38 +444,121 @@ __global__ void __launch_bounds__(384, 1)
           }
           return true;
         };
+        auto s_flags = [&](const Cursor& c) {
+          int f = kStepSB;
+          if (c.t < c.nkt_a) f |= kStepSA;
+          if (c.t == c.nkt_a - 1) f |= kStepQFreeA;
+          if (c.t == c.nkt - 1) f |= kStepQFreeB;
+          return f;
+        };
         Cursor cs{}, cp{};
-        int na = 0, nb = 0;  // P.V issued so far for tile A and tile B
-        bool ok = my_items > 0 && load_item(cs, true);
-        if (ok) {  // S of the first tile
-          ok = mbar_wait(kfull(cs.ks), cs.kph, kWhereWaitFull, abort_flag) &&
-               mbar_wait(qfull(1), 0, kWhereWaitQ, abort_flag);
-          if (ok) {
-            issue_s(cs, 0);
-            issue_s(cs, 1);
-          }
+        bool ok = true;
+        if (my_items > 0) {  // S of the first tile
+          ok = load_item(cs, true) &&
+               mbar_wait(kfull(cs.ks), cs.kph, kWhereWaitFull, abort_flag) &&
+               mbar_wait(qfull(1), 0, kWhereWaitQ, abort_flag) &&
+               emit(Tc2Step{s_flags(cs), 0, cs.ks, 0, 0});
+          if (ok && advance(cs)) ok = load_item(cs, true);
+          if (ok) ok = load_item(cp, false);  // the S cursor has waited for item 0's Q
         }
-        if (ok && advance(cs)) ok = load_item(cs, true);
-        if (ok) ok = load_item(cp, false);  // the S cursor has waited for item 0's Q
         while (ok && cp.k < my_items) {
-          const bool has_a = cp.t < cp.nkt_a;
           const bool s_next = cs.k < my_items;
           ok = v_ready(cp) &&
                (!s_next || mbar_wait(kfull(cs.ks), cs.kph, kWhereWaitFull, abort_flag));
-          if (ok && has_a) ok = issue_pv(cp, 0, na);
           if (!ok) break;
-          na += has_a;
-          if (s_next && cs.t < cs.nkt_a) issue_s(cs, 0);
-          ok = issue_pv(cp, 1, nb);
-          if (!ok) break;
-          ++nb;
-          if (s_next) {  // tile B's Q of a new item
-            if (cs.t == 0) ok = mbar_wait(qfull(1), cs.k & 1, kWhereWaitQ, abort_flag);
-            if (!ok) break;
-            issue_s(cs, 1);
+          Tc2Step st;
+          st.flags = kStepPvB | (cp.t < cp.nkt_a ? kStepPvA : 0) | (cp.t > 0 ? kStepAcc : 0) |
+                     (s_next ? s_flags(cs) : 0);
+          st.vs = cp.vs;
+          st.ks = cs.ks;
+          st.steps_a = (min(kTcKeys, cp.kv_end_a - cp.t * kTcKeys) + 15) >> 4;
+          st.steps_b = (min(kTcKeys, cp.kv_end - cp.t * kTcKeys) + 15) >> 4;
+          if (s_next && cs.t == 0) {
+            // S_B of a new item waits for its Q_B: hand over the rest of the
+            // step first, then S_B on its own
+            Tc2Step first = st;
+            first.flags &= ~(kStepSB | kStepQFreeB);
+            ok = emit(first) && mbar_wait(qfull(1), cs.k & 1, kWhereWaitQ, abort_flag) &&
+                 emit(Tc2Step{kStepSB | (st.flags & kStepQFreeB), st.vs, st.ks, 0, 0});
+          } else {
+            ok = emit(st);
           }
-          if (advance(cs)) ok = load_item(cs, true);
+          if (ok && advance(cs)) ok = load_item(cs, true);
           if (ok && advance(cp)) ok = load_item(cp, false);  // the S cursor is past it already
+        }
+        // the end of the CTA's steps (also when it has no items: the issuing
+        // thread waits for this)
+        if (ok) emit(Tc2Step{kStepEnd, 0, 0, 0, 0});
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issue
+      // One thread.  Per step, in this order: P.V_A(t), S_A(t+1), P.V_B(t),
+      // S_B(t+1) (steps prepared by warp 3).  S_x(t+1) overwrites the columns
+      // P.V_x(t) reads P from; it is issued after that P.V, and the tensor core
+      // executes them in order.  The P.V operands are computed before the wait
+      // for P, and the P.V MMAs past the last visible key are predicated off
+      // inside the instruction, not branched around.  (The other lanes go
+      // straight to the teardown barrier: this warp shares its SM
+      // sub-partition with two softmax warps.)
+      if (lane == 0) {
+        int na = 0, nb = 0;  // P.V issued so far for tile A and tile B
+        auto issue_s = [&](int x, int ks) {
+          // (no tcgen05 fence here: the softmax threads' last reads of S_x were
+          // ordered before this thread's tcgen05 operations by the fence after
+          // its wait on their P, earlier in this thread's program order)
+          const uint64_t qd = smem_desc_sw128(q_smem(x), 16, 1024);
+          const uint64_t kd = smem_desc_sw128(k_smem(ks), 16, L::kGroupBytes);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // descriptor start addresses advance in 16-byte units
+            const uint64_t qoff = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
+            const uint64_t koff = ((kk >> 2) * 1024 + (kk & 3) * 32) >> 4;
+            umma_ss(t_s(x), qd + qoff, kd + koff, kIdescS, kk > 0);
+          }
+          umma_commit(sfull(x));
+        };
+        auto issue_pv = [&](int x, int vs, int steps, uint32_t acc0, int nx) -> bool {
+          const uint64_t vd = smem_desc_sw128(v_smem(vs), 1024, L::kGroupBytes);
+          if (!mbar_wait(pfull(x), nx & 1, kWhereWaitMma, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTcKeys / 16; ++kk)
+            umma_ts(t_o(x), t_s(x) + kk * 8, vd + ((kk * 2 * L::kGroupBytes) >> 4), kIdescPV,
+                    kk > 0 ? 1u : acc0, kk < steps);
+          umma_commit(pdone(x));
+          return true;
+        };
+        bool ok = true;
+        for (int j = 0; ok; ++j) {
+          const int slot = j % L::kStepSlots;
+          if (!mbar_wait(bar(L::kBarStepFull + slot), (j / L::kStepSlots) & 1, kWhereWaitMma,
+                         abort_flag))
+            break;
+          const Tc2Step st = *reinterpret_cast<const Tc2Step*>(smem + L::kOffSteps +
+                                                               slot * L::kStepBytes);
+          mbar_arrive(bar(L::kBarStepFree + slot));
+          if (st.flags & kStepEnd) break;
+          const uint32_t acc0 = (st.flags & kStepAcc) ? 1u : 0u;
+          if (st.flags & kStepPvA) {
+            ok = issue_pv(0, st.vs, st.steps_a, acc0, na);
+            if (!ok) break;
+            ++na;
+          }
+          if (st.flags & kStepSA) {
+            issue_s(0, st.ks);
+            if (st.flags & kStepQFreeA) umma_commit(qfree(0));
+          }
+          if (st.flags & kStepPvB) {
+            ok = issue_pv(1, st.vs, st.steps_b, acc0, nb);
+            if (!ok) break;
+            ++nb;
+            umma_commit(vempty(st.vs));  // both tiles' P.V of this V tile issued
+          }
+          if (st.flags & kStepSB) {
+            issue_s(1, st.ks);
+            if (st.flags & kStepQFreeB) umma_commit(qfree(1));
+            umma_commit(kempty(st.ks));  // both tiles' S of this K tile issued
+          }
         }
         // no MMA of this CTA may still run when TMEM is freed
         umma_commit(drain);
