@@ -23,7 +23,9 @@
 //   read them has completed, so the K/V stream never waits for Q.
 // * one thread of warp 1 issues the MMAs in the order P.V_A(t), S_A(t+1),
 //   P.V_B(t), S_B(t+1), ...: while softmax A works on S_A the tensor core
-//   runs P.V_B and S_B, and the other way round.
+//   runs P.V_B and S_B, and the other way round.  One thread of warp 3 does
+//   the bookkeeping of those steps (cursors, checks that K, V and Q have
+//   landed, V padding rows) and hands each step over, ahead of time.
 // * warps 4-7 (tile A) and 8-11 (tile B): one thread per tile row (TMEM lane)
 //   reads the row's 128 scores, takes the masked maximum (key <= position),
 //   writes P rounded to the input type, and keeps the row sum of P.  The
