@@ -22,6 +22,9 @@
 //   order S(0), S(1), P.V(0), S(2), P.V(1), S(3), ...: S(g + 2) reuses the
 //   columns P.V(g) reads and follows it on the tensor core, so the tensor
 //   core computes the next S while the softmax works on the current one;
+//   one thread of warp 3 does the bookkeeping of those steps (cursors,
+//   checks that K, V and Q have landed, V padding rows) and hands each step
+//   over ahead of time;
 // * warps 4-7: one thread per tile row reads its 64 scores, takes the masked
 //   maximum, raises the reference maximum lazily (by more than 2^8 only; only
 //   then is O rescaled, after the previous P.V has completed), writes P
@@ -73,21 +76,37 @@ struct Tc1Layout {
   // phase, of the same parity, while P.V(g - 1) is still running.
   static constexpr int kBarPDone = kBarPFull + 2;
   static constexpr int kBarDrain = kBarPDone + 2;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kStepSlots = 4;                     // MMA step ring (warp 3 -> warp 1)
+  static constexpr int kBarStepFull = kBarDrain + 1;       // [kStepSlots]
+  static constexpr int kBarStepFree = kBarStepFull + kStepSlots;  // [kStepSlots]
+  static constexpr int kNumBars = kBarStepFree + kStepSlots;
   static constexpr int kOffItems = kOffBar + kNumBars * 8;
   static constexpr int kItemBytes = 64;
   static constexpr int kItemSlots = 8;
-  static constexpr int kOffTmem = kOffItems + kItemSlots * kItemBytes;
+  static constexpr int kOffSteps = kOffItems + kItemSlots * kItemBytes;
+  static constexpr int kStepBytes = 32;
+  static constexpr int kOffTmem = kOffSteps + kStepSlots * kStepBytes;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kBytes = kOffAbort + 12;
   static constexpr int kSmem = kBytes + 1024;  // slack to align the base to 1 KB
-  // warps 0: K/V loads, 1: MMA issue, 2: Q loads, 3: idle, 4-7: softmax
+  // warps 0: K/V loads, 1: MMA issue, 2: Q loads, 3: MMA step preparation,
+  // 4-7: softmax
   static constexpr int kThreads = 256;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffBar % 1024 == 0, "1 KB alignment");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
+
+// One MMA step of the one-tile form, as warp 3 prepares it for the issuing
+// thread: P.V of tile pv_g and S of tile s_g (two tiles ahead), their
+// operands checked to have landed.
+struct Tc1Step {
+  int flags;        // kStep1* bits
+  int pv_g, vs, steps;
+  int s_g, ks;
+};
+constexpr int kStep1Pv = 1, kStep1S = 2, kStep1QFree = 4, kStep1Acc = 8, kStep1End = 16;
 
 // One work item of the one-tile form.
 struct Tc1Item {
@@ -292,10 +311,14 @@ __global__ void __launch_bounds__(256, 1)
         mbar_wait(qfull, q_last & 1, kWhereWaitQ, &own_flag);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issue
-    // One thread.  Tile g of the CTA's sequence: S(g) into S(g % 2) (after
-    // P.V(g - 2), which read that buffer's P), P.V(g) once its P is written.
+  } else if (warp == 3) {
+    // ---------------------------------------------------- MMA step preparation
+    // One thread walks the CTA's tiles with two cursors, the S cursor two
+    // tiles ahead of the P.V cursor, waits until each step's V and K tiles
+    // (and a new item's Q) have landed, zeroes the V rows of an item's last
+    // 16-key step past its last key (padding slots, or rows no box covered),
+    // and hands the step to the issuing thread through a ring of shared-memory
+    // slots, so that the issuing thread only waits for P and issues.
     if (lane == 0) {
       struct Cursor {
         int k, t, g, nkt, kv_end;
@@ -315,36 +338,43 @@ __global__ void __launch_bounds__(256, 1)
         ++c.k;
         return true;
       };
-      auto issue_s = [&](const Cursor& c) -> bool {
-        const int ks = c.g % KS;
-        if (!mbar_wait(kfull(ks), (c.g / KS) & 1, kWhereWaitFull, abort_flag)) return false;
-        const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024);
-        const uint64_t kd = smem_desc_sw128(k_smem(ks), 16, L::kGroupBytes);
-        const uint32_t ts = t_s(c.g & 1);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // descriptor start addresses advance in 16-byte units
-          const uint64_t qoff = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
-          const uint64_t koff = ((kk >> 2) * 1024 + (kk & 3) * 32) >> 4;
-          umma_ss(ts, qd + qoff, kd + koff, kIdescS, kk > 0);
-        }
-        umma_commit(sfull(c.g & 1));
-        umma_commit(kempty(ks));
-        if (c.t == c.nkt - 1) umma_commit(qfree);  // the item's last S: Q may be replaced
+      int j = 0;  // steps handed over
+      auto emit = [&](const Tc1Step& st) -> bool {
+        const int slot = j % L::kStepSlots;
+        if (!mbar_wait(bar(L::kBarStepFree + slot), ((j / L::kStepSlots) & 1) ^ 1, kWhereWaitMma,
+                       abort_flag))
+          return false;
+        *reinterpret_cast<Tc1Step*>(smem + L::kOffSteps + slot * L::kStepBytes) = st;
+        mbar_arrive(bar(L::kBarStepFull + slot));
+        ++j;
         return true;
       };
-      auto issue_pv = [&](const Cursor& c) -> bool {
-        const int vs = c.g % VS;
-        const int key0 = c.t * kTc1Keys;
-        const int valid = min(kTc1Keys, c.kv_end - key0);
-        const int steps = (valid + 15) >> 4;  // 16-key MMA steps holding visible keys
-        const uint64_t vd = smem_desc_sw128(v_smem(vs), 1024, L::kGroupBytes);
-        const uint32_t acc0 = c.t > 0 ? 1u : 0u;  // the item's first tile starts O afresh
-        const uint32_t ts = t_s(c.g & 1);
-        if (!mbar_wait(vfull(vs), (c.g / VS) & 1, kWhereWaitFull, abort_flag)) return false;
-        if (c.t == c.nkt - 1) {
-          // the item's last V tile: zero the rows of its last 16-key step past
-          // the item's last key (padding slots, or rows no box covered)
+      // S of the S cursor's tile: its K tile landed
+      auto s_part = [&](const Cursor& c, Tc1Step& st) -> bool {
+        const int ks = c.g % KS;
+        if (!mbar_wait(kfull(ks), (c.g / KS) & 1, kWhereWaitFull, abort_flag)) return false;
+        st.flags |= kStep1S | (c.t == c.nkt - 1 ? kStep1QFree : 0);  // the item's last S
+        st.s_g = c.g;
+        st.ks = ks;
+        return true;
+      };
+      Cursor cs{}, cp{};  // the S cursor runs two tiles ahead of the P.V cursor
+      bool ok = true;
+      if (my_items > 0) {
+        ok = load_item(cs, true);
+        for (int i = 0; i < 2 && ok && cs.k < my_items; ++i) {
+          Tc1Step st{0, 0, 0, 0, 0, 0};
+          ok = s_part(cs, st) && emit(st);
+          if (ok && advance(cs)) ok = load_item(cs, true);
+        }
+        if (ok) ok = load_item(cp, false);  // the S cursor has waited for item 0's Q
+      }
+      while (ok && cp.k < my_items) {
+        const int vs = cp.g % VS;
+        const int valid = min(kTc1Keys, cp.kv_end - cp.t * kTc1Keys);
+        ok = mbar_wait(vfull(vs), (cp.g / VS) & 1, kWhereWaitFull, abort_flag);
+        if (!ok) break;
+        if (cp.t == cp.nkt - 1) {
           const int pad1 = min(kTc1Keys, (valid + 15) & ~15);
           for (int row = valid; row < pad1; ++row) {
             uint8_t* dst = smem + L::kOffV + vs * L::kKVBytes + (row >> 3) * L::kGroupBytes +
@@ -357,30 +387,66 @@ __global__ void __launch_bounds__(256, 1)
           }
           fence_proxy_async_smem();
         }
-        if (!mbar_wait(pfull(c.g & 1), (c.g >> 1) & 1, kWhereWaitMma, abort_flag)) return false;
+        Tc1Step st{kStep1Pv | (cp.t > 0 ? kStep1Acc : 0), cp.g, vs, (valid + 15) >> 4, 0, 0};
+        const bool s_next = cs.k < my_items;
+        if (s_next) ok = s_part(cs, st);
+        if (ok) ok = emit(st);
+        if (ok && s_next && advance(cs)) ok = load_item(cs, true);
+        if (ok && advance(cp)) ok = load_item(cp, false);  // the S cursor is past it already
+      }
+      // the end of the CTA's steps (also when it has no items: the issuing
+      // thread waits for this)
+      if (ok) emit(Tc1Step{kStep1End, 0, 0, 0, 0, 0});
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    // One thread.  Tile g of the CTA's sequence: S(g) into S(g % 2) (after
+    // P.V(g - 2), which read that buffer's P), P.V(g) once its P is written;
+    // per step P.V(g) then S(g + 2), as warp 3 hands them over.
+    if (lane == 0) {
+      auto issue_s = [&](int g, int ks) {
+        const uint64_t qd = smem_desc_sw128(q_smem, 16, 1024);
+        const uint64_t kd = smem_desc_sw128(k_smem(ks), 16, L::kGroupBytes);
+        const uint32_t ts = t_s(g & 1);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // descriptor start addresses advance in 16-byte units
+          const uint64_t qoff = ((kk >> 2) * L::kHalfBytes + (kk & 3) * 32) >> 4;
+          const uint64_t koff = ((kk >> 2) * 1024 + (kk & 3) * 32) >> 4;
+          umma_ss(ts, qd + qoff, kd + koff, kIdescS, kk > 0);
+        }
+        umma_commit(sfull(g & 1));
+        umma_commit(kempty(ks));
+      };
+      auto issue_pv = [&](int g, int vs, int steps, uint32_t acc0) -> bool {
+        const uint64_t vd = smem_desc_sw128(v_smem(vs), 1024, L::kGroupBytes);
+        const uint32_t ts = t_s(g & 1);
+        if (!mbar_wait(pfull(g & 1), (g >> 1) & 1, kWhereWaitMma, abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTc1Keys / 16; ++kk)
           umma_ts(t_o, ts + kk * 8, vd + ((kk * 2 * L::kGroupBytes) >> 4), kIdescPV,
                   kk > 0 ? 1u : acc0, kk < steps);
-        umma_commit(pdone(c.g & 1));
+        umma_commit(pdone(g & 1));
         umma_commit(vempty(vs));
         return true;
       };
-      Cursor cs{}, cp{};  // the S cursor runs two tiles ahead of the P.V cursor
-      bool ok = my_items > 0 && load_item(cs, true);
-      for (int i = 0; i < 2 && ok && cs.k < my_items; ++i) {
-        ok = issue_s(cs);
-        if (ok && advance(cs)) ok = load_item(cs, true);
-      }
-      if (ok) ok = load_item(cp, false);  // the S cursor has waited for item 0's Q
-      while (ok && cp.k < my_items) {
-        ok = issue_pv(cp);
-        if (ok && cs.k < my_items) {
-          ok = issue_s(cs);
-          if (ok && advance(cs)) ok = load_item(cs, true);
+      for (int j = 0;; ++j) {
+        const int slot = j % L::kStepSlots;
+        if (!mbar_wait(bar(L::kBarStepFull + slot), (j / L::kStepSlots) & 1, kWhereWaitMma,
+                       abort_flag))
+          break;
+        const Tc1Step st =
+            *reinterpret_cast<const Tc1Step*>(smem + L::kOffSteps + slot * L::kStepBytes);
+        mbar_arrive(bar(L::kBarStepFree + slot));
+        if (st.flags & kStep1End) break;
+        if ((st.flags & kStep1Pv) &&
+            !issue_pv(st.pv_g, st.vs, st.steps, (st.flags & kStep1Acc) ? 1u : 0u))
+          break;
+        if (st.flags & kStep1S) {
+          issue_s(st.s_g, st.ks);
+          if (st.flags & kStep1QFree) umma_commit(qfree);  // the item's last S: Q may be replaced
         }
-        if (ok && advance(cp)) ok = load_item(cp, false);  // the S cursor is past it already
       }
       // no MMA of this CTA may still run when TMEM is freed
       umma_commit(drain);
